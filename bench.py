@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 MoE layer with zero-computation experts.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+One step is one forward of the whole layer (router GEMM, routing, dispatch,
+gate/up and down expert GEMMs, combine) over one batch of T synthetic tokens,
+through the C ABI (moe_zc_forward).  The default workload is the
+LongCat-Flash-shaped prefill layer (T=16384, d=6144, N=512 SwiGLU experts with
+I=2048, Z=256 zero experts, K=12, ~30% zero-expert picks); --workload picks
+another (tiny, small, decode, skewed20/40/60).
+
+Timing: W untimed warm-up steps, then K steps between CUDA events on the
+launching stream, with a barrier and a device synchronize on both sides; the
+max over ranks is taken.  The expert weights the batch touches (several GB at
+prefill) are far larger than the 126 MB L2, so no L2 flush is done between
+steps.  With N > 1 GPUs each rank runs its own batch of T tokens against its
+own weight replica (tokens are independent: no collective in the step), so
+`value` is N*T*K / max-rank time ("weak" scaling).
+
+The JSON line also carries: `e2e` (the same metric with the step's input
+copied from pinned host memory and its output copied back inside the timed
+region), `roofline` (the dominant kernel's achieved rate against the measured
+peak in MEASURED_PEAKS.json, from per-stage CUDA events recorded during the
+timed steps), `cpu_baseline` (the fp64 CPU oracle, as it stands, timed on the
+host cores on a bounded token sample; rank 0, N=1 only), `clocks` (SM clocks
+and throttle reasons sampled during the timed region) and `gpu_launches`.
+
+--impl reference times the fp64 CPU oracle itself on the host cores (each
+step a bounded token sample of the same workload) and prints the same line
+with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mixture_experts_layer_28_b200 import workloads as wl  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; executed-FFN TFLOPS as % of B200 bf16 peak (HBM % at decode)"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 2 ** 20
+KERNELS_PER_FORWARD = 8   # router_gemm, route, scan, assign, permute, gateup, down, combine
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel
+# from an ncu capture of the current kernel build, per workload (None = not
+# captured for this build).
+NCU_TRAFFIC_BYTES = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"],
+                    bf16_sus=p["bf16_tflops_sustained"], src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ----------------------------------------------------------------- distributed
+class Dist:
+    def __init__(self, n_gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world != n_gpus:
+            raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={self.world}: launch N>1 with torchrun")
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+        elif torch.cuda.is_available():
+            torch.cuda.set_device(0)
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.5)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- inputs
+def make_inputs(w: wl.Workload):
+    ri = wl.routing_inputs(w)
+    b = ri.bias(w.N, w.delta)
+    ew = wl.expert_weights(w, "cuda")
+    dev = dict(x=ri.x.cuda(), W_r=ri.W_r.cuda(), b=b.cuda(),
+               off=None if ri.logit_offset is None else ri.logit_offset.cuda())
+    return ri, b, ew, dev
+
+
+def routing_stats(w, cnt):
+    ffn = cnt[: w.N].astype(np.int64)
+    P = int(ffn.sum())
+    hit = int((ffn > 0).sum())
+    return dict(ffn_pairs=P, experts_hit=hit, zero_pick_fraction=1.0 - P / float(w.T * w.K),
+                max_load=int(ffn.max()) if w.N else 0)
+
+
+def roofline_numbers(w, st, pk):
+    """Algorithmic FLOPs and bytes of the layer and of its kernels."""
+    P, hit = st["ffn_pairs"], st["experts_hit"]
+    d, I, T, E = w.d, w.I, w.T, w.E
+    F_gateup = 4.0 * d * I * P
+    F_down = 2.0 * d * I * P
+    B_gateup = hit * 2.0 * I * d * 2 + P * d * 2 + P * I * 2      # weights + Xp in + H out
+    B_down = hit * 1.0 * I * d * 2 + P * I * 2 + P * d * 2        # weights + H in + Y out
+    F_layer = F_gateup + F_down
+    B_layer = hit * 3.0 * d * I * 2 + E * d * 2 + E * 4 + 2.0 * T * d * 2
+    return dict(F_gateup=F_gateup, F_down=F_down, B_gateup=B_gateup, B_down=B_down,
+                F_layer=F_layer, B_layer=B_layer)
+
+
+# ----------------------------------------------------------------- oracle timing
+def oracle_sample_time(w, ri, b, ew, n_tokens, seed_offset=0):
+    """Seconds the fp64 oracle takes for the forward of n sampled tokens.
+
+    The weights of the experts those tokens pick are copied to host memory
+    (bf16) before timing; widening them to fp64 is part of the oracle's work.
+    """
+    from oracle import moe_zc_ref as ref
+    rows = wl.tokens_sample(w.T, n_tokens, w.seed + seed_offset)
+    xs = ri.x[rows]
+    r = ref.route(xs, ri.W_r, b, w.N, w.K, ri.logit_offset)
+    hit = np.unique(r.idx[r.idx < w.N])
+    host = {int(e): (ew.W_gate[e].cpu(), ew.W_up[e].cpu(), ew.W_down[e].cpu()) for e in hit}
+    t0 = time.perf_counter()
+    r = ref.route(xs, ri.W_r, b, w.N, w.K, ri.logit_offset)
+    ref.forward_rows(xs, r, lambda e: host[e])
+    return time.perf_counter() - t0, len(rows)
+
+
+def cpu_baseline(w, ri, b, ew, budget_s=15.0):
+    cores = len(os.sched_getaffinity(0))
+    n = min(w.T, 8)
+    dt, n = oracle_sample_time(w, ri, b, ew, n, 1)
+    if dt < budget_s / 4 and n < w.T:
+        n = int(min(w.T, max(n, n * budget_s / max(dt, 1e-3) / 2)))
+        dt, n = oracle_sample_time(w, ri, b, ew, n, 2)
+    return {"value": n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {w.T} tokens (seeded sample), fp64 NumPy oracle, {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------- arms
+def config_of(w, extra=None):
+    c = {"workload": w.name, "T": w.T, "d": w.d, "N": w.N, "Z": w.Z, "K": w.K, "I": w.I,
+         "target_zero_frac": w.zero_frac, "zipf_s": w.zipf_s, "seed": w.seed}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def run_ours(args, dist, w):
+    from mixture_experts_layer_28_b200 import moe_zc as mz
+    pk = peaks()
+    ri, b, ew, dev = make_inputs(w)
+    out = torch.empty_like(dev["x"])
+    stream = torch.cuda.current_stream()
+    mz.reserve(w.T, w.d, w.N, w.Z, w.K, w.I)
+
+    def step(x=None, o=None):
+        mz.forward(dev["x"] if x is None else x, dev["W_r"], dev["b"], ew.W_gate, ew.W_up,
+                   ew.W_down, w.N, w.Z, w.K, out=out if o is None else o,
+                   logit_offset=dev["off"], stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    mz.synchronize()
+    st = routing_stats(w, mz.expert_load(w.E))
+    rf = roofline_numbers(w, st, pk)
+
+    # ---- device-resident timed region
+    clocks = ClockSampler(dist.local) if dist.rank == 0 else None
+    if clocks:
+        clocks.start()
+    mz.profile(True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    stage_ms, nfw = mz.profile_read()
+    mz.profile(False)
+    clk = clocks.stop() if clocks else None
+    mz.synchronize()
+    ms_max = dist.max(ms)
+    value = dist.world * w.T / (ms_max / 1e3)
+
+    # ---- end to end: pinned host input -> device -> forward -> host output
+    x_host = ri.x.pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    x_dev = torch.empty_like(dev["x"])
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e2e_ms = dist.max(e0.elapsed_time(e1) / args.e2e_steps)
+    mz.synchronize()
+
+    # ---- roofline of the dominant kernel (largest share of the step)
+    per = {k: v / max(nfw, 1) for k, v in stage_ms.items()}
+    dom = max(per, key=per.get)
+    kern = {"gateup_gemm": (rf["F_gateup"], rf["B_gateup"]),
+            "down_gemm": (rf["F_down"], rf["B_down"])}.get(dom)
+    roof = None
+    if kern and per[dom] > 0:
+        F, B = kern
+        sec = per[dom] / 1e3
+        t_tensor, t_hbm = F / (pk["bf16_sus"] * 1e12), B / (pk["hbm"] * 1e9)
+        if t_tensor >= t_hbm:
+            ach = F / sec / 1e12
+            roof = {"bound": "tensor", "achieved": ach, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
+                    "frac": ach / pk["bf16_sus"],
+                    "peak_kind": f"bf16 dense, sustained ({pk['src']}, MEASURED_PEAKS.json)"}
+        else:
+            ach = B / sec / 1e9
+            roof = {"bound": "hbm", "achieved": ach, "peak": pk["hbm"], "unit": "GB/s",
+                    "frac": ach / pk["hbm"], "peak_kind": f"HBM copy ({pk['src']})"}
+        roof["kernel"] = dom
+        roof["ms_per_launch"] = per[dom]
+        tr = NCU_TRAFFIC_BYTES.get(w.name)
+        roof["traffic"] = tr
+
+    # whole-layer roofline: slower of executed FFN FLOPs at tensor peak and
+    # touched bytes at HBM peak, against the measured step time
+    t_bound = max(rf["F_layer"] / (pk["bf16_sus"] * 1e12), rf["B_layer"] / (pk["hbm"] * 1e9))
+    ffn_tflops = rf["F_layer"] / (ms_max / 1e3) / 1e12
+    layer = {"bound": "tensor" if rf["F_layer"] / (pk["bf16_sus"] * 1e12) >= rf["B_layer"] / (pk["hbm"] * 1e9) else "hbm",
+             "roofline_ms": t_bound * 1e3, "frac": t_bound / (ms_max / 1e3),
+             "executed_ffn_tflops": ffn_tflops,
+             "pct_of_bf16_peak_burst": 100.0 * ffn_tflops / pk["bf16"],
+             "pct_of_bf16_peak_sustained": 100.0 * ffn_tflops / pk["bf16_sus"],
+             "hbm_gbs": rf["B_layer"] / (ms_max / 1e3) / 1e9,
+             "pct_of_hbm": 100.0 * rf["B_layer"] / (ms_max / 1e3) / 1e9 / pk["hbm"]}
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, ri, b, ew)
+
+    touched = st["experts_hit"] * 3.0 * w.d * w.I * 2
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded inputs, random-init weights of the workload's shapes",
+        "config": config_of(w, {
+            "global_batch": w.T * dist.world, "parallelism": f"replicas{dist.world}",
+            "l2": f"no flush: expert weights touched per step {touched / 1e9:.2f} GB > L2 126 MB"}),
+        "e2e": {"value": dist.world * w.T / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": int(x_host.numel() * 2),
+                "d2h_bytes_per_step": int(out_host.numel() * 2), "ms_per_step": e2e_ms},
+        "roofline": roof,
+        "layer_roofline": layer,
+        "cpu_baseline": cpu,
+        "gpu_launches": KERNELS_PER_FORWARD * args.steps if w.N > 0 else 4 * args.steps,
+        "clocks": clk,
+        "routing": st,
+        "stage_ms": {k: round(v, 5) for k, v in per.items()},
+    }
+    return line
+
+
+def run_reference(args, dist, w):
+    """The fp64 CPU oracle, as it stands, on the host cores."""
+    if dist.rank != 0:
+        return None
+    ri = wl.routing_inputs(w)
+    b = ri.bias(w.N, w.delta)
+    ew = wl.expert_weights(w, "cuda" if torch.cuda.is_available() else "cpu")
+    cores = len(os.sched_getaffinity(0))
+    # size the per-step sample so the whole run stays within about two minutes
+    dt1, n1 = oracle_sample_time(w, ri, b, ew, 4, 100)
+    per_tok = dt1 / n1
+    n = int(max(1, min(w.T, 120.0 / max(args.steps + args.warmup, 1) / max(per_tok, 1e-6))))
+    for i in range(args.warmup):
+        oracle_sample_time(w, ri, b, ew, n, 200 + i)
+    tot = 0.0
+    for i in range(args.steps):
+        dt, n = oracle_sample_time(w, ri, b, ew, n, 300 + i)
+        tot += dt
+    ms = tot / args.steps * 1e3
+    value = n / (ms / 1e3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: seeded inputs, random-init weights of the workload's shapes",
+        "config": config_of(w, {"global_batch": w.T, "parallelism": "cpu"}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{n} of {w.T} tokens per step (seeded samples), fp64 NumPy oracle"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    w = wl.get(args.workload)
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        line = run_reference(args, Dist(1) if int(os.environ.get("WORLD_SIZE", "1")) == 1 else _Rank0(args.gpus), w)
+        print(json.dumps(line), flush=True)
+        return
+    dist = Dist(args.gpus)
+    try:
+        line = run_ours(args, dist, w)
+        if dist.rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.close()
+
+
+class _Rank0:
+    """Rank 0 of a torchrun launch of the reference arm: works alone."""
+
+    def __init__(self, n):
+        self.world, self.rank, self.local = n, 0, 0
+
+
+if __name__ == "__main__":
+    main()

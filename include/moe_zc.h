@@ -1,0 +1,161 @@
+/*
+ * moe_zc.h -- C ABI of the B200 (sm_100a) MoE layer with zero-computation
+ * experts.
+ *
+ * The layer (LongCat-Flash write-up "Meituan's large model goes viral for its
+ * speed", itouyu.top, section "Zero-computation experts"): the expert pool
+ * holds N SwiGLU FFN experts and Z zero-computation experts that return their
+ * input unchanged.  A softmax router R scores all E = N + Z experts of each
+ * token x_t; the expert bias b_i is added to those scores to pick the top K
+ * experts, and the gate of each pick is its unbiased softmax probability.  So
+ *
+ *   p_t   = softmax(x_t W_r^T)                 over all E experts
+ *   S_t   = top-K indices of p_t + b           (equal scores: lower index)
+ *   out_t = sum_{i in S_t, i >= N} p_{t,i} x_t
+ *         + sum_{i in S_t, i <  N} p_{t,i} W_down,i (SiLU(W_gate,i x_t) * W_up,i x_t)
+ *
+ * The page prints only the symbol glossary of this formula (the formula
+ * itself is lost); the readings above -- softmax over all E experts, bias
+ * added after the softmax and used for selection only, no renormalisation of
+ * the gates, SwiGLU without biases -- are the plainest ones it supports.
+ * The number of FFN experts a token runs varies from 0 to K.
+ *
+ * Data layout (all row-major, like nn.Linear.weight):
+ *   x       [T, d]     bf16     tokens
+ *   W_r     [E, d]     bf16     router; rows 0..N-1 FFN experts, N..E-1 zero experts
+ *   b       [E]        fp32     expert bias (selection only)
+ *   W_gate  [N, I, d]  bf16
+ *   W_up    [N, I, d]  bf16
+ *   W_down  [N, d, I]  bf16
+ *   out     [T, d]     bf16
+ *
+ * Ownership and concurrency: every pointer argument of moe_zc_forward* is
+ * device memory owned by the caller, 16-byte aligned, not freed or kept by the
+ * library past the call's stream work.  The library owns one workspace per
+ * device (grown on demand by moe_zc_forward*, or sized up front by
+ * moe_zc_reserve) and the routing of the last forward.  It is not re-entrant:
+ * one forward in flight per process; callers serialise.  Forward calls are
+ * asynchronous on `stream` (a cudaStream_t, NULL = legacy default stream).
+ *
+ * Errors: every call returns a moe_zc_status; nothing aborts or traps.
+ * Device-side waits are bounded; a wait that runs out sets a device flag that
+ * moe_zc_synchronize / moe_zc_expert_load report as MOE_ZC_ERR_TIMEOUT.
+ */
+#ifndef MOE_ZC_H
+#define MOE_ZC_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_zc_status {
+  MOE_ZC_OK = 0,
+  MOE_ZC_ERR_INVALID_ARG = -1,  /* null pointer, K < 1, K > E, T < 0, N < 0, Z < 0, E < 1 */
+  MOE_ZC_ERR_UNSUPPORTED = -2,  /* d % 128, I % 128, K > 32, E > 1024, misaligned pointer */
+  MOE_ZC_ERR_CUDA = -3,         /* a CUDA runtime or driver call failed */
+  MOE_ZC_ERR_OOM = -4,          /* workspace allocation failed */
+  MOE_ZC_ERR_TIMEOUT = -5,      /* a bounded device-side wait ran out */
+  MOE_ZC_ERR_NO_RESULT = -6     /* no forward has run yet on this device */
+} moe_zc_status;
+
+/* Largest supported sizes. */
+#define MOE_ZC_MAX_K 32
+#define MOE_ZC_MAX_E 1024
+
+/*
+ * Forward pass of the layer defined above ("Zero-computation experts").
+ * T may be 0 (no work, returns MOE_ZC_OK).  N may be 0 (every pick is a zero
+ * expert) and Z may be 0 (plain softmax top-K MoE).  Requires d % 128 == 0,
+ * I % 128 == 0, 1 <= K <= min(E, 32), E <= 1024, 16-byte aligned pointers.
+ * W_gate/W_up/W_down may be NULL only when N == 0.
+ * Asynchronous on `stream`; the expert-load histogram and routing of this
+ * call stay available through moe_zc_expert_load / moe_zc_last_routing.
+ */
+int moe_zc_forward(const void* x, const void* W_r, const float* b,
+                   const void* W_gate, const void* W_up, const void* W_down,
+                   int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I,
+                   void* out, void* stream);
+
+/*
+ * moe_zc_forward with an optional per-expert router-logit offset
+ * (logit_offset [E] fp32 device memory, or NULL), added to x_t W_r^T before
+ * the softmax, so it moves gates as well as picks.  It exists to skew expert
+ * load in synthetic workloads; the write-up's layer has no such term.
+ */
+int moe_zc_forward_ex(const void* x, const void* W_r, const float* b,
+                      const void* W_gate, const void* W_up, const void* W_down,
+                      int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I,
+                      const float* logit_offset, void* out, void* stream);
+
+/*
+ * Expert-load histogram of the last forward on the current device: the number
+ * of tokens that picked each of the E experts, zero experts included.  This is
+ * the "recent expert usage" that the write-up's bias controller (section
+ * "Zero-computation experts") steers b_i by.  out_counts: host int32[E].
+ * Waits for the last forward to finish; returns MOE_ZC_ERR_TIMEOUT if one of
+ * its device waits ran out, MOE_ZC_ERR_NO_RESULT before the first forward.
+ */
+int moe_zc_expert_load(int32_t* out_counts);
+
+/*
+ * Routing of the last forward (for tests and debugging): idx host int32[T*K],
+ * gate host float[T*K], row t holding token t's picks in descending biased
+ * score (ties: lower index first).  Either pointer may be NULL.  Waits like
+ * moe_zc_expert_load.
+ */
+int moe_zc_last_routing(int32_t* idx, float* gate);
+
+/*
+ * Intermediate activations of FFN expert e in the last forward (for tests):
+ * the tokens routed to e in slot order (tokens, host int32[n]), their SwiGLU
+ * hidden rows H (host bf16 [n, I]) and their expert outputs Y (host bf16
+ * [n, d]) before gating.  *n_rows receives the count n; at most max_rows rows
+ * are copied.  Any output pointer except n_rows may be NULL.
+ */
+int moe_zc_last_expert(int32_t e, int32_t max_rows, int32_t* n_rows,
+                       int32_t* tokens, void* H, void* Y);
+
+/* Wait for the last forward; report (and clear) a device-side timeout. */
+int moe_zc_synchronize(void);
+
+/*
+ * Size the current device's workspace for forwards up to these sizes, so
+ * later forwards allocate nothing.  Optional.
+ */
+int moe_zc_reserve(int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I);
+
+/* Free every device's workspace and cached state. */
+void moe_zc_release(void);
+
+/* Text for a status code. */
+const char* moe_zc_status_string(int status);
+
+/*
+ * Per-stage timing of forwards with CUDA events recorded on the forward's own
+ * stream between its kernels.  moe_zc_profile(1) starts (or restarts)
+ * recording on the current device -- at most 256 forwards are kept --
+ * moe_zc_profile(0) stops.  moe_zc_profile_read waits for the last recorded
+ * forward and writes, for each stage i < max_stages, the milliseconds summed
+ * over the recorded forwards (stage_ms: host float[max_stages]; 8 stages,
+ * named by moe_zc_stage_name: router_gemm, route, scan, assign_slots,
+ * permute, gateup_gemm, down_gemm, combine) and their count to *n_forwards.
+ */
+int moe_zc_profile(int32_t enable);
+int moe_zc_profile_read(float* stage_ms, int32_t max_stages, int32_t* n_forwards);
+const char* moe_zc_stage_name(int32_t i);
+
+/*
+ * Test hook for the error paths: make the next n workspace allocations fail
+ * (MOE_ZC_ERR_OOM), and/or make every bounded device wait of the next forward
+ * give up after `wait_limit` nanoseconds (0 = the normal 2 s), so that the
+ * timeout path runs without a fault.  Not for production use.
+ */
+void moe_zc_test_inject(int32_t fail_allocs, int64_t wait_limit);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_ZC_H */

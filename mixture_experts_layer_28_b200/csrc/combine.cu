@@ -1,0 +1,78 @@
+// combine.cu -- weighted combine of the expert outputs.
+//
+// LongCat-Flash write-up ("Meituan's large model goes viral for its speed",
+// section "Zero-computation experts"): the layer's output is the
+// gate-weighted sum of the picked experts' outputs, and a zero-computation
+// expert's output is its input.  So, per token t,
+//
+//   out_t = bf16( zsum_t * x_t + sum_{k : slot_{t,k} >= 0} gate_{t,k} * Y[slot_{t,k}] )
+//
+// with zsum_t the router's sum of zero-expert gates.  fp32 accumulation in a
+// fixed order (zero experts first, then picks k = 0..K-1), one rounding to
+// bf16: the result does not depend on where the dispatch put a token's rows.
+// One CTA per token; each thread handles 8 features with 16-byte loads.
+#include "kernels.cuh"
+
+namespace moezc {
+namespace {
+
+__device__ __forceinline__ void acc8(float (&a)[8], const uint4& v, float g) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    a[2 * i] = fmaf(g, __uint_as_float(w[i] << 16), a[2 * i]);
+    a[2 * i + 1] = fmaf(g, __uint_as_float(w[i] & 0xFFFF0000u), a[2 * i + 1]);
+  }
+}
+
+__global__ void combine_kernel(const uint4* __restrict__ x, const uint4* __restrict__ Y,
+                               const int* __restrict__ slot, const float* __restrict__ gate,
+                               const float* __restrict__ zsum, int d8, int K,
+                               uint4* __restrict__ out) {
+  const int64_t t = blockIdx.x;
+  __shared__ int sl[MOE_MAX_K_INTERNAL];
+  __shared__ float gt[MOE_MAX_K_INTERNAL];
+  __shared__ int nffn;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int k = 0; k < K; ++k) {
+      const int s = slot[t * K + k];
+      if (s >= 0) { sl[n] = s; gt[n] = gate[t * K + k]; ++n; }
+    }
+    nffn = n;
+  }
+  __syncthreads();
+  const float z = zsum[t];
+  const int n = nffn;
+  for (int c = threadIdx.x; c < d8; c += blockDim.x) {
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = 0.f;
+    acc8(a, x[t * d8 + c], z);
+    for (int k = 0; k < n; ++k) acc8(a, Y[static_cast<int64_t>(sl[k]) * d8 + c], gt[k]);
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+      ow[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    out[t * d8 + c] = o;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const __nv_bfloat16* x, const __nv_bfloat16* Y, const int* slot,
+                           const float* gate, const float* zsum, int64_t T, int d, int K,
+                           __nv_bfloat16* out, cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  const int d8 = d / 8;
+  const int threads = d8 < 256 ? ((d8 + 31) / 32) * 32 : 256;
+  combine_kernel<<<static_cast<unsigned>(T), threads, 0, stream>>>(
+      reinterpret_cast<const uint4*>(x), reinterpret_cast<const uint4*>(Y), slot, gate, zsum,
+      d8, K, reinterpret_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace moezc

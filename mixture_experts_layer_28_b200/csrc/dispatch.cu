@@ -1,0 +1,147 @@
+// dispatch.cu -- counting-sort dispatch of (token, pick) pairs to FFN experts.
+//
+// Only picks of the N FFN experts are dispatched; a zero-computation expert
+// returns its input (LongCat-Flash write-up "Meituan's large model goes viral
+// for its speed", section "Zero-computation experts"), so its picks were
+// already folded into zsum by the router and get slot -1 here.
+//
+//   scan      one CTA: per expert, rows = count rounded up to 16 and token
+//             tiles = ceil(count / 256); exclusive prefix sums give each
+//             expert's first row in the permuted buffers (grp_off) and its
+//             first GEMM token tile (grp_ttp); the GEMM grid walks grp_ttp.
+//   assign    one thread per (token, pick): lanes of a warp that picked the
+//             same expert are grouped with __match_any_sync and take their
+//             slots with one atomicAdd per group (warp-aggregated atomics).
+//   permute   one CTA per token: copies x_t (16-byte vectors) to each of its
+//             FFN slots of Xp, the B operand of the gate/up GEMM.
+// The histogram itself is integer and comes from the router, so it is exact.
+#include "kernels.cuh"
+
+namespace moezc {
+namespace {
+
+constexpr int SCAN_THREADS = 1024;
+
+__device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = (lane < SCAN_THREADS / 32) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
+    }
+    warp_sums[lane] = w;  // inclusive prefix over warps
+  }
+  __syncthreads();
+  const int base = warp ? warp_sums[warp - 1] : 0;
+  *total = warp_sums[SCAN_THREADS / 32 - 1];
+  __syncthreads();
+  return base + incl - v;
+}
+
+__global__ void __launch_bounds__(SCAN_THREADS)
+scan_kernel(const int* __restrict__ cnt, int N, int* __restrict__ grp_off,
+            int* __restrict__ grp_ttp, int* __restrict__ fill) {
+  __shared__ int warp_sums[32];
+  __shared__ int carry_rows, carry_tiles;
+  if (threadIdx.x == 0) { carry_rows = 0; carry_tiles = 0; }
+  __syncthreads();
+  for (int base = 0; base < N; base += SCAN_THREADS) {
+    const int g = base + threadIdx.x;
+    const int c = (g < N) ? cnt[g] : 0;
+    const int rows = (c + 15) & ~15;
+    const int tiles = (c + GEMM_BN - 1) / GEMM_BN;
+    int tot_rows, tot_tiles;
+    const int off = block_excl_scan(rows, warp_sums, &tot_rows);
+    const int ttp = block_excl_scan(tiles, warp_sums, &tot_tiles);
+    if (g < N) {
+      grp_off[g] = carry_rows + off;
+      grp_ttp[g] = carry_tiles + ttp;
+      fill[g] = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) { carry_rows += tot_rows; carry_tiles += tot_tiles; }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    grp_off[N] = carry_rows;
+    grp_ttp[N] = carry_tiles;
+  }
+}
+
+__global__ void assign_slots_kernel(const int* __restrict__ idx, int64_t pairs, int N,
+                                    const int* __restrict__ grp_off, int* __restrict__ fill,
+                                    int* __restrict__ slot) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const bool valid = i < pairs;
+  const int e = valid ? idx[i] : -1;
+  const bool ffn = valid && e >= 0 && e < N;
+  const unsigned act = __ballot_sync(0xffffffffu, ffn);
+  int s = -1;
+  if (ffn) {
+    const unsigned peers = __match_any_sync(act, e);
+    const int leader = __ffs(peers) - 1;
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    int base = 0;
+    if (lane == leader) base = atomicAdd(&fill[e], __popc(peers));
+    base = __shfl_sync(peers, base, leader);
+    s = grp_off[e] + base + rank;
+  }
+  if (valid) slot[i] = s;
+}
+
+__global__ void permute_kernel(const uint4* __restrict__ x, const int* __restrict__ slot,
+                               int d8, int K, uint4* __restrict__ Xp) {
+  const int64_t t = blockIdx.x;
+  __shared__ int sl[MOE_MAX_K_INTERNAL];
+  if (threadIdx.x < K) sl[threadIdx.x] = slot[t * K + threadIdx.x];
+  __syncthreads();
+  const uint4* src = x + t * d8;
+  for (int c = threadIdx.x; c < d8; c += blockDim.x) {
+    const uint4 v = src[c];
+    for (int k = 0; k < K; ++k) {
+      const int s = sl[k];
+      if (s >= 0) Xp[static_cast<int64_t>(s) * d8 + c] = v;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_scan(const int* cnt, int N, int* grp_off, int* grp_ttp, int* fill,
+                        cudaStream_t stream) {
+  scan_kernel<<<1, SCAN_THREADS, 0, stream>>>(cnt, N, grp_off, grp_ttp, fill);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_assign_slots(const int* idx, int64_t pairs, int N, const int* grp_off,
+                                int* fill, int* slot, cudaStream_t stream) {
+  if (pairs <= 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (pairs + threads - 1) / threads;
+  assign_slots_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(idx, pairs, N,
+                                                                            grp_off, fill, slot);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, int d, int K,
+                           __nv_bfloat16* Xp, cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  const int d8 = d / 8;
+  const int threads = d8 < 256 ? ((d8 + 31) / 32) * 32 : 256;
+  permute_kernel<<<static_cast<unsigned>(T), threads, 0, stream>>>(
+      reinterpret_cast<const uint4*>(x), slot, d8, K, reinterpret_cast<uint4*>(Xp));
+  return cudaGetLastError();
+}
+
+}  // namespace moezc

@@ -1,0 +1,311 @@
+// gemm_tcgen05.cu -- grouped "SwapAB" GEMM on the 5th-generation tensor cores.
+//
+// The three contractions of the MoE layer with zero-computation experts
+// (LongCat-Flash write-up "Meituan's large model goes viral for its speed",
+// section "Zero-computation experts"; SwiGLU expert form per the layer's
+// definition in moe_zc.h) run on this one engine:
+//
+//   router   logits[t, e]  = x_t . W_r[e]                  (fp32 out)
+//   gate/up  H[s, i]       = SiLU(Xp_s . W_gate[e,i]) * (Xp_s . W_up[e,i])
+//   down     Y[s, j]       = H_s . W_down[e, j]
+//
+// where s runs over the slots of the tokens routed to FFN expert e.  As in the
+// write-up's section on custom kernels ("SwapAB"), the weights are the left
+// operand: an A block is 128 weight rows (MMA M = 128) and the tokens of one
+// expert are the right operand (MMA N = 16..256 in steps of 16), so an expert
+// hit by a handful of decode tokens costs an N = 16 MMA rather than a padded
+// 128-row one.
+//
+// A tile is (expert g, token tile j, weight block m): two A blocks (gate and
+// up rows of block m, or two consecutive 128-row blocks of W_down / W_r)
+// against up to 256 tokens, giving two 128 x N fp32 accumulators in TMEM
+// (columns 0..255 and 256..511).
+//
+// Persistent, warp-specialised CTA (256 threads, one per SM):
+//   warp 0      TMA producer: A blocks [128 x 64] and B boxes [32 x 64],
+//               128-byte swizzle, into a 3-stage shared-memory ring
+//   warp 1      MMA issuer: tcgen05.mma kind::f16, commits free the stage
+//   warp 2      TMEM allocator
+//   warps 4..7  epilogue: tcgen05.ld -> fp32 math -> global stores
+// Every wait is time-bounded (ptx.cuh); on running out the CTA drains its
+// in-flight copies and MMAs, frees TMEM and returns with the error flag set.
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace moezc {
+namespace {
+
+constexpr long long DRAIN_NS = 2000000000LL;  // bound of the drain waits at exit
+
+struct Tile {
+  int g;        // group (expert)
+  int m;        // weight block
+  int tok0;     // first token of the tile inside its group
+  int ntok;     // valid tokens in the tile
+  int nmma;     // MMA N: ntok rounded up to 16
+  int brow0;    // first B row
+  int count;    // tokens in the group
+  bool has_a1;  // second A block present
+  int a0_row, a1_row;
+};
+
+template <int MODE>
+__device__ __forceinline__ int total_tiles(const GemmParams& p) {
+  if (MODE == MODE_ROUTER) return ((p.T + GEMM_BN - 1) / GEMM_BN) * p.mblocks;
+  return __ldg(p.grp_ttp + p.G) * p.mblocks;
+}
+
+template <int MODE>
+__device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
+  Tile tl;
+  const int tt = t / p.mblocks;
+  tl.m = t - tt * p.mblocks;
+  int j;
+  if (MODE == MODE_ROUTER) {
+    tl.g = 0;
+    j = tt;
+    tl.count = p.T;
+    tl.brow0 = 0;
+  } else {
+    // largest g with ttp[g] <= tt
+    int lo = 0, hi = p.G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(p.grp_ttp + mid) <= tt) lo = mid; else hi = mid - 1;
+    }
+    tl.g = lo;
+    j = tt - __ldg(p.grp_ttp + lo);
+    tl.count = __ldg(p.grp_count + lo);
+    tl.brow0 = __ldg(p.grp_off + lo);
+  }
+  tl.tok0 = j * GEMM_BN;
+  tl.ntok = min(GEMM_BN, tl.count - tl.tok0);
+  tl.nmma = (tl.ntok + 15) & ~15;
+  tl.brow0 += tl.tok0;
+  if (MODE == MODE_GATEUP) {
+    tl.a0_row = tl.g * p.a_rows + tl.m * GEMM_BM;   // W_gate rows
+    tl.a1_row = tl.a0_row;                           // W_up rows
+    tl.has_a1 = true;
+  } else {
+    const int r = tl.m * 2 * GEMM_BM;
+    tl.a0_row = tl.g * p.a_rows + r;
+    tl.a1_row = tl.a0_row + GEMM_BM;
+    tl.has_a1 = (r + GEMM_BM) < p.a_rows;
+  }
+  return tl;
+}
+
+__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
+
+template <int MODE>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+            const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[GEMM_STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[GEMM_STAGES];
+  __shared__ __align__(8) uint64_t acc_full_bar;
+  __shared__ __align__(8) uint64_t acc_empty_bar;
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_sh;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GEMM_STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&acc_full_bar, 1);
+    mbar_init(&acc_empty_bar, 128);
+    mbar_init(&drain_bar, 1);
+    abort_sh = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 2) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const int ntiles = total_tiles<MODE>(p);
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0;          // stages armed at least once
+    uint32_t last_par = 0;       // parity each stage was last armed with
+    for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x) {
+      const Tile tl = decode_tile<MODE>(p, t);
+      const int nbox = (tl.nmma + GEMM_B_BOX_ROWS - 1) / GEMM_B_BOX_ROWS;
+      const uint32_t bytes = GEMM_A_BYTES * (tl.has_a1 ? 2 : 1) +
+                             nbox * GEMM_B_BOX_ROWS * GEMM_BK * 2;
+      for (int ks = 0; ks < p.ksteps; ++ks) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1, p.wait_ns, p.err)) {
+          abort_sh = 1;
+          break;
+        }
+        uint8_t* st = smem + stage * GEMM_STAGE_BYTES;
+        mbar_arrive_expect_tx(&full_bar[stage], bytes);
+        armed |= 1u << stage;
+        last_par = (last_par & ~(1u << stage)) | (phase << stage);
+        const int kc = ks * GEMM_BK;
+        tma_load_2d(st, &tmA0, &full_bar[stage], kc, tl.a0_row);
+        if (tl.has_a1) tma_load_2d(st + GEMM_A_BYTES, &tmA1, &full_bar[stage], kc, tl.a1_row);
+        uint8_t* sb = st + 2 * GEMM_A_BYTES;
+        for (int bx = 0; bx < nbox; ++bx)
+          tma_load_2d(sb + bx * GEMM_B_BOX_ROWS * GEMM_BK * 2, &tmB, &full_bar[stage], kc,
+                      tl.brow0 + bx * GEMM_B_BOX_ROWS);
+        if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+    // Drain: every copy this thread started must land before the CTA exits.
+    for (int s = 0; s < GEMM_STAGES; ++s)
+      if (armed & (1u << s)) mbar_wait(&full_bar[s], (last_par >> s) & 1, DRAIN_NS, p.err);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int local = 0;
+    for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x, ++local) {
+      const Tile tl = decode_tile<MODE>(p, t);
+      if (local > 0 && !mbar_wait(&acc_empty_bar, (local - 1) & 1, p.wait_ns, p.err)) {
+        abort_sh = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16_f32(GEMM_BM, tl.nmma);
+      bool ok = true;
+      for (int ks = 0; ks < p.ksteps; ++ks) {
+        if (!mbar_wait(&full_bar[stage], phase, p.wait_ns, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + stage * GEMM_STAGE_BYTES);
+        const uint64_t a0 = smem_desc_sw128(st);
+        const uint64_t a1 = smem_desc_sw128(st + GEMM_A_BYTES);
+        const uint64_t bd = smem_desc_sw128(st + 2 * GEMM_A_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
+          const uint32_t acc = (ks | kk) != 0;
+          umma_bf16(tmem, a0 + 2 * kk, bd + 2 * kk, idesc, acc);
+          if (tl.has_a1) umma_bf16(tmem + 256, a1 + 2 * kk, bd + 2 * kk, idesc, acc);
+        }
+        umma_commit(&empty_bar[stage]);
+        if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) { abort_sh = 1; break; }
+      umma_commit(&acc_full_bar);
+    }
+    // Drain: all MMAs issued by this thread finish before TMEM is freed.
+    umma_commit(&drain_bar);
+    mbar_wait(&drain_bar, 0, DRAIN_NS, p.err);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                 // TMEM lane quadrant
+    const int row_in_blk = q * 32 + lane;   // weight row inside an A block
+    const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    int local = 0;
+    for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x, ++local) {
+      const Tile tl = decode_tile<MODE>(p, t);
+      if (!mbar_wait(&acc_full_bar, local & 1, p.wait_ns, p.err)) {
+        abort_sh = 1;
+        break;
+      }
+      tc_fence_after();
+      for (int c0 = 0; c0 < tl.nmma; c0 += 16) {
+        uint32_t r0[16], r1[16];
+        tmem_ld16(tq + c0, r0);
+        if (tl.has_a1) tmem_ld16(tq + 256 + c0, r1);
+        tmem_ld_wait();
+        if (MODE == MODE_ROUTER) {
+          float* out = static_cast<float*>(p.out);
+          const int e0 = tl.m * 2 * GEMM_BM + row_in_blk;
+          const int e1 = e0 + GEMM_BM;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int tok = tl.tok0 + c0 + i;
+            if (tok < tl.count) {
+              float* row = out + static_cast<size_t>(tok) * p.out_ld;
+              if (e0 < p.a_rows) row[e0] = __uint_as_float(r0[i]);
+              if (tl.has_a1 && e1 < p.a_rows) row[e1] = __uint_as_float(r1[i]);
+            }
+          }
+        } else if (MODE == MODE_GATEUP) {
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+          const int f = tl.m * GEMM_BM + row_in_blk;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c = tl.tok0 + c0 + i;
+            if (c < tl.count) {
+              const float h = silu_f(__uint_as_float(r0[i])) * __uint_as_float(r1[i]);
+              out[static_cast<size_t>(tl.brow0 - tl.tok0 + c) * p.out_ld + f] =
+                  __float2bfloat16_rn(h);
+            }
+          }
+        } else {
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+          const int f0 = tl.m * 2 * GEMM_BM + row_in_blk;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c = tl.tok0 + c0 + i;
+            if (c < tl.count) {
+              __nv_bfloat16* row = out + static_cast<size_t>(tl.brow0 - tl.tok0 + c) * p.out_ld;
+              row[f0] = __float2bfloat16_rn(__uint_as_float(r0[i]));
+              if (tl.has_a1) row[f0 + GEMM_BM] = __float2bfloat16_rn(__uint_as_float(r1[i]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty_bar);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap& a1,
+                        const CUtensorMap& b, const GemmParams& p, int grid,
+                        cudaStream_t stream) {
+  if (grid <= 0) return cudaSuccess;
+  cudaError_t e = cudaSuccess;
+  switch (mode) {
+    case MODE_ROUTER:
+      e = cudaFuncSetAttribute(gemm_kernel<MODE_ROUTER>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      gemm_kernel<MODE_ROUTER><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(a0, a1, b, p);
+      break;
+    case MODE_GATEUP:
+      e = cudaFuncSetAttribute(gemm_kernel<MODE_GATEUP>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      gemm_kernel<MODE_GATEUP><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(a0, a1, b, p);
+      break;
+    case MODE_DOWN:
+      e = cudaFuncSetAttribute(gemm_kernel<MODE_DOWN>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      gemm_kernel<MODE_DOWN><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(a0, a1, b, p);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moezc

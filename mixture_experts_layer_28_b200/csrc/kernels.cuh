@@ -1,0 +1,70 @@
+// kernels.cuh -- launchers of the five hot-path kernels (internal C++ API).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace moezc {
+
+constexpr int MOE_MAX_K_INTERNAL = 32;   // most picks per token
+
+// ------------------------------------------------------------------ GEMM
+// One tcgen05 engine serves the three contractions of the layer.  Weights are
+// the A operand (M = 128 rows per MMA, two A blocks per tile -> two fp32
+// accumulators in TMEM); tokens are the B operand (N = 16..256 per tile).
+enum GemmMode : int { MODE_ROUTER = 0, MODE_GATEUP = 1, MODE_DOWN = 2 };
+
+constexpr int GEMM_BM = 128;           // rows of one A block
+constexpr int GEMM_BN = 256;           // tokens per tile at most
+constexpr int GEMM_BK = 64;            // K per pipeline stage (128-byte rows)
+constexpr int GEMM_STAGES = 3;
+constexpr int GEMM_B_BOX_ROWS = 32;    // tokens per TMA box of B
+constexpr int GEMM_THREADS = 256;
+constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;
+constexpr int GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;
+constexpr int GEMM_STAGE_BYTES = 2 * GEMM_A_BYTES + GEMM_B_BYTES;
+constexpr int GEMM_SMEM_BYTES = GEMM_STAGES * GEMM_STAGE_BYTES + 1024;
+
+struct GemmParams {
+  // Token groups (FFN experts).  For MODE_ROUTER there is one group of T
+  // tokens starting at row 0 and the arrays are unused.
+  const int* grp_count;   // [G] tokens in group g
+  const int* grp_off;     // [G] first B row of group g (multiple of 16)
+  const int* grp_ttp;     // [G+1] prefix sum of token tiles per group
+  int G;
+  int T;                  // MODE_ROUTER: tokens
+  int ksteps;             // contraction length / GEMM_BK
+  int mblocks;            // tiles along the weight rows of one group
+  int a_rows;             // weight rows per group: E (router), I (gate/up), d (down)
+  void* out;              // fp32 logits [T, E] | bf16 H [rows, I] | bf16 Y [rows, d]
+  int out_ld;             // elements per output row
+  int* err;               // device error flag
+  long long wait_ns;      // bound of every pipeline wait
+};
+
+cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap& a1,
+                        const CUtensorMap& b, const GemmParams& p, int grid,
+                        cudaStream_t stream);
+
+// ------------------------------------------------------------------ router
+// softmax over E logits (+offset), + bias, top-K, zero-gate sums, histogram.
+cudaError_t launch_route(const float* logits, const float* b, const float* offset, int64_t T,
+                         int E, int N, int K, int* idx, float* gate, float* zsum, int* cnt,
+                         cudaStream_t stream);
+
+// ------------------------------------------------------------------ dispatch
+cudaError_t launch_scan(const int* cnt, int N, int* grp_off, int* grp_ttp, int* fill,
+                        cudaStream_t stream);
+cudaError_t launch_assign_slots(const int* idx, int64_t pairs, int N, const int* grp_off,
+                                int* fill, int* slot, cudaStream_t stream);
+cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, int d, int K,
+                           __nv_bfloat16* Xp, cudaStream_t stream);
+
+// ------------------------------------------------------------------ combine
+cudaError_t launch_combine(const __nv_bfloat16* x, const __nv_bfloat16* Y, const int* slot,
+                           const float* gate, const float* zsum, int64_t T, int d, int K,
+                           __nv_bfloat16* out, cudaStream_t stream);
+
+}  // namespace moezc

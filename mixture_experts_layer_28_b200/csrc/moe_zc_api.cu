@@ -1,0 +1,524 @@
+// moe_zc_api.cu -- the C ABI (include/moe_zc.h): argument checks, per-device
+// workspace, TMA descriptors and the launch sequence of one forward.
+//
+// One forward of the MoE layer with zero-computation experts (LongCat-Flash
+// write-up "Meituan's large model goes viral for its speed", section
+// "Zero-computation experts") is, all on the caller's stream:
+//
+//   1  router GEMM        logits = x W_r^T              tcgen05, fp32 out
+//   2  route              softmax, + b, top-K, zsum, histogram
+//   3  scan               per-expert row offsets and GEMM token tiles
+//   4  assign slots       warp-aggregated atomics, FFN picks only
+//   5  permute            x rows -> Xp (grouped by expert)
+//   6  gate/up GEMM       H = SiLU(Xp W_gate^T) * (Xp W_up^T)
+//   7  down GEMM          Y = H W_down^T
+//   8  combine            out = zsum x + sum gate * Y
+//
+// No step reads anything back to the host: the GEMM tile lists are built on
+// the device and walked by persistent kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/moe_zc.h"
+#include "kernels.cuh"
+
+namespace {
+
+using namespace moezc;
+
+constexpr int kMaxDevices = 16;
+constexpr long long kWaitNs = 2000000000LL;  // 2 s bound of every pipeline wait
+
+struct Buf {
+  void* p = nullptr;
+  size_t bytes = 0;
+};
+
+struct Ctx {
+  bool init = false;
+  int sms = 0;
+  Buf logits, idx, gate, zsum, slot, cnt, fill, grp_off, grp_ttp, Xp, H, Y, err;
+  cudaEvent_t done = nullptr;
+  bool has_result = false;
+  int64_t T = 0;
+  int d = 0, N = 0, Z = 0, K = 0, I = 0;
+  int64_t rows_cap = 0;
+};
+
+Ctx g_ctx[kMaxDevices];
+std::mutex g_mu;
+
+// Per-stage CUDA-event timing of forwards (moe_zc_profile / moe_zc_profile_read).
+constexpr int kStages = 8;
+constexpr int kRing = 256;
+const char* const kStageNames[kStages] = {"router_gemm", "route",        "scan",
+                                          "assign_slots", "permute",     "gateup_gemm",
+                                          "down_gemm",    "combine"};
+struct Prof {
+  bool on = false;
+  int device = -1;
+  int n = 0;          // forwards recorded since the last reset
+  bool created = false;
+  cudaEvent_t ev[kRing][kStages + 1];
+};
+Prof g_prof;
+int g_fail_allocs = 0;
+long long g_wait_ns_next = 0;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, k] (row-major), box [box_rows, 64], 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t k, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {k, rows};
+  cuuint64_t strides[1] = {k * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(GEMM_BK), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int ensure(Ctx& c, Buf& b, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  if (b.bytes >= bytes) return MOE_ZC_OK;
+  if (g_fail_allocs > 0) {
+    --g_fail_allocs;
+    return MOE_ZC_ERR_OOM;
+  }
+  if (b.p) {
+    // the previous forward may still read it
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ZC_ERR_CUDA;
+    cudaFree(b.p);
+    b.p = nullptr;
+    b.bytes = 0;
+  }
+  if (cudaMalloc(&b.p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ZC_ERR_OOM;
+  }
+  b.bytes = bytes;
+  (void)c;
+  return MOE_ZC_OK;
+}
+
+int get_ctx(Ctx** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ZC_ERR_CUDA;
+  Ctx& c = g_ctx[dev];
+  if (!c.init) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return MOE_ZC_ERR_CUDA;
+    if (major != 10) return MOE_ZC_ERR_UNSUPPORTED;   // sm_100a only
+    if (cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MOE_ZC_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&c.done, cudaEventDisableTiming) != cudaSuccess)
+      return MOE_ZC_ERR_CUDA;
+    c.init = true;
+  }
+  *out = &c;
+  return MOE_ZC_OK;
+}
+
+int reserve_impl(Ctx& c, int64_t T, int d, int N, int Z, int K, int I) {
+  const int64_t E = static_cast<int64_t>(N) + Z;
+  const int64_t pairs = T * K;
+  const int64_t rows_cap = N > 0 ? pairs + 15LL * N + 16 : 16;
+  int s;
+  const bool fresh_err = c.err.p == nullptr;
+  if ((s = ensure(c, c.err, sizeof(int))) != MOE_ZC_OK) return s;
+  if (fresh_err && cudaMemset(c.err.p, 0, sizeof(int)) != cudaSuccess) return MOE_ZC_ERR_CUDA;
+  if ((s = ensure(c, c.logits, static_cast<size_t>(T * E) * sizeof(float))) != MOE_ZC_OK) return s;
+  if ((s = ensure(c, c.idx, static_cast<size_t>(pairs) * sizeof(int))) != MOE_ZC_OK) return s;
+  if ((s = ensure(c, c.gate, static_cast<size_t>(pairs) * sizeof(float))) != MOE_ZC_OK) return s;
+  if ((s = ensure(c, c.slot, static_cast<size_t>(pairs) * sizeof(int))) != MOE_ZC_OK) return s;
+  if ((s = ensure(c, c.zsum, static_cast<size_t>(T) * sizeof(float))) != MOE_ZC_OK) return s;
+  if ((s = ensure(c, c.cnt, static_cast<size_t>(E) * sizeof(int))) != MOE_ZC_OK) return s;
+  if ((s = ensure(c, c.fill, static_cast<size_t>(N + 1) * sizeof(int))) != MOE_ZC_OK) return s;
+  if ((s = ensure(c, c.grp_off, static_cast<size_t>(N + 1) * sizeof(int))) != MOE_ZC_OK) return s;
+  if ((s = ensure(c, c.grp_ttp, static_cast<size_t>(N + 1) * sizeof(int))) != MOE_ZC_OK) return s;
+  if (N > 0) {
+    if ((s = ensure(c, c.Xp, static_cast<size_t>(rows_cap) * d * 2)) != MOE_ZC_OK) return s;
+    if ((s = ensure(c, c.H, static_cast<size_t>(rows_cap) * I * 2)) != MOE_ZC_OK) return s;
+    if ((s = ensure(c, c.Y, static_cast<size_t>(rows_cap) * d * 2)) != MOE_ZC_OK) return s;
+  }
+  c.rows_cap = rows_cap;
+  return MOE_ZC_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_args(const void* x, const void* W_r, const float* b, const void* W_gate,
+               const void* W_up, const void* W_down, int64_t T, int32_t d, int32_t N, int32_t Z,
+               int32_t K, int32_t I, const float* off, const void* out) {
+  if (!x || !W_r || !b || !out) return MOE_ZC_ERR_INVALID_ARG;
+  if (T < 0 || N < 0 || Z < 0 || d <= 0) return MOE_ZC_ERR_INVALID_ARG;
+  const int64_t E = static_cast<int64_t>(N) + Z;
+  if (E < 1 || K < 1 || K > E) return MOE_ZC_ERR_INVALID_ARG;
+  if (N > 0 && (!W_gate || !W_up || !W_down || I <= 0)) return MOE_ZC_ERR_INVALID_ARG;
+  if (K > MOE_ZC_MAX_K || E > MOE_ZC_MAX_E) return MOE_ZC_ERR_UNSUPPORTED;
+  if (d % 128 != 0) return MOE_ZC_ERR_UNSUPPORTED;
+  if (N > 0 && I % 128 != 0) return MOE_ZC_ERR_UNSUPPORTED;
+  if (T * K + 16LL * N + 16 > (1LL << 31) - 1) return MOE_ZC_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(N) * (d > I ? d : I) > (1LL << 31) - 1) return MOE_ZC_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(W_r) || !aligned16(b) || !aligned16(out))
+    return MOE_ZC_ERR_UNSUPPORTED;
+  if (off && !aligned16(off)) return MOE_ZC_ERR_UNSUPPORTED;
+  if (N > 0 && (!aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down)))
+    return MOE_ZC_ERR_UNSUPPORTED;
+  return MOE_ZC_OK;
+}
+
+#define CK(expr)                                   \
+  do {                                             \
+    if ((expr) != cudaSuccess) {                   \
+      cudaGetLastError();                          \
+      return MOE_ZC_ERR_CUDA;                      \
+    }                                              \
+  } while (0)
+
+// Records event `i` of the current profiled forward (no-op when profiling is off).
+struct StageRec {
+  cudaEvent_t* ev = nullptr;
+  cudaStream_t st = nullptr;
+  void mark(int i) const {
+    if (ev) cudaEventRecord(ev[i], st);
+  }
+};
+
+int forward_impl(const void* x, const void* W_r, const float* b, const void* W_gate,
+                 const void* W_up, const void* W_down, int64_t T, int32_t d, int32_t N,
+                 int32_t Z, int32_t K, int32_t I, const float* off, void* out, void* stream) {
+  int s = check_args(x, W_r, b, W_gate, W_up, W_down, T, d, N, Z, K, I, off, out);
+  if (s != MOE_ZC_OK) return s;
+  Ctx* cp = nullptr;
+  if ((s = get_ctx(&cp)) != MOE_ZC_OK) return s;
+  Ctx& c = *cp;
+  if ((s = reserve_impl(c, T, d, N, Z, K, N > 0 ? I : 128)) != MOE_ZC_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int E = N + Z;
+  const long long wait_ns = g_wait_ns_next > 0 ? g_wait_ns_next : kWaitNs;
+  g_wait_ns_next = 0;
+  int* err = static_cast<int*>(c.err.p);
+  int* cnt = static_cast<int*>(c.cnt.p);
+  int* idx = static_cast<int*>(c.idx.p);
+  float* gate = static_cast<float*>(c.gate.p);
+  float* zsum = static_cast<float*>(c.zsum.p);
+  int* slot = static_cast<int*>(c.slot.p);
+  int* grp_off = static_cast<int*>(c.grp_off.p);
+  int* grp_ttp = static_cast<int*>(c.grp_ttp.p);
+  int* fill = static_cast<int*>(c.fill.p);
+
+  StageRec rec;
+  int dev_now = -1;
+  cudaGetDevice(&dev_now);
+  if (g_prof.on && g_prof.device == dev_now && g_prof.n < kRing) {
+    rec.ev = g_prof.ev[g_prof.n];
+    rec.st = st;
+  }
+  rec.mark(0);
+  CK(cudaMemsetAsync(cnt, 0, sizeof(int) * E, st));
+  if (T > 0) {
+    // 1  router GEMM
+    CUtensorMap mWr, mX;
+    if (!make_map(&mWr, W_r, E, d, GEMM_BM) || !make_map(&mX, x, T, d, GEMM_B_BOX_ROWS))
+      return MOE_ZC_ERR_CUDA;
+    GemmParams pr{};
+    pr.G = 1;
+    pr.T = static_cast<int>(T);
+    pr.ksteps = d / GEMM_BK;
+    pr.mblocks = (E + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
+    pr.a_rows = E;
+    pr.out = c.logits.p;
+    pr.out_ld = E;
+    pr.err = err;
+    pr.wait_ns = wait_ns;
+    const int64_t rtiles = ((T + GEMM_BN - 1) / GEMM_BN) * pr.mblocks;
+    CK(launch_gemm(MODE_ROUTER, mWr, mWr, mX, pr,
+                   static_cast<int>(rtiles < c.sms ? rtiles : c.sms), st));
+    rec.mark(1);
+    // 2  route
+    CK(launch_route(static_cast<const float*>(c.logits.p), b, off, T, E, N, K, idx, gate, zsum,
+                    cnt, st));
+    rec.mark(2);
+    if (N > 0) {
+      // 3-5  dispatch
+      CK(launch_scan(cnt, N, grp_off, grp_ttp, fill, st));
+      rec.mark(3);
+      CK(launch_assign_slots(idx, T * K, N, grp_off, fill, slot, st));
+      rec.mark(4);
+      CK(launch_permute(static_cast<const __nv_bfloat16*>(x), slot, T, d, K,
+                        static_cast<__nv_bfloat16*>(c.Xp.p), st));
+      rec.mark(5);
+      const int64_t tiles_ub = (T * K + GEMM_BN - 1) / GEMM_BN + N;
+      // 6  gate/up GEMM
+      CUtensorMap mWg, mWu, mXp;
+      if (!make_map(&mWg, W_gate, static_cast<uint64_t>(N) * I, d, GEMM_BM) ||
+          !make_map(&mWu, W_up, static_cast<uint64_t>(N) * I, d, GEMM_BM) ||
+          !make_map(&mXp, c.Xp.p, c.rows_cap, d, GEMM_B_BOX_ROWS))
+        return MOE_ZC_ERR_CUDA;
+      GemmParams pg{};
+      pg.grp_count = cnt;
+      pg.grp_off = grp_off;
+      pg.grp_ttp = grp_ttp;
+      pg.G = N;
+      pg.ksteps = d / GEMM_BK;
+      pg.mblocks = I / GEMM_BM;
+      pg.a_rows = I;
+      pg.out = c.H.p;
+      pg.out_ld = I;
+      pg.err = err;
+      pg.wait_ns = wait_ns;
+      const int64_t g_ub = tiles_ub * pg.mblocks;
+      CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, pg, static_cast<int>(g_ub < c.sms ? g_ub : c.sms),
+                     st));
+      rec.mark(6);
+      // 7  down GEMM
+      CUtensorMap mWd, mH;
+      if (!make_map(&mWd, W_down, static_cast<uint64_t>(N) * d, I, GEMM_BM) ||
+          !make_map(&mH, c.H.p, c.rows_cap, I, GEMM_B_BOX_ROWS))
+        return MOE_ZC_ERR_CUDA;
+      GemmParams pd = pg;
+      pd.ksteps = I / GEMM_BK;
+      pd.mblocks = (d + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
+      pd.a_rows = d;
+      pd.out = c.Y.p;
+      pd.out_ld = d;
+      const int64_t d_ub = tiles_ub * pd.mblocks;
+      CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, pd, static_cast<int>(d_ub < c.sms ? d_ub : c.sms),
+                     st));
+      rec.mark(7);
+    } else {
+      rec.mark(3);
+      CK(launch_assign_slots(idx, T * K, N, grp_off, fill, slot, st));
+      for (int i = 4; i <= 7; ++i) rec.mark(i);
+    }
+    // 8  combine
+    CK(launch_combine(static_cast<const __nv_bfloat16*>(x),
+                      static_cast<const __nv_bfloat16*>(c.Y.p), slot, gate, zsum, T, d, K,
+                      static_cast<__nv_bfloat16*>(out), st));
+  } else {
+    for (int i = 1; i <= 7; ++i) rec.mark(i);
+  }
+  rec.mark(8);
+  if (rec.ev) ++g_prof.n;
+  CK(cudaEventRecord(c.done, st));
+  c.has_result = true;
+  c.T = T;
+  c.d = d;
+  c.N = N;
+  c.Z = Z;
+  c.K = K;
+  c.I = I;
+  return MOE_ZC_OK;
+}
+
+int sync_impl(Ctx& c) {
+  if (!c.has_result) return MOE_ZC_ERR_NO_RESULT;
+  CK(cudaEventSynchronize(c.done));
+  int e = 0;
+  CK(cudaMemcpy(&e, c.err.p, sizeof(int), cudaMemcpyDeviceToHost));
+  if (e != 0) {
+    CK(cudaMemset(c.err.p, 0, sizeof(int)));
+    return MOE_ZC_ERR_TIMEOUT;
+  }
+  return MOE_ZC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_zc_forward(const void* x, const void* W_r, const float* b, const void* W_gate,
+                   const void* W_up, const void* W_down, int64_t T, int32_t d, int32_t N,
+                   int32_t Z, int32_t K, int32_t I, void* out, void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return forward_impl(x, W_r, b, W_gate, W_up, W_down, T, d, N, Z, K, I, nullptr, out, stream);
+}
+
+int moe_zc_forward_ex(const void* x, const void* W_r, const float* b, const void* W_gate,
+                      const void* W_up, const void* W_down, int64_t T, int32_t d, int32_t N,
+                      int32_t Z, int32_t K, int32_t I, const float* logit_offset, void* out,
+                      void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return forward_impl(x, W_r, b, W_gate, W_up, W_down, T, d, N, Z, K, I, logit_offset, out,
+                      stream);
+}
+
+int moe_zc_synchronize(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  Ctx* c = nullptr;
+  int s = get_ctx(&c);
+  if (s != MOE_ZC_OK) return s;
+  return sync_impl(*c);
+}
+
+int moe_zc_expert_load(int32_t* out_counts) {
+  if (!out_counts) return MOE_ZC_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Ctx* c = nullptr;
+  int s = get_ctx(&c);
+  if (s != MOE_ZC_OK) return s;
+  if ((s = sync_impl(*c)) != MOE_ZC_OK) return s;
+  CK(cudaMemcpy(out_counts, c->cnt.p, sizeof(int32_t) * (c->N + c->Z), cudaMemcpyDeviceToHost));
+  return MOE_ZC_OK;
+}
+
+int moe_zc_last_routing(int32_t* idx, float* gate) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  Ctx* c = nullptr;
+  int s = get_ctx(&c);
+  if (s != MOE_ZC_OK) return s;
+  if ((s = sync_impl(*c)) != MOE_ZC_OK) return s;
+  const size_t n = static_cast<size_t>(c->T) * c->K;
+  if (n == 0) return MOE_ZC_OK;
+  if (idx) CK(cudaMemcpy(idx, c->idx.p, n * sizeof(int32_t), cudaMemcpyDeviceToHost));
+  if (gate) CK(cudaMemcpy(gate, c->gate.p, n * sizeof(float), cudaMemcpyDeviceToHost));
+  return MOE_ZC_OK;
+}
+
+int moe_zc_last_expert(int32_t e, int32_t max_rows, int32_t* n_rows, int32_t* tokens, void* H,
+                       void* Y) {
+  if (!n_rows || max_rows < 0) return MOE_ZC_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Ctx* c = nullptr;
+  int s = get_ctx(&c);
+  if (s != MOE_ZC_OK) return s;
+  if ((s = sync_impl(*c)) != MOE_ZC_OK) return s;
+  if (e < 0 || e >= c->N) return MOE_ZC_ERR_INVALID_ARG;
+  int cnt = 0, off = 0;
+  if (c->T > 0) {
+    CK(cudaMemcpy(&cnt, static_cast<int*>(c->cnt.p) + e, sizeof(int), cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(&off, static_cast<int*>(c->grp_off.p) + e, sizeof(int),
+                  cudaMemcpyDeviceToHost));
+  }
+  *n_rows = cnt;
+  const int n = cnt < max_rows ? cnt : max_rows;
+  if (n == 0) return MOE_ZC_OK;
+  if (tokens) {
+    const size_t pairs = static_cast<size_t>(c->T) * c->K;
+    std::vector<int32_t> sl(pairs);
+    CK(cudaMemcpy(sl.data(), c->slot.p, pairs * sizeof(int32_t), cudaMemcpyDeviceToHost));
+    for (size_t i = 0; i < pairs; ++i) {
+      const int r = sl[i] - off;
+      if (sl[i] >= 0 && r >= 0 && r < n) tokens[r] = static_cast<int32_t>(i / c->K);
+    }
+  }
+  if (H)
+    CK(cudaMemcpy(H, static_cast<const char*>(c->H.p) + static_cast<size_t>(off) * c->I * 2,
+                  static_cast<size_t>(n) * c->I * 2, cudaMemcpyDeviceToHost));
+  if (Y)
+    CK(cudaMemcpy(Y, static_cast<const char*>(c->Y.p) + static_cast<size_t>(off) * c->d * 2,
+                  static_cast<size_t>(n) * c->d * 2, cudaMemcpyDeviceToHost));
+  return MOE_ZC_OK;
+}
+
+int moe_zc_reserve(int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I) {
+  if (T < 0 || d <= 0 || N < 0 || Z < 0 || K < 1 || N + Z < 1 || K > N + Z)
+    return MOE_ZC_ERR_INVALID_ARG;
+  if (N > 0 && I <= 0) return MOE_ZC_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Ctx* c = nullptr;
+  int s = get_ctx(&c);
+  if (s != MOE_ZC_OK) return s;
+  return reserve_impl(*c, T, d, N, Z, K, N > 0 ? I : 128);
+}
+
+void moe_zc_release(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int prev = 0;
+  cudaGetDevice(&prev);
+  for (int dev = 0; dev < kMaxDevices; ++dev) {
+    Ctx& c = g_ctx[dev];
+    if (!c.init) continue;
+    cudaSetDevice(dev);
+    cudaDeviceSynchronize();
+    Buf* bufs[] = {&c.logits, &c.idx, &c.gate, &c.zsum, &c.slot, &c.cnt, &c.fill,
+                   &c.grp_off, &c.grp_ttp, &c.Xp, &c.H, &c.Y, &c.err};
+    for (Buf* b : bufs) {
+      if (b->p) cudaFree(b->p);
+      *b = Buf{};
+    }
+    if (c.done) cudaEventDestroy(c.done);
+    c = Ctx{};
+  }
+  cudaSetDevice(prev);
+}
+
+const char* moe_zc_status_string(int status) {
+  switch (status) {
+    case MOE_ZC_OK: return "ok";
+    case MOE_ZC_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ZC_ERR_UNSUPPORTED: return "unsupported size, alignment or device";
+    case MOE_ZC_ERR_CUDA: return "CUDA call failed";
+    case MOE_ZC_ERR_OOM: return "workspace allocation failed";
+    case MOE_ZC_ERR_TIMEOUT: return "device-side wait timed out";
+    case MOE_ZC_ERR_NO_RESULT: return "no forward has run on this device";
+    default: return "unknown status";
+  }
+}
+
+int moe_zc_profile(int32_t enable) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ZC_ERR_CUDA;
+  if (enable && g_prof.created && g_prof.device != dev) return MOE_ZC_ERR_UNSUPPORTED;
+  if (enable && !g_prof.created) {
+    for (int r = 0; r < kRing; ++r)
+      for (int i = 0; i <= kStages; ++i)
+        if (cudaEventCreate(&g_prof.ev[r][i]) != cudaSuccess) return MOE_ZC_ERR_CUDA;
+    g_prof.created = true;
+    g_prof.device = dev;
+  }
+  g_prof.on = enable != 0;
+  g_prof.n = 0;
+  return MOE_ZC_OK;
+}
+
+int moe_zc_profile_read(float* stage_ms, int32_t max_stages, int32_t* n_forwards) {
+  if (!stage_ms || !n_forwards || max_stages < 0) return MOE_ZC_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  *n_forwards = g_prof.n;
+  const int ns = max_stages < kStages ? max_stages : kStages;
+  for (int i = 0; i < ns; ++i) stage_ms[i] = 0.f;
+  if (g_prof.n == 0) return MOE_ZC_OK;
+  CK(cudaEventSynchronize(g_prof.ev[g_prof.n - 1][kStages]));
+  for (int r = 0; r < g_prof.n; ++r)
+    for (int i = 0; i < ns; ++i) {
+      float ms = 0.f;
+      CK(cudaEventElapsedTime(&ms, g_prof.ev[r][i], g_prof.ev[r][i + 1]));
+      stage_ms[i] += ms;
+    }
+  return MOE_ZC_OK;
+}
+
+const char* moe_zc_stage_name(int32_t i) {
+  return (i >= 0 && i < kStages) ? kStageNames[i] : nullptr;
+}
+
+void moe_zc_test_inject(int32_t fail_allocs, int64_t wait_limit) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_fail_allocs = fail_allocs > 0 ? fail_allocs : 0;
+  g_wait_ns_next = wait_limit > 0 ? wait_limit : 0;
+}
+
+}  // extern "C"

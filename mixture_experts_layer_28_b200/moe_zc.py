@@ -1,0 +1,193 @@
+"""ctypes binding of libmoe_zc.so (include/moe_zc.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  There is no
+fallback: if the library is missing or the tensors are not on a CUDA device,
+the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_zc.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "moe_zc.h")
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED = -2
+ERR_CUDA = -3
+ERR_OOM = -4
+ERR_TIMEOUT = -5
+ERR_NO_RESULT = -6
+
+
+class MoeZcError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m mixture_experts_layer_28_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+        L.moe_zc_forward.argtypes = [vp] * 6 + [i64, i32, i32, i32, i32, i32, vp, vp]
+        L.moe_zc_forward.restype = ctypes.c_int
+        L.moe_zc_forward_ex.argtypes = [vp] * 6 + [i64, i32, i32, i32, i32, i32, vp, vp, vp]
+        L.moe_zc_forward_ex.restype = ctypes.c_int
+        L.moe_zc_expert_load.argtypes = [vp]
+        L.moe_zc_expert_load.restype = ctypes.c_int
+        L.moe_zc_last_routing.argtypes = [vp, vp]
+        L.moe_zc_last_routing.restype = ctypes.c_int
+        L.moe_zc_last_expert.argtypes = [i32, i32, vp, vp, vp, vp]
+        L.moe_zc_last_expert.restype = ctypes.c_int
+        L.moe_zc_synchronize.argtypes = []
+        L.moe_zc_synchronize.restype = ctypes.c_int
+        L.moe_zc_reserve.argtypes = [i64, i32, i32, i32, i32, i32]
+        L.moe_zc_reserve.restype = ctypes.c_int
+        L.moe_zc_release.argtypes = []
+        L.moe_zc_release.restype = None
+        L.moe_zc_status_string.argtypes = [ctypes.c_int]
+        L.moe_zc_status_string.restype = ctypes.c_char_p
+        L.moe_zc_profile.argtypes = [i32]
+        L.moe_zc_profile.restype = ctypes.c_int
+        L.moe_zc_profile_read.argtypes = [vp, i32, vp]
+        L.moe_zc_profile_read.restype = ctypes.c_int
+        L.moe_zc_stage_name.argtypes = [i32]
+        L.moe_zc_stage_name.restype = ctypes.c_char_p
+        L.moe_zc_test_inject.argtypes = [i32, i64]
+        L.moe_zc_test_inject.restype = None
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().moe_zc_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != OK:
+        raise MoeZcError(status, what)
+
+
+def _dev_ptr(t: Optional[torch.Tensor], dtype, name: str) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def forward(x: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor,
+            W_gate: Optional[torch.Tensor], W_up: Optional[torch.Tensor],
+            W_down: Optional[torch.Tensor], N: int, Z: int, K: int,
+            out: Optional[torch.Tensor] = None,
+            logit_offset: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """moe_zc_forward(_ex) on CUDA tensors; returns out [T, d] bf16."""
+    T, d = x.shape
+    I = int(W_gate.shape[1]) if (W_gate is not None and N > 0) else 0
+    if out is None:
+        out = torch.empty_like(x)
+    bf = torch.bfloat16
+    args = [_dev_ptr(x, bf, "x"), _dev_ptr(W_r, bf, "W_r"), _dev_ptr(b, torch.float32, "b"),
+            _dev_ptr(W_gate, bf, "W_gate"), _dev_ptr(W_up, bf, "W_up"),
+            _dev_ptr(W_down, bf, "W_down"), T, d, N, Z, K, I]
+    o = _dev_ptr(out, bf, "out")
+    s = _stream_ptr(stream)
+    if logit_offset is None:
+        st = lib().moe_zc_forward(*args, o, s)
+    else:
+        st = lib().moe_zc_forward_ex(*args, _dev_ptr(logit_offset, torch.float32, "logit_offset"),
+                                     o, s)
+    _check(st, "moe_zc_forward")
+    return out
+
+
+def expert_load(E: int) -> np.ndarray:
+    counts = np.zeros(E, dtype=np.int32)
+    _check(lib().moe_zc_expert_load(counts.ctypes.data), "moe_zc_expert_load")
+    return counts
+
+
+def last_routing(T: int, K: int):
+    idx = np.zeros((T, K), dtype=np.int32)
+    gate = np.zeros((T, K), dtype=np.float32)
+    _check(lib().moe_zc_last_routing(idx.ctypes.data, gate.ctypes.data), "moe_zc_last_routing")
+    return idx, gate
+
+
+def last_expert(e: int, d: int, I: int, max_rows: int):
+    """(tokens int32 [n], H bf16 [n, I], Y bf16 [n, d]) of FFN expert e, last forward."""
+    n = ctypes.c_int32(0)
+    tokens = np.zeros(max_rows, dtype=np.int32)
+    H = torch.zeros(max_rows, I, dtype=torch.bfloat16)
+    Y = torch.zeros(max_rows, d, dtype=torch.bfloat16)
+    _check(lib().moe_zc_last_expert(e, max_rows, ctypes.byref(n), tokens.ctypes.data,
+                                    H.data_ptr(), Y.data_ptr()), "moe_zc_last_expert")
+    k = min(n.value, max_rows)
+    return tokens[:k], H[:k], Y[:k], n.value
+
+
+def synchronize() -> None:
+    _check(lib().moe_zc_synchronize(), "moe_zc_synchronize")
+
+
+def reserve(T: int, d: int, N: int, Z: int, K: int, I: int) -> None:
+    _check(lib().moe_zc_reserve(T, d, N, Z, K, I), "moe_zc_reserve")
+
+
+def release() -> None:
+    lib().moe_zc_release()
+
+
+STAGES = 8
+
+
+def profile(enable: bool) -> None:
+    _check(lib().moe_zc_profile(1 if enable else 0), "moe_zc_profile")
+
+
+def profile_read() -> tuple[dict, int]:
+    """({stage name: summed ms}, forwards recorded) since profile(True)."""
+    ms = np.zeros(STAGES, dtype=np.float32)
+    n = ctypes.c_int32(0)
+    _check(lib().moe_zc_profile_read(ms.ctypes.data, STAGES, ctypes.byref(n)),
+           "moe_zc_profile_read")
+    names = [lib().moe_zc_stage_name(i).decode() for i in range(STAGES)]
+    return dict(zip(names, ms.tolist())), n.value
+
+
+def test_inject(fail_allocs: int = 0, wait_limit_ns: int = 0) -> None:
+    lib().moe_zc_test_inject(fail_allocs, wait_limit_ns)
+
+
+def declared_symbols() -> list[str]:
+    """Function names declared in include/moe_zc.h."""
+    import re
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:int|void|const char\*)\s+(moe_zc_\w+)\s*\(", text, re.M)))

@@ -1,0 +1,85 @@
+"""The C-ABI library loads and exports what include/moe_zc.h declares, and its
+host-side argument checks return the documented status codes (no GPU needed:
+invalid arguments are rejected before any CUDA call)."""
+import ctypes
+
+import pytest
+
+from mixture_experts_layer_28_b200 import build as mb
+from mixture_experts_layer_28_b200 import moe_zc as mz
+
+
+@pytest.fixture(scope="module")
+def L():
+    mb.build()
+    return mz.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = mz.declared_symbols()
+    assert "moe_zc_forward" in names and "moe_zc_expert_load" in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in (mz.OK, mz.ERR_INVALID_ARG, mz.ERR_UNSUPPORTED, mz.ERR_CUDA, mz.ERR_OOM,
+                 mz.ERR_TIMEOUT, mz.ERR_NO_RESULT):
+        s = mz.status_string(code)
+        assert s and s != "unknown status"
+    assert mz.status_string(12345) == "unknown status"
+
+
+FAKE = 1 << 20   # an aligned, never-dereferenced address
+
+
+def _fwd(L, x=FAKE, W_r=FAKE, b=FAKE, Wg=FAKE, Wu=FAKE, Wd=FAKE, T=16, d=128, N=4, Z=2, K=2,
+         I=128, out=FAKE):
+    return L.moe_zc_forward(x, W_r, b, Wg, Wu, Wd, T, d, N, Z, K, I, out, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), mz.ERR_INVALID_ARG),
+    (dict(out=None), mz.ERR_INVALID_ARG),
+    (dict(b=None), mz.ERR_INVALID_ARG),
+    (dict(K=0), mz.ERR_INVALID_ARG),
+    (dict(K=7), mz.ERR_INVALID_ARG),              # K > E = 6
+    (dict(T=-1), mz.ERR_INVALID_ARG),
+    (dict(N=-1), mz.ERR_INVALID_ARG),
+    (dict(N=0, Z=0, K=1), mz.ERR_INVALID_ARG),    # empty expert pool
+    (dict(Wg=None), mz.ERR_INVALID_ARG),          # FFN experts need weights
+    (dict(I=0), mz.ERR_INVALID_ARG),
+    (dict(d=192), mz.ERR_UNSUPPORTED),            # d % 128
+    (dict(I=64), mz.ERR_UNSUPPORTED),             # I % 128
+    (dict(N=40, Z=0, K=33), mz.ERR_UNSUPPORTED),  # K > 32
+    (dict(N=1000, Z=100, K=2), mz.ERR_UNSUPPORTED),  # E > 1024
+    (dict(x=FAKE + 8), mz.ERR_UNSUPPORTED),       # misaligned
+    (dict(Wd=FAKE + 2), mz.ERR_UNSUPPORTED),
+])
+def test_argument_checks(L, kw, status):
+    assert _fwd(L, **kw) == status
+
+
+def test_zero_ffn_experts_need_no_weights(L):
+    # N = 0: weights may be NULL and I is ignored; only the device call can fail here
+    st = _fwd(L, Wg=None, Wu=None, Wd=None, N=0, Z=4, K=2, I=0)
+    assert st in (mz.OK, mz.ERR_CUDA, mz.ERR_UNSUPPORTED)
+
+
+def test_reserve_argument_checks(L):
+    assert L.moe_zc_reserve(-1, 128, 4, 2, 2, 128) == mz.ERR_INVALID_ARG
+    assert L.moe_zc_reserve(16, 128, 4, 2, 0, 128) == mz.ERR_INVALID_ARG
+    assert L.moe_zc_reserve(16, 128, 0, 0, 1, 128) == mz.ERR_INVALID_ARG
+
+
+def test_host_queries_reject_null(L):
+    assert L.moe_zc_expert_load(None) == mz.ERR_INVALID_ARG
+    assert L.moe_zc_last_expert(0, 4, None, None, None, None) == mz.ERR_INVALID_ARG
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(16, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        mz.forward(x, torch.zeros(6, 128, dtype=torch.bfloat16), torch.zeros(6), None, None, None,
+                   N=0, Z=6, K=2)

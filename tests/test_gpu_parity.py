@@ -1,0 +1,208 @@
+"""CUDA path (through the C ABI) against the fp64 oracle on seeded inputs.
+
+Small workloads are compared on every token; the full-size workloads on all
+tokens' routing and histogram, and on a seeded sample of output rows that the
+oracle computes one by one (rows are independent).  Tolerances: parity.py.
+"""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_28_b200 import moe_zc as mz
+from mixture_experts_layer_28_b200 import workloads as wl
+from oracle import moe_zc_ref as ref
+from parity import Case, check_expert_rows, check_output, check_routing
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _free_memory():
+    yield
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def _gpu_result(case):
+    out = case.run()
+    torch.cuda.synchronize()
+    mz.synchronize()
+    idx, gate = mz.last_routing(case.T, case.w.K)
+    cnt = mz.expert_load(case.w.E)
+    return out.float().cpu().numpy().astype(np.float64), idx, gate, cnt
+
+
+def _full_check(case, n_expert_checks=4):
+    out_g, idx, gate, cnt = _gpu_result(case)
+    r = case.oracle_routing()
+    ok = check_routing(case, r, idx, gate, cnt)
+    out_o = ref.forward_rows(case.x, r, case.expert)
+    err, rms = check_output(out_g[ok], out_o[ok])
+    hit = np.unique(r.idx[r.idx < case.w.N])
+    for e in hit[:n_expert_checks]:
+        check_expert_rows(case, int(e))
+    return err, rms
+
+
+def _sampled_check(case, n_rows=48, n_expert_checks=3):
+    out_g, idx, gate, cnt = _gpu_result(case)
+    r_all = case.oracle_routing()
+    ok = check_routing(case, r_all, idx, gate, cnt)
+    rows = wl.tokens_sample(case.T, n_rows, case.w.seed).numpy()
+    rows = rows[ok[rows]]
+    r = case.oracle_routing(rows=torch.from_numpy(rows))
+    out_o = ref.forward_rows(case.x[torch.from_numpy(rows)], r, case.expert)
+    err, rms = check_output(out_g[rows], out_o)
+    counts = np.bincount(r_all.idx[r_all.idx < case.w.N].ravel(), minlength=case.w.N)
+    # the busiest expert (several GEMM tiles) and a few lightly loaded ones
+    order = np.argsort(-counts)
+    picks = [int(order[0])] + [int(e) for e in order[::-1] if counts[e] > 0][:n_expert_checks - 1]
+    for e in picks:
+        check_expert_rows(case, e)
+    return err, rms
+
+
+def test_tiny_full():
+    _full_check(Case(wl.get("tiny")))
+
+
+def test_small_full():
+    _full_check(Case(wl.get("small")), n_expert_checks=6)
+
+
+@pytest.mark.parametrize("T", [1, 17, 300])
+def test_ragged_token_counts(T):
+    _full_check(Case(wl.get("small", T=T)))
+
+
+def test_zero_experts_absent():
+    """Z = 0: a plain softmax top-K MoE."""
+    _full_check(Case(wl.get("small", T=512, Z=0, K=4)))
+
+
+def test_no_ffn_experts():
+    """N = 0: every pick is an identity expert, no GEMM runs; out = (sum g) x."""
+    w = wl.get("tiny", N=0, Z=12, K=3)
+    case = Case(w)
+    out_g, idx, gate, cnt = _gpu_result(case)
+    r = case.oracle_routing()
+    check_routing(case, r, idx, gate, cnt)
+    check_output(out_g, r.zsum[:, None] * case.x.double().numpy())
+
+
+def test_all_picks_zero_experts_closed_form():
+    """Zero experts' bias +10: every pick is a zero expert, out = (sum g) x."""
+    w = wl.get("small", T=1000)
+    ri = wl.routing_inputs(w, 1000)
+    b = ri.b0.clone()
+    b[w.N:] += 10.0
+    case = Case(w, T=1000, bias=b)
+    out_g, idx, gate, cnt = _gpu_result(case)
+    assert (idx >= w.N).all()
+    assert cnt[: w.N].sum() == 0 and cnt.sum() == 1000 * w.K
+    r = case.oracle_routing()
+    check_routing(case, r, idx, gate, cnt)
+    check_output(out_g, r.zsum[:, None] * case.x.double().numpy())
+
+
+def test_one_expert_takes_every_token():
+    """FFN expert 3 gets all T tokens (several 256-token GEMM tiles)."""
+    w = wl.get("small", T=1100)
+    ri = wl.routing_inputs(w, 1100)
+    b = ri.b0.clone()
+    b[3] += 10.0
+    case = Case(w, T=1100, bias=b)
+    _, _, _, cnt = _gpu_result(case)
+    assert cnt[3] == 1100
+    _full_check(case)
+    assert check_expert_rows(case, 3, max_rows=1100) == 1100
+
+
+def test_dense_limit_k_equals_e():
+    w = wl.get("tiny", T=64, N=6, Z=2, K=8)
+    _full_check(Case(w), n_expert_checks=6)
+
+
+def test_minimum_widths():
+    w = wl.get("tiny", d=128, I=128, T=200)
+    _full_check(Case(w))
+
+
+def test_odd_weight_blocks():
+    """d = 384 and I = 384: the last 256-row weight block is half full."""
+    w = wl.get("tiny", d=384, I=384, T=260)
+    _full_check(Case(w))
+
+
+def test_empty_batch_is_noop():
+    w = wl.get("tiny")
+    case = Case(wl.get("tiny", T=1))
+    d = case.dev
+    x0 = torch.empty(0, w.d, dtype=torch.bfloat16, device="cuda")
+    out = torch.full((0, w.d), 1.0, dtype=torch.bfloat16, device="cuda")
+    ew = case.ew
+    mz.forward(x0, d["W_r"], d["b"], ew.W_gate, ew.W_up, ew.W_down, w.N, w.Z, w.K, out=out)
+    torch.cuda.synchronize()
+    assert (mz.expert_load(w.E) == 0).all()
+
+
+def test_deterministic_and_batch_split():
+    """Bitwise-equal out, idx, histogram on a rerun; a split batch gives the same rows."""
+    w = wl.get("small", T=1024)
+    case = Case(w)
+    o1, i1, g1, c1 = _gpu_result(case)
+    o2, i2, g2, c2 = _gpu_result(case)
+    assert np.array_equal(o1, o2) and np.array_equal(i1, i2) and np.array_equal(c1, c2)
+    assert np.array_equal(g1, g2)
+    d = case.dev
+    ew = case.ew
+    halves = []
+    for sl in (slice(0, 400), slice(400, 1024)):
+        halves.append(mz.forward(d["x"][sl].contiguous(), d["W_r"], d["b"], ew.W_gate, ew.W_up,
+                                 ew.W_down, w.N, w.Z, w.K).float().cpu().numpy())
+    assert np.array_equal(np.concatenate(halves).astype(np.float64), o1)
+
+
+def test_logit_offset_moves_routing():
+    w = wl.get("skewed40", T=2048, d=512, I=256)
+    _full_check(Case(w))
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill"])
+def test_full_size_longcat_shaped(name):
+    _sampled_check(Case(wl.get(name)))
+
+
+@pytest.mark.parametrize("name", ["skewed20", "skewed60"])
+def test_full_size_skewed(name):
+    _sampled_check(Case(wl.get(name)))
+
+
+def test_allocation_failure_reports_oom():
+    w = wl.get("tiny")
+    case = Case(w)
+    mz.release()
+    mz.test_inject(fail_allocs=1)
+    with pytest.raises(mz.MoeZcError) as ei:
+        case.run()
+    assert ei.value.status == mz.ERR_OOM
+    mz.test_inject(0, 0)
+    _full_check(case)          # recovers on the next call
+
+
+def test_device_wait_timeout_is_reported():
+    """Bounded device waits given a 1 ns limit give up, report TIMEOUT, and the
+    context stays usable for the next forward."""
+    w = wl.get("small", T=512)
+    case = Case(w)
+    case.run()
+    mz.synchronize()
+    mz.test_inject(0, 1)
+    case.run()
+    torch.cuda.synchronize()
+    with pytest.raises(mz.MoeZcError) as ei:
+        mz.synchronize()
+    assert ei.value.status == mz.ERR_TIMEOUT
+    _full_check(case)
