@@ -70,7 +70,19 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shape", default="",
+                    help="override workload sizes, e.g. T=4096,N=32,Z=16 (for profiling runs)")
     return ap.parse_args()
+
+
+def workload_of(args) -> wl.Workload:
+    kw = {}
+    for item in filter(None, args.shape.split(",")):
+        k, v = item.split("=")
+        kw[k.strip()] = int(v)
+    if kw:
+        kw["name"] = f"{args.workload}[{args.shape}]"
+    return wl.get(args.workload, **kw)
 
 
 def peaks():
@@ -406,7 +418,7 @@ def run_reference(args, dist, w):
 
 def main():
     args = parse()
-    w = wl.get(args.workload)
+    w = workload_of(args)
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         if rank != 0:

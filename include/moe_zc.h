@@ -66,7 +66,8 @@ typedef enum moe_zc_status {
 
 /*
  * Forward pass of the layer defined above ("Zero-computation experts").
- * T may be 0 (no work, returns MOE_ZC_OK).  N may be 0 (every pick is a zero
+ * T may be 0 (no work, returns MOE_ZC_OK; x and out may then be NULL, and
+ * the expert-load histogram of the call is all zero).  N may be 0 (every pick is a zero
  * expert) and Z may be 0 (plain softmax top-K MoE).  Requires d % 128 == 0,
  * I % 128 == 0, 1 <= K <= min(E, 32), E <= 1024, 16-byte aligned pointers.
  * W_gate/W_up/W_down may be NULL only when N == 0.

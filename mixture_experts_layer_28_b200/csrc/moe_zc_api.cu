@@ -170,7 +170,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 int check_args(const void* x, const void* W_r, const float* b, const void* W_gate,
                const void* W_up, const void* W_down, int64_t T, int32_t d, int32_t N, int32_t Z,
                int32_t K, int32_t I, const float* off, const void* out) {
-  if (!x || !W_r || !b || !out) return MOE_ZC_ERR_INVALID_ARG;
+  if (!W_r || !b) return MOE_ZC_ERR_INVALID_ARG;
+  if (T != 0 && (!x || !out)) return MOE_ZC_ERR_INVALID_ARG;   // T == 0: may be NULL
   if (T < 0 || N < 0 || Z < 0 || d <= 0) return MOE_ZC_ERR_INVALID_ARG;
   const int64_t E = static_cast<int64_t>(N) + Z;
   if (E < 1 || K < 1 || K > E) return MOE_ZC_ERR_INVALID_ARG;
@@ -180,7 +181,7 @@ int check_args(const void* x, const void* W_r, const float* b, const void* W_gat
   if (N > 0 && I % 128 != 0) return MOE_ZC_ERR_UNSUPPORTED;
   if (T * K + 16LL * N + 16 > (1LL << 31) - 1) return MOE_ZC_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(N) * (d > I ? d : I) > (1LL << 31) - 1) return MOE_ZC_ERR_UNSUPPORTED;
-  if (!aligned16(x) || !aligned16(W_r) || !aligned16(b) || !aligned16(out))
+  if (!aligned16(x) || !aligned16(W_r) || !aligned16(b) || !aligned16(out))  // NULL is aligned
     return MOE_ZC_ERR_UNSUPPORTED;
   if (off && !aligned16(off)) return MOE_ZC_ERR_UNSUPPORTED;
   if (N > 0 && (!aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down)))

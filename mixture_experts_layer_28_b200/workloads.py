@@ -81,9 +81,9 @@ WORKLOADS = {
 WORKLOADS = {k: replace(w, delta=_DELTA.get(k, 0.0)) for k, w in WORKLOADS.items()}
 
 
-def get(name: str, **overrides) -> Workload:
+def get(workload: str, **overrides) -> Workload:
     """The named workload, optionally with fields replaced (e.g. T=512)."""
-    return replace(WORKLOADS[name], **overrides)
+    return replace(WORKLOADS[workload], **overrides)
 
 
 @dataclass

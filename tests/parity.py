@@ -5,8 +5,11 @@ Tolerances:
   * routing -- bit-exact expert sets and an exact histogram on every token
     whose K-th and (K+1)-th biased scores (fp64 oracle) differ by at least
     TIE = 1e-5; for the rest (near-ties, where both choices are correct) the
-    GPU's picks must be a valid top-K within TIE.  Gates: fp32 softmax vs
-    fp64, rtol 1e-5.
+    GPU's picks must be a valid top-K within TIE.  Gates: rtol 1e-4.  A
+    gate's relative error is about its logit's absolute error (softmax), and
+    the logits are fp32 sums of d bf16 products accumulated by the tensor
+    cores (d = 6144: ~2e-5 measured).  That is far below what could move a
+    pick: s = p + b with p ~ 1e-3 moves by ~1e-8, against the 1e-5 margin.
   * output -- the contract max|err| <= 2e-2 (1 + |ref|), and, because that
     bound is loose at these magnitudes (|out| ~ 1e-2..1), also
     |err| <= 5u (|ref| + rms(ref)) elementwise, u = 2^-8 the unit roundoff of
@@ -77,7 +80,7 @@ def check_routing(case: Case, r: ref.Routing, idx_g, gate_g, cnt_g):
     # gates, matched by expert
     og = np.take_along_axis(r.gate, np.argsort(r.idx, 1), 1)
     gg = np.take_along_axis(gate_g.astype(np.float64), np.argsort(idx_g, 1), 1)
-    np.testing.assert_allclose(gg[ok], og[ok], rtol=1e-5, atol=1e-9)
+    np.testing.assert_allclose(gg[ok], og[ok], rtol=1e-4, atol=1e-9)
     # histogram: exact against the GPU's own picks, and against the oracle
     # once near-tie tokens are taken out of both
     assert np.array_equal(cnt_g, np.bincount(idx_g.ravel(), minlength=E))

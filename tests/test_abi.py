@@ -40,6 +40,7 @@ def _fwd(L, x=FAKE, W_r=FAKE, b=FAKE, Wg=FAKE, Wu=FAKE, Wd=FAKE, T=16, d=128, N=
 
 @pytest.mark.parametrize("kw,status", [
     (dict(x=None), mz.ERR_INVALID_ARG),
+    (dict(W_r=None), mz.ERR_INVALID_ARG),
     (dict(out=None), mz.ERR_INVALID_ARG),
     (dict(b=None), mz.ERR_INVALID_ARG),
     (dict(K=0), mz.ERR_INVALID_ARG),
