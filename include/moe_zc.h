@@ -148,6 +148,39 @@ int moe_zc_profile_read(float* stage_ms, int32_t max_stages, int32_t* n_forwards
 const char* moe_zc_stage_name(int32_t i);
 
 /*
+ * Routing without any device allocation.  The write-up has no counterpart to
+ * this entry point: it exists for callers that cannot let a library call
+ * cudaMalloc while they run -- e.g. a server that hands all device memory to
+ * its own pool at start-up, or a process under a hard device-memory cap --
+ * because a late allocation can fail, take memory promised elsewhere, or
+ * synchronise the device mid-step.
+ *
+ * It computes exactly the routing part of moe_zc_forward_ex (same kernels):
+ * idx (device int32 [T*K], picks in descending biased score), gate (device
+ * float [T*K], unbiased softmax probabilities) and counts (device int32 [E],
+ * expert-load histogram, cleared by the call).  x, W_r, b, logit_offset
+ * (may be NULL) as for moe_zc_forward_ex.  dev_status: device int32 that the
+ * call clears and the kernels set non-zero if a bounded wait runs out; NULL
+ * uses a word of the library's own array.  Asynchronous on `stream`.
+ *
+ * Its scratch (fp32 logits and zero-gate sums) is one fixed array of
+ * MOE_ZC_NOALLOC_SCRATCH_BYTES in the library image, held by every GPU that
+ * loads the library until the process exits; sizes need
+ * 256*ceil(T*E*4/256) + 256*ceil(T*4/256) + 256 <= that, else the call
+ * returns MOE_ZC_ERR_UNSUPPORTED and launches nothing (e.g. E = 768 allows
+ * T <= 1363).  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  All calls share the array and it keeps the
+ * last call's contents, so calls whose GPU work overlaps (two streams or two
+ * threads) race: serialise them.
+ */
+#define MOE_ZC_NOALLOC_SCRATCH_BYTES (4u << 20)
+int moe_zc_route_noalloc(const void* x, const void* W_r, const float* b,
+                         const float* logit_offset, int64_t T, int32_t d, int32_t N,
+                         int32_t Z, int32_t K, int32_t* idx, float* gate, int32_t* counts,
+                         int32_t* dev_status, void* stream);
+
+/*
  * Test hook for the error paths: make the next n workspace allocations fail
  * (MOE_ZC_ERR_OOM), and/or make every bounded device wait of the next forward
  * give up after `wait_limit` nanoseconds (0 = the normal 2 s), so that the

@@ -70,6 +70,9 @@ def lib() -> ctypes.CDLL:
         L.moe_zc_profile_read.restype = ctypes.c_int
         L.moe_zc_stage_name.argtypes = [i32]
         L.moe_zc_stage_name.restype = ctypes.c_char_p
+        L.moe_zc_route_noalloc.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32,
+                                           vp, vp, vp, vp, vp]
+        L.moe_zc_route_noalloc.restype = ctypes.c_int
         L.moe_zc_test_inject.argtypes = [i32, i64]
         L.moe_zc_test_inject.restype = None
         _lib = L
@@ -163,6 +166,26 @@ def reserve(T: int, d: int, N: int, Z: int, K: int, I: int) -> None:
 
 def release() -> None:
     lib().moe_zc_release()
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def route_noalloc(x: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor, N: int, Z: int, K: int,
+                  idx: torch.Tensor, gate: torch.Tensor, counts: torch.Tensor,
+                  logit_offset: Optional[torch.Tensor] = None,
+                  status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """moe_zc_route_noalloc: routing into caller-owned device tensors
+    (idx int32 [T, K], gate fp32 [T, K], counts int32 [E], status int32 [1]),
+    with no device allocation by the library."""
+    T, d = x.shape
+    st = lib().moe_zc_route_noalloc(
+        _dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(W_r, torch.bfloat16, "W_r"),
+        _dev_ptr(b, torch.float32, "b"), _dev_ptr(logit_offset, torch.float32, "logit_offset"),
+        T, d, N, Z, K, _dev_ptr(idx, torch.int32, "idx"), _dev_ptr(gate, torch.float32, "gate"),
+        _dev_ptr(counts, torch.int32, "counts"), _dev_ptr(status, torch.int32, "status"),
+        _stream_ptr(stream))
+    _check(st, "moe_zc_route_noalloc")
 
 
 STAGES = 8
