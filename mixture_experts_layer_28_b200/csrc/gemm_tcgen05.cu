@@ -38,6 +38,8 @@ namespace {
 constexpr long long DRAIN_NS = 2000000000LL;  // bound of the drain waits at exit
 
 struct Tile {
+  int k0, k1;   // k-step range of this tile
+  int split;    // router: K slice index
   int g;        // group (expert)
   int m;        // weight block
   int tok0;     // first token of the tile inside its group
@@ -51,13 +53,24 @@ struct Tile {
 
 template <int MODE>
 __device__ __forceinline__ int total_tiles(const GemmParams& p) {
-  if (MODE == MODE_ROUTER) return ((p.T + GEMM_BN - 1) / GEMM_BN) * p.mblocks;
+  if (MODE == MODE_ROUTER)
+    return ((p.T + GEMM_BN - 1) / GEMM_BN) * p.mblocks * (p.ksplit > 1 ? p.ksplit : 1);
   return __ldg(p.grp_ttp + p.G) * p.mblocks;
 }
 
 template <int MODE>
 __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   Tile tl;
+  tl.split = 0;
+  tl.k0 = 0;
+  tl.k1 = p.ksteps;
+  if (MODE == MODE_ROUTER && p.ksplit > 1) {
+    const int per = ((p.T + GEMM_BN - 1) / GEMM_BN) * p.mblocks;
+    tl.split = t / per;
+    t -= tl.split * per;
+    tl.k0 = static_cast<int>(static_cast<long long>(p.ksteps) * tl.split / p.ksplit);
+    tl.k1 = static_cast<int>(static_cast<long long>(p.ksteps) * (tl.split + 1) / p.ksplit);
+  }
   const int tt = t / p.mblocks;
   tl.m = t - tt * p.mblocks;
   int j;
@@ -87,10 +100,10 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
     tl.a1_row = tl.a0_row;                           // W_up rows
     tl.has_a1 = true;
   } else {
-    const int r = tl.m * 2 * GEMM_BM;
+    const int r = tl.m * (p.single_a ? 1 : 2) * GEMM_BM;
     tl.a0_row = tl.g * p.a_rows + r;
     tl.a1_row = tl.a0_row + GEMM_BM;
-    tl.has_a1 = (r + GEMM_BM) < p.a_rows;
+    tl.has_a1 = !p.single_a && (r + GEMM_BM) < p.a_rows;
   }
   return tl;
 }
@@ -150,7 +163,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       const int nbox = (tl.nmma + GEMM_B_BOX_ROWS - 1) / GEMM_B_BOX_ROWS;
       const uint32_t bytes = GEMM_A_BYTES * (tl.has_a1 ? 2 : 1) +
                              nbox * GEMM_B_BOX_ROWS * GEMM_BK * 2;
-      for (int ks = 0; ks < p.ksteps; ++ks) {
+      for (int ks = tl.k0; ks < tl.k1; ++ks) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1, p.wait_ns, p.err)) {
           abort_sh = 1;
           break;
@@ -186,7 +199,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       tc_fence_after();
       const uint32_t idesc = idesc_bf16_f32(GEMM_BM, tl.nmma);
       bool ok = true;
-      for (int ks = 0; ks < p.ksteps; ++ks) {
+      for (int ks = tl.k0; ks < tl.k1; ++ks) {
         if (!mbar_wait(&full_bar[stage], phase, p.wait_ns, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = smem_u32(smem + stage * GEMM_STAGE_BYTES);
@@ -195,7 +208,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         const uint64_t bd = smem_desc_sw128(st + 2 * GEMM_A_BYTES);
 #pragma unroll
         for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-          const uint32_t acc = (ks | kk) != 0;
+          const uint32_t acc = (ks != tl.k0 || kk != 0) ? 1u : 0u;
           umma_bf16(tmem, a0 + 2 * kk, bd + 2 * kk, idesc, acc);
           if (tl.has_a1) umma_bf16(tmem + 256, a1 + 2 * kk, bd + 2 * kk, idesc, acc);
         }
@@ -227,8 +240,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         if (tl.has_a1) tmem_ld16(tq + 256 + c0, r1);
         tmem_ld_wait();
         if (MODE == MODE_ROUTER) {
-          float* out = static_cast<float*>(p.out);
-          const int e0 = tl.m * 2 * GEMM_BM + row_in_blk;
+          float* out = static_cast<float*>(p.out) + tl.split * p.split_stride;
+          const int e0 = tl.m * (p.single_a ? 1 : 2) * GEMM_BM + row_in_blk;
           const int e1 = e0 + GEMM_BM;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -253,7 +266,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
           }
         } else {
           __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-          const int f0 = tl.m * 2 * GEMM_BM + row_in_blk;
+          const int f0 = tl.m * (p.single_a ? 1 : 2) * GEMM_BM + row_in_blk;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int c = tl.tok0 + c0 + i;

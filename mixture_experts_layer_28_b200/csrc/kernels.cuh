@@ -36,6 +36,10 @@ struct GemmParams {
   int G;
   int T;                  // MODE_ROUTER: tokens
   int ksteps;             // contraction length / GEMM_BK
+  int ksplit;             // MODE_ROUTER: K split into this many slices (0 or 1: none);
+                          // slice s writes its partial sums to out + s * split_stride
+  long long split_stride;
+  int single_a;           // MODE_ROUTER/MODE_DOWN: 1 = one 128-row A block per tile (no pair)
   int mblocks;            // tiles along the weight rows of one group
   int a_rows;             // weight rows per group: E (router), I (gate/up), d (down)
   void* out;              // fp32 logits [T, E] | bf16 H [rows, I] | bf16 Y [rows, d]
@@ -50,9 +54,11 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
 
 // ------------------------------------------------------------------ router
 // softmax over E logits (+offset), + bias, top-K, zero-gate sums, histogram.
+// The logits may come as `splits` partial sums [splits][T][E], added in
+// slice order.
 cudaError_t launch_route(const float* logits, const float* b, const float* offset, int64_t T,
                          int E, int N, int K, int* idx, float* gate, float* zsum, int* cnt,
-                         cudaStream_t stream);
+                         cudaStream_t stream, int splits = 1);
 
 // ------------------------------------------------------------------ dispatch
 cudaError_t launch_scan(const int* cnt, int N, int* grp_off, int* grp_ttp, int* fill,

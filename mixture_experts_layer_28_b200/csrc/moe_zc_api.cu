@@ -139,6 +139,30 @@ int get_ctx(Ctx** out) {
   return MOE_ZC_OK;
 }
 
+// Router GEMM layout for T tokens: with few token tiles (decode) each tile is
+// one 128-row block of W_r and K is split into slices so that the tiles fill
+// the SMs, each slice at least 4 k-steps (256 of d); otherwise tiles pair two
+// blocks and K is not split.
+struct RouterPlan {
+  int single_a, mblocks, splits;
+  int64_t tiles;   // token tiles x weight blocks (per slice)
+};
+RouterPlan router_plan(int64_t T, int E, int ksteps, int sms) {
+  RouterPlan rp{0, (E + 2 * GEMM_BM - 1) / (2 * GEMM_BM), 1, 0};
+  const int64_t ttiles = (T + GEMM_BN - 1) / GEMM_BN;
+  rp.tiles = ttiles * rp.mblocks;
+  if (rp.tiles > 0 && rp.tiles < sms / 2) {
+    rp.single_a = 1;
+    rp.mblocks = (E + GEMM_BM - 1) / GEMM_BM;
+    rp.tiles = ttiles * rp.mblocks;
+    int64_t s = sms / rp.tiles;
+    const int64_t cap = ksteps / 4 > 0 ? ksteps / 4 : 1;
+    if (s > cap) s = cap;
+    rp.splits = s < 1 ? 1 : static_cast<int>(s);
+  }
+  return rp;
+}
+
 int reserve_impl(Ctx& c, int64_t T, int d, int N, int Z, int K, int I) {
   const int64_t E = static_cast<int64_t>(N) + Z;
   const int64_t pairs = T * K;
@@ -147,7 +171,12 @@ int reserve_impl(Ctx& c, int64_t T, int d, int N, int Z, int K, int I) {
   const bool fresh_err = c.err.p == nullptr;
   if ((s = ensure(c, c.err, sizeof(int))) != MOE_ZC_OK) return s;
   if (fresh_err && cudaMemset(c.err.p, 0, sizeof(int)) != cudaSuccess) return MOE_ZC_ERR_CUDA;
-  if ((s = ensure(c, c.logits, static_cast<size_t>(T * E) * sizeof(float))) != MOE_ZC_OK) return s;
+  {
+    const RouterPlan rp = router_plan(T, static_cast<int>(E), d / GEMM_BK, c.sms);
+    if ((s = ensure(c, c.logits, static_cast<size_t>(T * E * rp.splits) * sizeof(float))) !=
+        MOE_ZC_OK)
+      return s;
+  }
   if ((s = ensure(c, c.idx, static_cast<size_t>(pairs) * sizeof(int))) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.gate, static_cast<size_t>(pairs) * sizeof(float))) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.slot, static_cast<size_t>(pairs) * sizeof(int))) != MOE_ZC_OK) return s;
@@ -247,19 +276,27 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     pr.G = 1;
     pr.T = static_cast<int>(T);
     pr.ksteps = d / GEMM_BK;
-    pr.mblocks = (E + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
     pr.a_rows = E;
     pr.out = c.logits.p;
     pr.out_ld = E;
     pr.err = err;
     pr.wait_ns = wait_ns;
-    const int64_t rtiles = ((T + GEMM_BN - 1) / GEMM_BN) * pr.mblocks;
+    // Few token tiles (decode): single blocks and K slices so that every SM
+    // streams a part of W_r; the slices' partial logits are summed in slice
+    // order by the route kernel.
+    const RouterPlan rp = router_plan(T, E, pr.ksteps, c.sms);
+    pr.mblocks = rp.mblocks;
+    pr.single_a = rp.single_a;
+    const int splits = rp.splits;
+    pr.ksplit = splits;
+    pr.split_stride = T * E;
+    const int64_t rgrid = rp.tiles * splits;
     CK(launch_gemm(MODE_ROUTER, mWr, mWr, mX, pr,
-                   static_cast<int>(rtiles < c.sms ? rtiles : c.sms), st));
+                   static_cast<int>(rgrid < c.sms ? rgrid : c.sms), st));
     rec.mark(1);
     // 2  route
     CK(launch_route(static_cast<const float*>(c.logits.p), b, off, T, E, N, K, idx, gate, zsum,
-                    cnt, st));
+                    cnt, st, splits));
     rec.mark(2);
     if (N > 0) {
       // 3-5  dispatch

@@ -8,7 +8,11 @@
 //
 //   p_t = softmax(logits_t + offset)      over all E experts, fp32
 //   s_t = p_t + b                         selection score
-//   picks: K rounds of a warp-wide argmax of s (ties -> lower expert index)
+//   picks: K rounds of a warp-wide argmax of s (ties -> lower expert index):
+//          scores become order-preserving uint32 keys, each lane keeps its
+//          best slot, a round is two warp reductions (max key, then min
+//          index among the lanes holding it), and only the winning lane
+//          rescans its slots
 //   gate_{t,k} = p_t at pick k            (unbiased, not renormalised)
 //   zsum_t     = sum of the gates of zero-expert picks (index >= N)
 //
@@ -26,82 +30,122 @@ namespace {
 
 constexpr int ROUTE_WARPS = 8;
 
+// fp32 -> uint32 with the same order (larger float -> larger key); the key 0
+// is below every float's key and marks a taken or absent expert.
+__device__ __forceinline__ uint32_t order_key(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Best key of this lane's VPL slots (lower slot on equal keys), as a tree so
+// the dependency depth is log2(VPL).
+template <int VPL>
+__device__ __forceinline__ void lane_best(const uint32_t (&key)[VPL], const float (&p)[VPL],
+                                          uint32_t& bk, int& bi, float& bp) {
+  uint32_t k[VPL];
+  int ix[VPL];
+  float pv[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) { k[i] = key[i]; ix[i] = i; pv[i] = p[i]; }
+#pragma unroll
+  for (int w = 1; w < VPL; w <<= 1) {
+#pragma unroll
+    for (int i = 0; i + w < VPL; i += 2 * w) {
+      if (k[i + w] > k[i]) { k[i] = k[i + w]; ix[i] = ix[i + w]; pv[i] = pv[i + w]; }
+    }
+  }
+  bk = k[0];
+  bi = ix[0];
+  bp = pv[0];
+}
+
 template <int VPL>  // logits per lane: E <= 32 * VPL
 __global__ void __launch_bounds__(ROUTE_WARPS * 32)
 route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
              const float* __restrict__ offset, int64_t T, int E, int N, int K,
              int* __restrict__ idx, float* __restrict__ gate, float* __restrict__ zsum,
-             int* __restrict__ cnt) {
+             int* __restrict__ cnt, int splits) {
   extern __shared__ int hist[];  // [E]
   for (int j = threadIdx.x; j < E; j += blockDim.x) hist[j] = 0;
   __syncthreads();
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int64_t split_stride = T * E;
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * ROUTE_WARPS + warp; t < T;
        t += static_cast<int64_t>(gridDim.x) * ROUTE_WARPS) {
     const float* lrow = logits + t * E;
-    float p[VPL], s[VPL];
+    // logits: the router GEMM's K slices summed in slice order
+    float l[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int j = lane + 32 * i;
+      l[i] = (j < E) ? lrow[j] : 0.f;
+    }
+    for (int sp = 1; sp < splits; ++sp) {
+      const float* srow = lrow + sp * split_stride;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int j = lane + 32 * i;
+        if (j < E) l[i] += srow[j];
+      }
+    }
     float mx = -FLT_MAX;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int j = lane + 32 * i;
-      float l = -FLT_MAX;
       if (j < E) {
-        l = lrow[j];
-        if (offset) l += offset[j];
+        if (offset) l[i] += offset[j];
+        mx = fmaxf(mx, l[i]);
       }
-      p[i] = l;
-      mx = fmaxf(mx, l);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float p[VPL];
     float sum = 0.f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int j = lane + 32 * i;
-      p[i] = (j < E) ? expf(p[i] - mx) : 0.f;
+      p[i] = (j < E) ? expf(l[i] - mx) : 0.f;
       sum += p[i];
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float inv = 1.0f / sum;
+    uint32_t key[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int j = lane + 32 * i;
-      p[i] *= inv;
+      p[i] = p[i] / sum;
       // A NaN score (only from non-finite logits) ranks below every real
       // score but above a taken or absent expert, so each round still picks
       // a valid index.
       const float sc = p[i] + (j < E ? bias[j] : 0.f);
-      s[i] = (j < E) ? (sc == sc ? sc : -FLT_MAX) : -INFINITY;
+      key[i] = (j < E) ? order_key(sc == sc ? sc : -FLT_MAX) : 0u;
     }
 
+    uint32_t bk;
+    int bi;
+    float bp;
+    lane_best<VPL>(key, p, bk, bi, bp);
     float zs = 0.f;
     for (int k = 0; k < K; ++k) {
-      // best of this lane (values visited in increasing index: strict > keeps the lower one)
-      float bs = -INFINITY, bp = 0.f;
-      int bj = INT_MAX;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        if (s[i] > bs) { bs = s[i]; bj = lane + 32 * i; bp = p[i]; }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-        const float op = __shfl_xor_sync(0xffffffffu, bp, o);
-        if (os > bs || (os == bs && oj < bj)) { bs = os; bj = oj; bp = op; }
-      }
-      // remove the winner from its lane
-#pragma unroll
-      for (int i = 0; i < VPL; ++i)
-        if (lane + 32 * i == bj) s[i] = -INFINITY;
-      if (bj >= N) zs += bp;
+      // the largest score; among equal scores the lowest expert index
+      const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t cand = (bk == mk) ? static_cast<uint32_t>(lane + 32 * bi) : 0xffffffffu;
+      const int jw = static_cast<int>(__reduce_min_sync(0xffffffffu, cand));
+      const float pw = __shfl_sync(0xffffffffu, bp, jw & 31);
+      if (jw >= N) zs += pw;
       if (lane == 0) {
-        idx[t * K + k] = bj;
-        gate[t * K + k] = bp;
-        atomicAdd(&hist[bj], 1);
+        idx[t * K + k] = jw;
+        gate[t * K + k] = pw;
+        atomicAdd(&hist[jw], 1);
+      }
+      if (lane == (jw & 31)) {
+        const int iw = jw >> 5;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+          if (i == iw) key[i] = 0u;
+        lane_best<VPL>(key, p, bk, bi, bp);
       }
     }
     if (lane == 0) zsum[t] = zs;
@@ -114,7 +158,7 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
 template <int VPL>
 cudaError_t launch_route_vpl(const float* logits, const float* b, const float* offset, int64_t T,
                              int E, int N, int K, int* idx, float* gate, float* zsum, int* cnt,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, int splits) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -123,7 +167,7 @@ cudaError_t launch_route_vpl(const float* logits, const float* b, const float* o
   const int64_t cap = static_cast<int64_t>(sms) * 8;
   const int grid = static_cast<int>(want < cap ? want : cap);
   route_kernel<VPL><<<grid, ROUTE_WARPS * 32, E * sizeof(int), stream>>>(
-      logits, b, offset, T, E, N, K, idx, gate, zsum, cnt);
+      logits, b, offset, T, E, N, K, idx, gate, zsum, cnt, splits);
   return cudaGetLastError();
 }
 
@@ -131,12 +175,24 @@ cudaError_t launch_route_vpl(const float* logits, const float* b, const float* o
 
 cudaError_t launch_route(const float* logits, const float* b, const float* offset, int64_t T,
                          int E, int N, int K, int* idx, float* gate, float* zsum, int* cnt,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, int splits) {
   if (T <= 0) return cudaSuccess;
-  if (E <= 128) return launch_route_vpl<4>(logits, b, offset, T, E, N, K, idx, gate, zsum, cnt, stream);
-  if (E <= 256) return launch_route_vpl<8>(logits, b, offset, T, E, N, K, idx, gate, zsum, cnt, stream);
-  if (E <= 512) return launch_route_vpl<16>(logits, b, offset, T, E, N, K, idx, gate, zsum, cnt, stream);
-  return launch_route_vpl<32>(logits, b, offset, T, E, N, K, idx, gate, zsum, cnt, stream);
+  if (splits < 1) splits = 1;
+#define MOEZC_ROUTE(V)                                                                     \
+  if (E <= 32 * (V))                                                                       \
+    return launch_route_vpl<V>(logits, b, offset, T, E, N, K, idx, gate, zsum, cnt, stream, \
+                               splits);
+  MOEZC_ROUTE(1)
+  MOEZC_ROUTE(2)
+  MOEZC_ROUTE(3)
+  MOEZC_ROUTE(4)
+  MOEZC_ROUTE(6)
+  MOEZC_ROUTE(8)
+  MOEZC_ROUTE(12)
+  MOEZC_ROUTE(16)
+  MOEZC_ROUTE(24)
+#undef MOEZC_ROUTE
+  return launch_route_vpl<32>(logits, b, offset, T, E, N, K, idx, gate, zsum, cnt, stream, splits);
 }
 
 }  // namespace moezc
