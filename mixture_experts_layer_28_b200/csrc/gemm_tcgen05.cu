@@ -21,12 +21,13 @@
 // against up to 256 tokens, giving two 128 x N fp32 accumulators in TMEM
 // (columns 0..255 and 256..511).
 //
-// Persistent, warp-specialised CTA (256 threads, one per SM):
+// Persistent, warp-specialised CTA (384 threads, one per SM):
 //   warp 0      TMA producer: A blocks [128 x 64] and B boxes [32 x 64],
 //               128-byte swizzle, into a 3-stage shared-memory ring
 //   warp 1      MMA issuer: tcgen05.mma kind::f16, commits free the stage
 //   warp 2      TMEM allocator
-//   warps 4..7  epilogue: tcgen05.ld -> fp32 math -> global stores
+//   warps 4..11 epilogue: tcgen05.ld -> fp32 math -> shared staging ->
+//               coalesced 16-byte global stores
 // Every wait is time-bounded (ptx.cuh); on running out the CTA drains its
 // in-flight copies and MMAs, frees TMEM and returns with the error flag set.
 #include "kernels.cuh"
@@ -108,7 +109,60 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   return tl;
 }
 
-__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
+// One warp's 32 features x ncol tokens of fp32 results (thread = feature,
+// v[i] = token i) -> bf16 rows out[i * ld + 0..31] for i < rows, through a
+// [32 tokens][32 features] staging tile: 2-byte shared stores by feature,
+// then 16-byte loads and global stores, four lanes per 64-byte row.
+__device__ __forceinline__ void stage_store_bf16(uint8_t* stg, int lane, const uint32_t (&v)[32],
+                                                 int ncol, int rows, __nv_bfloat16* out,
+                                                 int64_t ld) {
+  __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(stg);
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (i < ncol) st[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = (lane >> 2) + 8 * k;
+    const int part = lane & 3;
+    if (r < rows) {
+      const uint4 val = *reinterpret_cast<const uint4*>(stg + r * 64 + part * 16);
+      *reinterpret_cast<uint4*>(out + r * ld + part * 8) = val;
+    }
+  }
+  __syncwarp();
+}
+
+// fp32 variant for the router's logits: features ebase + 0..31 of rows
+// tok_base + i, features >= E dropped; 128-byte rows, eight lanes per row.
+__device__ __forceinline__ void stage_store_f32(uint8_t* stg, int lane, const uint32_t (&v)[32],
+                                                int ncol, int rows, float* out, int tok_base,
+                                                int ld, int ebase, int E) {
+  uint32_t* st = reinterpret_cast<uint32_t*>(stg);
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (i < ncol) st[i * 32 + lane] = v[i];
+  __syncwarp();
+  const bool vec = (ld % 4 == 0) && (ebase + 32 <= E);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = (lane >> 3) + 4 * k;
+    const int part = lane & 7;
+    if (r < rows) {
+      float* dst = out + static_cast<int64_t>(tok_base + r) * ld + ebase + part * 4;
+      const uint4 val = *reinterpret_cast<const uint4*>(stg + r * 128 + part * 16);
+      if (vec) {
+        *reinterpret_cast<uint4*>(dst) = val;
+      } else {
+        const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (ebase + part * 4 + e < E) dst[e] = __uint_as_float(w[e]);
+      }
+    }
+  }
+  __syncwarp();
+}
 
 template <int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
@@ -134,7 +188,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_full_bar, 1);
-    mbar_init(&acc_empty_bar, 128);
+    mbar_init(&acc_empty_bar, GEMM_EPI_THREADS);
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
     fence_mbar_init();
@@ -142,6 +196,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB);
   }
+  __syncwarp();
   if (warp == 2) {
     tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
@@ -152,7 +207,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   const uint32_t tmem = tmem_base_sh;
   const int ntiles = total_tiles<MODE>(p);
 
-  if (warp == 0 && lane == 0) {
+  // Single-thread roles run on lane 0; the other lanes of their warp wait at
+  // a __syncwarp so that every warp reaches the final CTA barrier converged.
+  if (warp == 0) {
+   if (lane == 0) {
     // ------------------------------------------------------------ producer
     int stage = 0;
     uint32_t phase = 0;
@@ -185,7 +243,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     // Drain: every copy this thread started must land before the CTA exits.
     for (int s = 0; s < GEMM_STAGES; ++s)
       if (armed & (1u << s)) mbar_wait(&full_bar[s], (last_par >> s) & 1, DRAIN_NS, p.err);
-  } else if (warp == 1 && lane == 0) {
+   }
+   __syncwarp();
+  } else if (warp == 1) {
+   if (lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     int stage = 0;
     uint32_t phase = 0;
@@ -221,11 +282,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     // Drain: all MMAs issued by this thread finish before TMEM is freed.
     umma_commit(&drain_bar);
     mbar_wait(&drain_bar, 0, DRAIN_NS, p.err);
+   }
+   __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;                 // TMEM lane quadrant
-    const int row_in_blk = q * 32 + lane;   // weight row inside an A block
+    // Eight warps: warp w drains TMEM lanes (w % 4) * 32 .. +31 (the quadrant
+    // its warp id may access) and every other 32-column chunk of the tile
+    // (half = 0 or 1).  Each chunk goes TMEM -> registers (one wait per
+    // chunk) -> math -> a per-warp staging tile in shared memory -> 16-byte
+    // coalesced global stores, one output row of 64 (bf16) or 128 (fp32)
+    // bytes per 4 or 8 lanes.
+    const int q = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const int row_in_blk = q * 32 + lane;
     const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    uint8_t* stg = smem + GEMM_STAGES * GEMM_STAGE_BYTES + (warp - 4) * GEMM_STG_BYTES;
     int local = 0;
     for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x, ++local) {
       const Tile tl = decode_tile<MODE>(p, t);
@@ -234,53 +305,52 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         break;
       }
       tc_fence_after();
-      for (int c0 = 0; c0 < tl.nmma; c0 += 16) {
-        uint32_t r0[16], r1[16];
-        tmem_ld16(tq + c0, r0);
-        if (tl.has_a1) tmem_ld16(tq + 256 + c0, r1);
+      for (int c0 = half * 32; c0 < tl.nmma; c0 += 64) {
+        const bool wide = c0 + 32 <= tl.nmma;   // 32 columns, else 16
+        uint32_t r0[32], r1[32];
+        tmem_ld16(tq + c0, *reinterpret_cast<uint32_t(*)[16]>(&r0[0]));
+        if (wide) tmem_ld16(tq + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r0[16]));
+        if (tl.has_a1) {
+          tmem_ld16(tq + 256 + c0, *reinterpret_cast<uint32_t(*)[16]>(&r1[0]));
+          if (wide) tmem_ld16(tq + 256 + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r1[16]));
+        }
         tmem_ld_wait();
+        const int ncol = wide ? 32 : 16;
+        const int tok_base = tl.tok0 + c0;              // token index in group of column 0
+        const int rows = min(ncol, tl.count - tok_base);  // valid output rows
         if (MODE == MODE_ROUTER) {
+          const int ebase = tl.m * (p.single_a ? 1 : 2) * GEMM_BM + q * 32;
           float* out = static_cast<float*>(p.out) + tl.split * p.split_stride;
-          const int e0 = tl.m * (p.single_a ? 1 : 2) * GEMM_BM + row_in_blk;
-          const int e1 = e0 + GEMM_BM;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int tok = tl.tok0 + c0 + i;
-            if (tok < tl.count) {
-              float* row = out + static_cast<size_t>(tok) * p.out_ld;
-              if (e0 < p.a_rows) row[e0] = __uint_as_float(r0[i]);
-              if (tl.has_a1 && e1 < p.a_rows) row[e1] = __uint_as_float(r1[i]);
-            }
-          }
+          stage_store_f32(stg, lane, r0, ncol, rows, out, tok_base, p.out_ld, ebase, p.a_rows);
+          if (tl.has_a1)
+            stage_store_f32(stg, lane, r1, ncol, rows, out, tok_base, p.out_ld, ebase + GEMM_BM,
+                            p.a_rows);
         } else if (MODE == MODE_GATEUP) {
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-          const int f = tl.m * GEMM_BM + row_in_blk;
+          uint32_t h[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c = tl.tok0 + c0 + i;
-            if (c < tl.count) {
-              const float h = silu_f(__uint_as_float(r0[i])) * __uint_as_float(r1[i]);
-              out[static_cast<size_t>(tl.brow0 - tl.tok0 + c) * p.out_ld + f] =
-                  __float2bfloat16_rn(h);
-            }
+          for (int i = 0; i < 32; ++i) {
+            const float g = __uint_as_float(r0[i]);
+            const float u = __uint_as_float(r1[i]);
+            h[i] = __float_as_uint(g * __frcp_rn(1.0f + __expf(-g)) * u);
           }
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+          const int64_t row0 = tl.brow0 - tl.tok0 + tok_base;   // first output row
+          stage_store_bf16(stg, lane, h, ncol, rows, out + row0 * p.out_ld + tl.m * GEMM_BM + q * 32,
+                           p.out_ld);
         } else {
           __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-          const int f0 = tl.m * (p.single_a ? 1 : 2) * GEMM_BM + row_in_blk;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c = tl.tok0 + c0 + i;
-            if (c < tl.count) {
-              __nv_bfloat16* row = out + static_cast<size_t>(tl.brow0 - tl.tok0 + c) * p.out_ld;
-              row[f0] = __float2bfloat16_rn(__uint_as_float(r0[i]));
-              if (tl.has_a1) row[f0 + GEMM_BM] = __float2bfloat16_rn(__uint_as_float(r1[i]));
-            }
-          }
+          const int64_t row0 = tl.brow0 - tl.tok0 + tok_base;
+          const int f0 = tl.m * (p.single_a ? 1 : 2) * GEMM_BM + q * 32;
+          stage_store_bf16(stg, lane, r0, ncol, rows, out + row0 * p.out_ld + f0, p.out_ld);
+          if (tl.has_a1)
+            stage_store_bf16(stg, lane, r1, ncol, rows, out + row0 * p.out_ld + f0 + GEMM_BM,
+                             p.out_ld);
         }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty_bar);
     }
+    (void)row_in_blk;
   }
 
   tc_fence_before();

@@ -21,11 +21,15 @@ constexpr int GEMM_BN = 256;           // tokens per tile at most
 constexpr int GEMM_BK = 64;            // K per pipeline stage (128-byte rows)
 constexpr int GEMM_STAGES = 3;
 constexpr int GEMM_B_BOX_ROWS = 32;    // tokens per TMA box of B
-constexpr int GEMM_THREADS = 256;
+constexpr int GEMM_EPI_WARPS = 8;          // two per TMEM lane quadrant
+constexpr int GEMM_EPI_THREADS = GEMM_EPI_WARPS * 32;
+constexpr int GEMM_THREADS = 128 + GEMM_EPI_THREADS;
+constexpr int GEMM_STG_BYTES = 32 * 32 * 4;  // per epilogue warp: 32 tokens x 32 fp32
 constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;
 constexpr int GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;
 constexpr int GEMM_STAGE_BYTES = 2 * GEMM_A_BYTES + GEMM_B_BYTES;
-constexpr int GEMM_SMEM_BYTES = GEMM_STAGES * GEMM_STAGE_BYTES + 1024;
+constexpr int GEMM_SMEM_BYTES =
+    GEMM_STAGES * GEMM_STAGE_BYTES + GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024;
 
 struct GemmParams {
   // Token groups (FFN experts).  For MODE_ROUTER there is one group of T
