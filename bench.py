@@ -19,9 +19,9 @@ steps.  With N > 1 GPUs each rank runs its own batch of T tokens against its
 own weight replica (tokens are independent: no collective in the step), so
 `value` is N*T*K / max-rank time ("weak" scaling).
 
-The JSON line also carries: `e2e` (the same metric with the step's input
-copied from pinned host memory and its output copied back inside the timed
-region), `roofline` (the dominant kernel's achieved rate against the measured
+The JSON line also carries: `e2e` (the same metric through moe_zc_forward_host: the
+step's input is copied from pinned host memory and its output back inside the
+timed region, in chunks whose copies overlap the kernels), `roofline` (the dominant kernel's achieved rate against the measured
 peak in MEASURED_PEAKS.json, from per-stage CUDA events recorded during the
 timed steps), `cpu_baseline` (the fp64 CPU oracle, as it stands, timed on the
 host cores on a bounded token sample; rank 0, N=1 only), `clocks` (SM clocks
@@ -70,6 +70,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--chunk-tokens", type=int, default=0,
+                    help="chunk size of the host-buffer forward (0: library default)")
     ap.add_argument("--shape", default="",
                     help="override workload sizes, e.g. T=4096,N=32,Z=16 (for profiling runs)")
     return ap.parse_args()
@@ -299,22 +301,25 @@ def run_ours(args, dist, w):
     ms_max = dist.max(ms)
     value = dist.world * w.T / (ms_max / 1e3)
 
-    # ---- end to end: pinned host input -> device -> forward -> host output
+    # ---- end to end through the host-buffer entry point: the step's input
+    # goes from pinned host memory to the device and its output comes back,
+    # in chunks whose copies overlap the kernels (moe_zc_forward_host)
     x_host = ri.x.pin_memory()
     out_host = torch.empty_like(x_host).pin_memory()
-    x_dev = torch.empty_like(dev["x"])
+
+    def step_host():
+        mz.forward_host(x_host, dev["W_r"], dev["b"], ew.W_gate, ew.W_up, ew.W_down,
+                        w.N, w.Z, w.K, out_host=out_host, logit_offset=dev["off"],
+                        chunk_tokens=args.chunk_tokens, stream=stream)
+
     for _ in range(2):
-        x_dev.copy_(x_host, non_blocking=True)
-        step(x_dev)
-        out_host.copy_(out, non_blocking=True)
+        step_host()
     torch.cuda.synchronize()
     dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(args.e2e_steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        step(x_dev)
-        out_host.copy_(out, non_blocking=True)
+        step_host()
     e1.record(stream)
     torch.cuda.synchronize()
     dist.barrier()

@@ -91,6 +91,26 @@ int moe_zc_forward_ex(const void* x, const void* W_r, const float* b,
                       const float* logit_offset, void* out, void* stream);
 
 /*
+ * moe_zc_forward_ex on HOST buffers: x_host [T, d] bf16 in, out_host [T, d]
+ * bf16 out (page-locked memory for overlap; pageable memory works but its
+ * copies do not overlap).  The weights, b and logit_offset stay device
+ * memory.  The tokens go in chunks of chunk_tokens (<= 0: T/8 rounded up to
+ * 256, at least 1024): while the kernels of one chunk run on `stream`, the
+ * next chunk is copied in and the previous one out on two streams of the
+ * library's own, so copies overlap compute.  Tokens are independent, so the
+ * result equals moe_zc_forward_ex's bit for bit.  Asynchronous: out_host is
+ * complete when `stream` is.  Afterwards moe_zc_expert_load reports the
+ * histogram of all T tokens; moe_zc_last_routing and moe_zc_last_expert
+ * describe the last chunk only.  Uses device staging for two chunks in and
+ * two out (4 * chunk_tokens * d * 2 bytes) in the workspace.
+ */
+int moe_zc_forward_host(const void* x_host, const void* W_r, const float* b,
+                        const void* W_gate, const void* W_up, const void* W_down,
+                        int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I,
+                        const float* logit_offset, void* out_host, int64_t chunk_tokens,
+                        void* stream);
+
+/*
  * Expert-load histogram of the last forward on the current device: the number
  * of tokens that picked each of the E experts, zero experts included.  This is
  * the "recent expert usage" that the write-up's bias controller (section

@@ -116,7 +116,17 @@ __global__ void permute_kernel(const uint4* __restrict__ x, const int* __restric
   }
 }
 
+__global__ void add_counts_kernel(const int* __restrict__ cnt, int E, int* __restrict__ total) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j < E) total[j] += cnt[j];
+}
+
 }  // namespace
+
+cudaError_t launch_add_counts(const int* cnt, int E, int* total, cudaStream_t stream) {
+  add_counts_kernel<<<(E + 255) / 256, 256, 0, stream>>>(cnt, E, total);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_scan(const int* cnt, int N, int* grp_off, int* grp_ttp, int* fill,
                         cudaStream_t stream) {

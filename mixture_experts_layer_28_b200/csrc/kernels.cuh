@@ -69,6 +69,8 @@ cudaError_t launch_scan(const int* cnt, int N, int* grp_off, int* grp_ttp, int* 
                         cudaStream_t stream);
 cudaError_t launch_assign_slots(const int* idx, int64_t pairs, int N, const int* grp_off,
                                 int* fill, int* slot, cudaStream_t stream);
+// total[j] += cnt[j] for j < E (histogram summed over the chunks of a forward)
+cudaError_t launch_add_counts(const int* cnt, int E, int* total, cudaStream_t stream);
 cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, int d, int K,
                            __nv_bfloat16* Xp, cudaStream_t stream);
 

@@ -44,6 +44,12 @@ struct Ctx {
   bool init = false;
   int sms = 0;
   Buf logits, idx, gate, zsum, slot, cnt, fill, grp_off, grp_ttp, Xp, H, Y, err;
+  // host-buffer forwards: device staging for two chunks in and out, the
+  // histogram summed over chunks, copy streams and their events
+  Buf xin[2], yout[2], cnt_total;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {};
+  bool counts_total = false;   // last forward was chunked: report cnt_total
   cudaEvent_t done = nullptr;
   bool has_result = false;
   int64_t T = 0;
@@ -361,12 +367,98 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   if (rec.ev) ++g_prof.n;
   CK(cudaEventRecord(c.done, st));
   c.has_result = true;
+  c.counts_total = false;
   c.T = T;
   c.d = d;
   c.N = N;
   c.Z = Z;
   c.K = K;
   c.I = I;
+  return MOE_ZC_OK;
+}
+
+int host_streams(Ctx& c) {
+  if (c.s_in) return MOE_ZC_OK;
+  CK(cudaStreamCreateWithFlags(&c.s_in, cudaStreamNonBlocking));
+  CK(cudaStreamCreateWithFlags(&c.s_out, cudaStreamNonBlocking));
+  CK(cudaEventCreateWithFlags(&c.ev_start, cudaEventDisableTiming));
+  for (int i = 0; i < 2; ++i) {
+    CK(cudaEventCreateWithFlags(&c.ev_in[i], cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&c.ev_comp[i], cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&c.ev_out[i], cudaEventDisableTiming));
+  }
+  return MOE_ZC_OK;
+}
+
+// The forward on host buffers: T tokens in chunks, each chunk copied in on
+// one stream, computed on the caller's stream and copied out on a third, so
+// that the copies of chunk c +- 1 overlap the kernels of chunk c.
+int forward_host_impl(const void* x_host, const void* W_r, const float* b, const void* W_gate,
+                      const void* W_up, const void* W_down, int64_t T, int32_t d, int32_t N,
+                      int32_t Z, int32_t K, int32_t I, const float* off, void* out_host,
+                      int64_t chunk, void* stream) {
+  if (T < 0) return MOE_ZC_ERR_INVALID_ARG;
+  if (T > 0 && (!x_host || !out_host)) return MOE_ZC_ERR_INVALID_ARG;
+  // the device-side checks of one chunk (fake aligned buffers stand in)
+  int s = check_args(reinterpret_cast<const void*>(16), W_r, b, W_gate, W_up, W_down, T, d, N,
+                     Z, K, I, off, reinterpret_cast<void*>(16));
+  if (s != MOE_ZC_OK) return s;
+  if (chunk <= 0) {
+    chunk = (T + 7) / 8;
+    chunk = ((chunk + 255) / 256) * 256;
+    if (chunk < 1024) chunk = 1024;
+  }
+  if (chunk > T) chunk = T;
+  Ctx* cp = nullptr;
+  if ((s = get_ctx(&cp)) != MOE_ZC_OK) return s;
+  Ctx& c = *cp;
+  const int E = N + Z;
+  if ((s = host_streams(c)) != MOE_ZC_OK) return s;
+  if ((s = ensure(c, c.cnt_total, sizeof(int) * E)) != MOE_ZC_OK) return s;
+  const size_t row_bytes = static_cast<size_t>(d) * 2;
+  for (int i = 0; i < 2 && T > 0; ++i) {
+    if ((s = ensure(c, c.xin[i], chunk * row_bytes)) != MOE_ZC_OK) return s;
+    if ((s = ensure(c, c.yout[i], chunk * row_bytes)) != MOE_ZC_OK) return s;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CK(cudaMemsetAsync(c.cnt_total.p, 0, sizeof(int) * E, st));
+  CK(cudaEventRecord(c.ev_start, st));
+  CK(cudaStreamWaitEvent(c.s_in, c.ev_start, 0));
+  CK(cudaStreamWaitEvent(c.s_out, c.ev_start, 0));
+  const char* xh = static_cast<const char*>(x_host);
+  char* oh = static_cast<char*>(out_host);
+  const int64_t nchunks = T > 0 ? (T + chunk - 1) / chunk : 0;
+  for (int64_t ci = 0; ci < nchunks; ++ci) {
+    const int bi = static_cast<int>(ci & 1);
+    const int64_t t0 = ci * chunk;
+    const int64_t n = (T - t0) < chunk ? (T - t0) : chunk;
+    // copy in once the kernels of chunk ci-2 are done with this buffer
+    if (ci >= 2) CK(cudaStreamWaitEvent(c.s_in, c.ev_comp[bi], 0));
+    CK(cudaMemcpyAsync(c.xin[bi].p, xh + t0 * row_bytes, n * row_bytes, cudaMemcpyHostToDevice,
+                       c.s_in));
+    CK(cudaEventRecord(c.ev_in[bi], c.s_in));
+    // compute once the input is here and chunk ci-2's output has left
+    CK(cudaStreamWaitEvent(st, c.ev_in[bi], 0));
+    if (ci >= 2) CK(cudaStreamWaitEvent(st, c.ev_out[bi], 0));
+    s = forward_impl(c.xin[bi].p, W_r, b, W_gate, W_up, W_down, n, d, N, Z, K, I, off,
+                     c.yout[bi].p, stream);
+    if (s != MOE_ZC_OK) return s;
+    CK(launch_add_counts(static_cast<const int*>(c.cnt.p), E,
+                         static_cast<int*>(c.cnt_total.p), st));
+    CK(cudaEventRecord(c.ev_comp[bi], st));
+    // copy out
+    CK(cudaStreamWaitEvent(c.s_out, c.ev_comp[bi], 0));
+    CK(cudaMemcpyAsync(oh + t0 * row_bytes, c.yout[bi].p, n * row_bytes, cudaMemcpyDeviceToHost,
+                       c.s_out));
+    CK(cudaEventRecord(c.ev_out[bi], c.s_out));
+  }
+  // the caller's stream completes only after every copy out
+  for (int i = 0; i < 2 && i < nchunks; ++i) CK(cudaStreamWaitEvent(st, c.ev_out[i], 0));
+  CK(cudaEventRecord(c.done, st));
+  c.has_result = true;
+  c.counts_total = true;
+  c.N = N;
+  c.Z = Z;
   return MOE_ZC_OK;
 }
 
@@ -402,6 +494,16 @@ int moe_zc_forward_ex(const void* x, const void* W_r, const float* b, const void
                       stream);
 }
 
+int moe_zc_forward_host(const void* x_host, const void* W_r, const float* b,
+                        const void* W_gate, const void* W_up, const void* W_down, int64_t T,
+                        int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I,
+                        const float* logit_offset, void* out_host, int64_t chunk_tokens,
+                        void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return forward_host_impl(x_host, W_r, b, W_gate, W_up, W_down, T, d, N, Z, K, I, logit_offset,
+                           out_host, chunk_tokens, stream);
+}
+
 int moe_zc_synchronize(void) {
   std::lock_guard<std::mutex> lk(g_mu);
   Ctx* c = nullptr;
@@ -417,7 +519,8 @@ int moe_zc_expert_load(int32_t* out_counts) {
   int s = get_ctx(&c);
   if (s != MOE_ZC_OK) return s;
   if ((s = sync_impl(*c)) != MOE_ZC_OK) return s;
-  CK(cudaMemcpy(out_counts, c->cnt.p, sizeof(int32_t) * (c->N + c->Z), cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(out_counts, c->counts_total ? c->cnt_total.p : c->cnt.p,
+                sizeof(int32_t) * (c->N + c->Z), cudaMemcpyDeviceToHost));
   return MOE_ZC_OK;
 }
 
@@ -490,13 +593,23 @@ void moe_zc_release(void) {
     if (!c.init) continue;
     cudaSetDevice(dev);
     cudaDeviceSynchronize();
-    Buf* bufs[] = {&c.logits, &c.idx, &c.gate, &c.zsum, &c.slot, &c.cnt, &c.fill,
-                   &c.grp_off, &c.grp_ttp, &c.Xp, &c.H, &c.Y, &c.err};
+    Buf* bufs[] = {&c.logits, &c.idx,     &c.gate,    &c.zsum,      &c.slot,
+                   &c.cnt,    &c.fill,    &c.grp_off, &c.grp_ttp,   &c.Xp,
+                   &c.H,      &c.Y,       &c.err,     &c.xin[0],    &c.xin[1],
+                   &c.yout[0], &c.yout[1], &c.cnt_total};
     for (Buf* b : bufs) {
       if (b->p) cudaFree(b->p);
       *b = Buf{};
     }
     if (c.done) cudaEventDestroy(c.done);
+    for (int i = 0; i < 2; ++i) {
+      if (c.ev_in[i]) cudaEventDestroy(c.ev_in[i]);
+      if (c.ev_comp[i]) cudaEventDestroy(c.ev_comp[i]);
+      if (c.ev_out[i]) cudaEventDestroy(c.ev_out[i]);
+    }
+    if (c.ev_start) cudaEventDestroy(c.ev_start);
+    if (c.s_in) cudaStreamDestroy(c.s_in);
+    if (c.s_out) cudaStreamDestroy(c.s_out);
     c = Ctx{};
   }
   cudaSetDevice(prev);

@@ -50,6 +50,8 @@ def lib() -> ctypes.CDLL:
         L.moe_zc_forward.restype = ctypes.c_int
         L.moe_zc_forward_ex.argtypes = [vp] * 6 + [i64, i32, i32, i32, i32, i32, vp, vp, vp]
         L.moe_zc_forward_ex.restype = ctypes.c_int
+        L.moe_zc_forward_host.argtypes = [vp] * 6 + [i64, i32, i32, i32, i32, i32, vp, vp, i64, vp]
+        L.moe_zc_forward_host.restype = ctypes.c_int
         L.moe_zc_expert_load.argtypes = [vp]
         L.moe_zc_expert_load.restype = ctypes.c_int
         L.moe_zc_last_routing.argtypes = [vp, vp]
@@ -129,6 +131,34 @@ def forward(x: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor,
                                      o, s)
     _check(st, "moe_zc_forward")
     return out
+
+
+def forward_host(x_host: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor,
+                 W_gate: Optional[torch.Tensor], W_up: Optional[torch.Tensor],
+                 W_down: Optional[torch.Tensor], N: int, Z: int, K: int,
+                 out_host: Optional[torch.Tensor] = None,
+                 logit_offset: Optional[torch.Tensor] = None, chunk_tokens: int = 0,
+                 stream=None) -> torch.Tensor:
+    """moe_zc_forward_host: x_host and out_host are CPU tensors (pin them for
+    overlap); the weights are CUDA tensors.  Asynchronous on `stream`."""
+    if x_host.is_cuda:
+        raise ValueError("x_host must be a CPU tensor")
+    if x_host.dtype != torch.bfloat16 or not x_host.is_contiguous():
+        raise ValueError("x_host must be contiguous bf16")
+    T, d = x_host.shape
+    I = int(W_gate.shape[1]) if (W_gate is not None and N > 0) else 0
+    if out_host is None:
+        out_host = torch.empty_like(x_host, pin_memory=x_host.is_pinned())
+    if out_host.is_cuda or out_host.dtype != torch.bfloat16 or not out_host.is_contiguous():
+        raise ValueError("out_host must be a contiguous bf16 CPU tensor")
+    bf = torch.bfloat16
+    st = lib().moe_zc_forward_host(
+        x_host.data_ptr(), _dev_ptr(W_r, bf, "W_r"), _dev_ptr(b, torch.float32, "b"),
+        _dev_ptr(W_gate, bf, "W_gate"), _dev_ptr(W_up, bf, "W_up"), _dev_ptr(W_down, bf, "W_down"),
+        T, d, N, Z, K, I, _dev_ptr(logit_offset, torch.float32, "logit_offset"),
+        out_host.data_ptr(), chunk_tokens, _stream_ptr(stream))
+    _check(st, "moe_zc_forward_host")
+    return out_host
 
 
 def expert_load(E: int) -> np.ndarray:

@@ -180,6 +180,25 @@ def test_full_size_skewed(name):
     _sampled_check(Case(wl.get(name)))
 
 
+@pytest.mark.parametrize("T,chunk", [(1000, 256), (300, 0), (64, 1000), (2048, 512)])
+def test_host_buffer_forward_matches_device_forward(T, chunk):
+    """moe_zc_forward_host (chunked copies overlapping compute) gives the same
+    bits as moe_zc_forward, and its histogram covers all T tokens."""
+    w = wl.get("small", T=T)
+    case = Case(w)
+    out_d, idx, _, cnt = _gpu_result(case)
+    x_host = case.x.clone().pin_memory()
+    out_host = torch.full_like(x_host, 7.0).pin_memory()
+    ew = case.ew
+    d = case.dev
+    mz.forward_host(x_host, d["W_r"], d["b"], ew.W_gate, ew.W_up, ew.W_down, w.N, w.Z, w.K,
+                    out_host=out_host, chunk_tokens=chunk)
+    torch.cuda.synchronize()
+    mz.synchronize()
+    assert np.array_equal(out_host.float().numpy().astype(np.float64), out_d)
+    assert np.array_equal(mz.expert_load(w.E), cnt)
+
+
 def test_allocation_failure_reports_oom():
     w = wl.get("tiny")
     case = Case(w)
