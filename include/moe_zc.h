@@ -138,6 +138,35 @@ int moe_zc_last_routing(int32_t* idx, float* gate);
 int moe_zc_last_expert(int32_t e, int32_t max_rows, int32_t* n_rows,
                        int32_t* tokens, void* H, void* Y);
 
+/*
+ * Host-side PID controller of the expert biases (write-up, section
+ * "Zero-computation experts": the biases follow recent expert usage through
+ * a PID controller; no gains, set-point or window are given).  Plain host
+ * code: it reads a histogram (e.g. from moe_zc_expert_load, summed over
+ * ranks and steps as the caller sees fit) and writes new biases, which the
+ * caller hands to the next forward.
+ *
+ *   set-point  zero experts together get target_zero_frac = rho of the
+ *              tokens*K picks, FFN experts share the rest evenly:
+ *              L*_i = (1-rho) tokens K / N (i < N), rho tokens K / Z (i >= N)
+ *   error      e_i = (L*_i - counts_i) / (tokens K / E)
+ *   update     b_i = base_i + clip(kp e_i + ki sum e_i + kd (e_i - e_prev,i))
+ *
+ * state: host float[3E] = [base | integral | previous error], set up by
+ * moe_zc_bias_controller_init from the starting biases b (host float[E]).
+ * moe_zc_bias_controller_step updates state and writes b (host float[E]).
+ * max_shift <= 0 disables the clip.  rho must be 1 when N == 0 and 0 when
+ * Z == 0.  Not thread-safe on a shared state.
+ */
+typedef struct moe_zc_pid {
+  float target_zero_frac;
+  float kp, ki, kd;
+  float max_shift;
+} moe_zc_pid;
+int moe_zc_bias_controller_init(const float* b, int32_t E, float* state);
+int moe_zc_bias_controller_step(const int32_t* counts, int32_t N, int32_t Z, int64_t tokens,
+                                int32_t K, const moe_zc_pid* pid, float* state, float* b);
+
 /* Wait for the last forward; report (and clear) a device-side timeout. */
 int moe_zc_synchronize(void);
 

@@ -2,7 +2,8 @@
 
     python -m mixture_experts_layer_28_b200.build [--force] [--ptxas-v]
 
-Each .cu under csrc/ is compiled with nvcc for sm_100a only and linked into
+Each .cu (and host-only .cpp) under csrc/ is compiled with nvcc for sm_100a
+only and linked into
 one shared library with the CUDA runtime linked statically; the library's
 only external dependency is the NVIDIA driver.
 """
@@ -36,11 +37,12 @@ def nvcc() -> str:
 
 
 def _sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _deps():
-    return _sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(INCLUDE, "moe_zc.h")]
+    return (_sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(INCLUDE, "moe_zc.h")]
+            + [os.path.abspath(__file__)])
 
 
 def up_to_date() -> bool:

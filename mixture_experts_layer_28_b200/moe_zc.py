@@ -33,6 +33,12 @@ class MoeZcError(RuntimeError):
         super().__init__(f"{what}: {status_string(status)} ({status})")
 
 
+class Pid(ctypes.Structure):
+    """moe_zc_pid: set-point and gains of the bias controller."""
+    _fields_ = [("target_zero_frac", ctypes.c_float), ("kp", ctypes.c_float),
+                ("ki", ctypes.c_float), ("kd", ctypes.c_float), ("max_shift", ctypes.c_float)]
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 
@@ -75,6 +81,11 @@ def lib() -> ctypes.CDLL:
         L.moe_zc_route_noalloc.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32,
                                            vp, vp, vp, vp, vp]
         L.moe_zc_route_noalloc.restype = ctypes.c_int
+        L.moe_zc_bias_controller_init.argtypes = [vp, i32, vp]
+        L.moe_zc_bias_controller_init.restype = ctypes.c_int
+        L.moe_zc_bias_controller_step.argtypes = [vp, i32, i32, i64, i32,
+                                                  ctypes.POINTER(Pid), vp, vp]
+        L.moe_zc_bias_controller_step.restype = ctypes.c_int
         L.moe_zc_test_inject.argtypes = [i32, i64]
         L.moe_zc_test_inject.restype = None
         _lib = L
@@ -233,6 +244,44 @@ def profile_read() -> tuple[dict, int]:
            "moe_zc_profile_read")
     names = [lib().moe_zc_stage_name(i).decode() for i in range(STAGES)]
     return dict(zip(names, ms.tolist())), n.value
+
+
+class BiasController:
+    """Host-side PID controller of the expert biases (moe_zc_bias_controller_*).
+
+    step(counts) takes an expert-load histogram over `tokens` tokens and
+    returns the new biases (numpy float32 [E]).
+    """
+
+    def __init__(self, b0, N: int, Z: int, K: int, target_zero_frac: float,
+                 kp: float, ki: float, kd: float = 0.0, max_shift: float = 0.0):
+        self.N, self.Z, self.K = N, Z, K
+        self.pid = Pid(target_zero_frac, kp, ki, kd, max_shift)
+        self.b = np.ascontiguousarray(np.asarray(b0, dtype=np.float32)).copy()
+        self.state = np.zeros(3 * (N + Z), dtype=np.float32)
+        _check(lib().moe_zc_bias_controller_init(self.b.ctypes.data, N + Z,
+                                                 self.state.ctypes.data),
+               "moe_zc_bias_controller_init")
+
+    def step(self, counts, tokens: int) -> np.ndarray:
+        c = np.ascontiguousarray(np.asarray(counts, dtype=np.int32))
+        _check(lib().moe_zc_bias_controller_step(c.ctypes.data, self.N, self.Z, tokens, self.K,
+                                                 ctypes.byref(self.pid), self.state.ctypes.data,
+                                                 self.b.ctypes.data),
+               "moe_zc_bias_controller_step")
+        return self.b.copy()
+
+
+def allreduce_expert_load(counts: np.ndarray, group=None) -> np.ndarray:
+    """Sum an expert-load histogram over the ranks of a torch.distributed
+    group (exact: int64 counts), so a controller on every rank sees the
+    global usage."""
+    import torch.distributed as dist
+    backend = dist.get_backend(group)
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    t = torch.as_tensor(np.asarray(counts, dtype=np.int64), device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+    return t.cpu().numpy()
 
 
 def test_inject(fail_allocs: int = 0, wait_limit_ns: int = 0) -> None:
