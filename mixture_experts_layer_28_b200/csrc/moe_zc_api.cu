@@ -404,7 +404,9 @@ int forward_host_impl(const void* x_host, const void* W_r, const float* b, const
                      Z, K, I, off, reinterpret_cast<void*>(16));
   if (s != MOE_ZC_OK) return s;
   if (chunk <= 0) {
-    chunk = (T + 7) / 8;
+    // four chunks: measured best at the prefill workload (2048: 13.0 ms,
+    // 4096: 12.1 ms, 8192: 12.8 ms per step, B200)
+    chunk = (T + 3) / 4;
     chunk = ((chunk + 255) / 256) * 256;
     if (chunk < 1024) chunk = 1024;
   }
