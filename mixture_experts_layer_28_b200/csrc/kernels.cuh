@@ -44,6 +44,7 @@ struct GemmParams {
                           // slice s writes its partial sums to out + s * split_stride
   long long split_stride;
   int single_a;           // MODE_ROUTER/MODE_DOWN: 1 = one 128-row A block per tile (no pair)
+  int mgroup;             // pair kernel: weight blocks per tile group (divides mblocks; 0 = all)
   int mblocks;            // tiles along the weight rows of one group
   int a_rows;             // weight rows per group: E (router), I (gate/up), d (down)
   void* out;              // fp32 logits [T, E] | bf16 H [rows, I] | bf16 Y [rows, d]
@@ -55,6 +56,20 @@ struct GemmParams {
 cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap& a1,
                         const CUtensorMap& b, const GemmParams& p, int grid,
                         cudaStream_t stream);
+
+// The FFN expert GEMMs on CTA pairs (cta_group::2, M = 256 per MMA), for
+// batches with many tokens per expert; `clusters` pairs are launched.
+//   gate/up: a0 = W_gate [N*I, d] and a1 = W_up with 64-row boxes; mblocks = I/128
+//   down:    a0 = a1 = W_down [N*d, I] with 128-row boxes; mblocks = d/256
+//   b: tokens with 32-row boxes, as for launch_gemm
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_A_BYTES = GEMM_BM * GEMM_BK * 2;          // 128 weight rows per CTA
+constexpr int PAIR_STAGE_BYTES = PAIR_A_BYTES + 128 * GEMM_BK * 2;   // + 128 tokens per CTA
+constexpr int PAIR_XCHG_BYTES = 2 * 4096;                     // gate/up swap, reused for staging
+constexpr int PAIR_SMEM_BYTES = PAIR_STAGES * PAIR_STAGE_BYTES + 4 * PAIR_XCHG_BYTES + 1024;
+cudaError_t launch_gemm_pair(GemmMode mode, const CUtensorMap& a0, const CUtensorMap& a1,
+                             const CUtensorMap& b, const GemmParams& p, int clusters,
+                             cudaStream_t stream);
 
 // ------------------------------------------------------------------ router
 // softmax over E logits (+offset), + bias, top-K, zero-gate sums, histogram.

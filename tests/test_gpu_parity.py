@@ -199,6 +199,35 @@ def test_host_buffer_forward_matches_device_forward(T, chunk):
     assert np.array_equal(mz.expert_load(w.E), cnt)
 
 
+def _bias_hot_expert(w, e, T):
+    ri = wl.routing_inputs(w, T)
+    b = ri.b0.clone()
+    b[e] += 10.0
+    return b
+
+
+@pytest.mark.parametrize("path", ["0", "1"])
+@pytest.mark.parametrize("case_id", ["tiny", "ragged17", "hot_expert", "dense", "small"])
+def test_expert_gemm_paths(path, case_id, monkeypatch):
+    """Both expert-GEMM engines -- single SM (MOE_ZC_GEMM_PAIR=0) and CTA
+    pairs with cta_group::2 (=1) -- on the edge cases."""
+    monkeypatch.setenv("MOE_ZC_GEMM_PAIR", path)
+    if case_id == "tiny":
+        case = Case(wl.get("tiny"))
+    elif case_id == "ragged17":
+        case = Case(wl.get("small", T=17))
+    elif case_id == "hot_expert":
+        w = wl.get("small", T=1100)
+        case = Case(w, T=1100, bias=_bias_hot_expert(w, 3, 1100))
+    elif case_id == "dense":
+        case = Case(wl.get("tiny", T=64, N=6, Z=2, K=8))
+    else:
+        case = Case(wl.get("small", T=2048))
+    _full_check(case, n_expert_checks=6)
+    if case_id == "hot_expert":
+        assert check_expert_rows(case, 3, max_rows=1100) == 1100
+
+
 def test_allocation_failure_reports_oom():
     w = wl.get("tiny")
     case = Case(w)
