@@ -36,34 +36,40 @@ __device__ __forceinline__ void stage_store_bf16(uint8_t* stg, int lane, const u
 }
 
 // fp32 variant for the router's logits: features ebase + 0..31 of rows
-// tok_base + i, features >= E dropped; 128-byte rows, eight lanes per row.
+// tok_base + i, features >= E dropped; 128-byte rows, eight lanes per row,
+// staged 16 tokens at a time (2 KB).
 __device__ __forceinline__ void stage_store_f32(uint8_t* stg, int lane, const uint32_t (&v)[32],
                                                 int ncol, int rows, float* out, int tok_base,
                                                 int ld, int ebase, int E) {
   uint32_t* st = reinterpret_cast<uint32_t*>(stg);
-#pragma unroll
-  for (int i = 0; i < 32; ++i)
-    if (i < ncol) st[i * 32 + lane] = v[i];
-  __syncwarp();
   const bool vec = (ld % 4 == 0) && (ebase + 32 <= E);
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int r = (lane >> 3) + 4 * k;
-    const int part = lane & 7;
-    if (r < rows) {
-      float* dst = out + static_cast<int64_t>(tok_base + r) * ld + ebase + part * 4;
-      const uint4 val = *reinterpret_cast<const uint4*>(stg + r * 128 + part * 16);
-      if (vec) {
-        *reinterpret_cast<uint4*>(dst) = val;
-      } else {
-        const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+  for (int hf = 0; hf < 2; ++hf) {
+    if (hf * 16 >= ncol) break;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (ebase + part * 4 + e < E) dst[e] = __uint_as_float(w[e]);
+    for (int i = 0; i < 16; ++i)
+      if (hf * 16 + i < ncol) st[i * 32 + lane] = v[hf * 16 + i];
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int r = (lane >> 3) + 4 * k;
+      const int row = hf * 16 + r;
+      const int part = lane & 7;
+      if (row < rows) {
+        float* dst = out + static_cast<int64_t>(tok_base + row) * ld + ebase + part * 4;
+        const uint4 val = *reinterpret_cast<const uint4*>(stg + r * 128 + part * 16);
+        if (vec) {
+          *reinterpret_cast<uint4*>(dst) = val;
+        } else {
+          const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (ebase + part * 4 + e < E) dst[e] = __uint_as_float(w[e]);
+        }
       }
     }
+    __syncwarp();
   }
-  __syncwarp();
 }
 
 }  // namespace moezc

@@ -77,7 +77,7 @@ __device__ __forceinline__ PairTile pair_tile(const GemmParams& p, int t, uint32
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(PAIR_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                  const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -104,7 +104,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full_bar[b], 1);
-      mbar_init(&acc_empty_bar[b], 2 * GEMM_EPI_WARPS);   // one per epilogue warp, both CTAs
+      mbar_init(&acc_empty_bar[b], 2 * PAIR_EPI_WARPS);   // one per epilogue warp, both CTAs
     }
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
@@ -292,7 +292,7 @@ cudaError_t launch_gemm_pair(GemmMode mode, const CUtensorMap& a0, const CUtenso
   if (clusters <= 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
-  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.blockDim = dim3(PAIR_THREADS, 1, 1);
   cfg.dynamicSmemBytes = PAIR_SMEM_BYTES;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -232,14 +232,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
    __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
-    // Eight warps: warp w drains TMEM lanes (w % 4) * 32 .. +31 (the quadrant
-    // its warp id may access) and every other 32-column chunk of the tile
-    // (half = 0 or 1).  Each chunk goes TMEM -> registers (one wait per
+    // Twelve warps: warp w drains TMEM lanes (w % 4) * 32 .. +31 (the quadrant
+    // its warp id may access) and every third 32-column chunk of the tile
+    // (group = 0, 1 or 2).  Each chunk goes TMEM -> registers (one wait per
     // chunk) -> math -> a per-warp staging tile in shared memory -> 16-byte
     // coalesced global stores, one output row of 64 (bf16) or 128 (fp32)
     // bytes per 4 or 8 lanes.
     const int q = warp & 3;
-    const int half = (warp - 4) >> 2;
+    const int group = (warp - 4) >> 2;
     const int row_in_blk = q * 32 + lane;
     const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
     uint8_t* stg = smem + GEMM_STAGES * GEMM_STAGE_BYTES + (warp - 4) * GEMM_STG_BYTES;
@@ -251,7 +251,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         break;
       }
       tc_fence_after();
-      for (int c0 = half * 32; c0 < tl.nmma; c0 += 64) {
+      for (int c0 = group * 32; c0 < tl.nmma; c0 += 32 * GEMM_EPI_GROUPS) {
         const bool wide = c0 + 32 <= tl.nmma;   // 32 columns, else 16
         uint32_t r0[32], r1[32];
         tmem_ld16(tq + c0, *reinterpret_cast<uint32_t(*)[16]>(&r0[0]));
@@ -277,7 +277,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
           for (int i = 0; i < 32; ++i) {
             const float g = __uint_as_float(r0[i]);
             const float u = __uint_as_float(r1[i]);
-            h[i] = __float_as_uint(g * __frcp_rn(1.0f + __expf(-g)) * u);
+            // SiLU(g) * u; the exponent is clamped so 1 + e^-g stays finite
+            h[i] = __float_as_uint(__fdividef(g, 1.0f + __expf(-fmaxf(g, -80.0f))) * u);
           }
           __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
           const int64_t row0 = tl.brow0 - tl.tok0 + tok_base;   // first output row

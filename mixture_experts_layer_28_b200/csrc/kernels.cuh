@@ -21,10 +21,11 @@ constexpr int GEMM_BN = 256;           // tokens per tile at most
 constexpr int GEMM_BK = 64;            // K per pipeline stage (128-byte rows)
 constexpr int GEMM_STAGES = 3;
 constexpr int GEMM_B_BOX_ROWS = 32;    // tokens per TMA box of B
-constexpr int GEMM_EPI_WARPS = 8;          // two per TMEM lane quadrant
+constexpr int GEMM_EPI_GROUPS = 3;          // epilogue warps per TMEM lane quadrant
+constexpr int GEMM_EPI_WARPS = 4 * GEMM_EPI_GROUPS;
 constexpr int GEMM_EPI_THREADS = GEMM_EPI_WARPS * 32;
 constexpr int GEMM_THREADS = 128 + GEMM_EPI_THREADS;
-constexpr int GEMM_STG_BYTES = 32 * 32 * 4;  // per epilogue warp: 32 tokens x 32 fp32
+constexpr int GEMM_STG_BYTES = 32 * 32 * 2;  // per epilogue warp: 32 tokens x 32 bf16 (or 16 x 32 fp32)
 constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;
 constexpr int GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;
 constexpr int GEMM_STAGE_BYTES = 2 * GEMM_A_BYTES + GEMM_B_BYTES;
@@ -62,6 +63,8 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
 //   gate/up: a0 = W_gate [N*I, d] and a1 = W_up with 64-row boxes; mblocks = I/128
 //   down:    a0 = a1 = W_down [N*d, I] with 128-row boxes; mblocks = d/256
 //   b: tokens with 32-row boxes, as for launch_gemm
+constexpr int PAIR_EPI_WARPS = 8;           // two per TMEM lane quadrant
+constexpr int PAIR_THREADS = 128 + PAIR_EPI_WARPS * 32;
 constexpr int PAIR_STAGES = 6;
 constexpr int PAIR_A_BYTES = GEMM_BM * GEMM_BK * 2;          // 128 weight rows per CTA
 constexpr int PAIR_STAGE_BYTES = PAIR_A_BYTES + 128 * GEMM_BK * 2;   // + 128 tokens per CTA
