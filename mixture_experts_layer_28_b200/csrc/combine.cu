@@ -12,6 +12,7 @@
 // bf16: the result does not depend on where the dispatch put a token's rows.
 // One CTA per token; each thread handles 8 features with 16-byte loads.
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace moezc {
 namespace {
@@ -33,6 +34,8 @@ __global__ void combine_kernel(const uint4* __restrict__ x, const uint4* __restr
   __shared__ int sl[MOE_MAX_K_INTERNAL];
   __shared__ float gt[MOE_MAX_K_INTERNAL];
   __shared__ int nffn;
+  griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     int n = 0;
     for (int k = 0; k < K; ++k) {
@@ -69,10 +72,9 @@ cudaError_t launch_combine(const __nv_bfloat16* x, const __nv_bfloat16* Y, const
   if (T <= 0) return cudaSuccess;
   const int d8 = d / 8;
   const int threads = d8 < 256 ? ((d8 + 31) / 32) * 32 : 256;
-  combine_kernel<<<static_cast<unsigned>(T), threads, 0, stream>>>(
-      reinterpret_cast<const uint4*>(x), reinterpret_cast<const uint4*>(Y), slot, gate, zsum,
-      d8, K, reinterpret_cast<uint4*>(out));
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(static_cast<unsigned>(T)), dim3(threads), 0, stream,
+                    reinterpret_cast<const uint4*>(x), reinterpret_cast<const uint4*>(Y), slot,
+                    gate, zsum, d8, K, reinterpret_cast<uint4*>(out));
 }
 
 }  // namespace moezc

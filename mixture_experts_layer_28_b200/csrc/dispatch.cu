@@ -16,6 +16,7 @@
 //             FFN slots of Xp, the B operand of the gate/up GEMM.
 // The histogram itself is integer and comes from the router, so it is exact.
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace moezc {
 namespace {
@@ -53,6 +54,8 @@ scan_kernel(const int* __restrict__ cnt, int N, int* __restrict__ grp_off,
             int* __restrict__ grp_ttp, int* __restrict__ fill) {
   __shared__ int warp_sums[32];
   __shared__ int carry_rows, carry_tiles;
+  griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x == 0) { carry_rows = 0; carry_tiles = 0; }
   __syncthreads();
   for (int base = 0; base < N; base += SCAN_THREADS) {
@@ -81,6 +84,8 @@ scan_kernel(const int* __restrict__ cnt, int N, int* __restrict__ grp_off,
 __global__ void assign_slots_kernel(const int* __restrict__ idx, int64_t pairs, int N,
                                     const int* __restrict__ grp_off, int* __restrict__ fill,
                                     int* __restrict__ slot) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
   const bool valid = i < pairs;
@@ -104,6 +109,8 @@ __global__ void permute_kernel(const uint4* __restrict__ x, const int* __restric
                                int d8, int K, uint4* __restrict__ Xp) {
   const int64_t t = blockIdx.x;
   __shared__ int sl[MOE_MAX_K_INTERNAL];
+  griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x < K) sl[threadIdx.x] = slot[t * K + threadIdx.x];
   __syncthreads();
   const uint4* src = x + t * d8;
@@ -117,6 +124,8 @@ __global__ void permute_kernel(const uint4* __restrict__ x, const int* __restric
 }
 
 __global__ void add_counts_kernel(const int* __restrict__ cnt, int E, int* __restrict__ total) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j < E) total[j] += cnt[j];
 }
@@ -124,14 +133,13 @@ __global__ void add_counts_kernel(const int* __restrict__ cnt, int E, int* __res
 }  // namespace
 
 cudaError_t launch_add_counts(const int* cnt, int E, int* total, cudaStream_t stream) {
-  add_counts_kernel<<<(E + 255) / 256, 256, 0, stream>>>(cnt, E, total);
-  return cudaGetLastError();
+  return launch_pdl(add_counts_kernel, dim3((E + 255) / 256), dim3(256), 0, stream, cnt, E, total);
 }
 
 cudaError_t launch_scan(const int* cnt, int N, int* grp_off, int* grp_ttp, int* fill,
                         cudaStream_t stream) {
-  scan_kernel<<<1, SCAN_THREADS, 0, stream>>>(cnt, N, grp_off, grp_ttp, fill);
-  return cudaGetLastError();
+  return launch_pdl(scan_kernel, dim3(1), dim3(SCAN_THREADS), 0, stream, cnt, N, grp_off, grp_ttp,
+                    fill);
 }
 
 cudaError_t launch_assign_slots(const int* idx, int64_t pairs, int N, const int* grp_off,
@@ -139,9 +147,8 @@ cudaError_t launch_assign_slots(const int* idx, int64_t pairs, int N, const int*
   if (pairs <= 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (pairs + threads - 1) / threads;
-  assign_slots_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(idx, pairs, N,
-                                                                            grp_off, fill, slot);
-  return cudaGetLastError();
+  return launch_pdl(assign_slots_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0,
+                    stream, idx, pairs, N, grp_off, fill, slot);
 }
 
 cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, int d, int K,
@@ -149,9 +156,8 @@ cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, i
   if (T <= 0) return cudaSuccess;
   const int d8 = d / 8;
   const int threads = d8 < 256 ? ((d8 + 31) / 32) * 32 : 256;
-  permute_kernel<<<static_cast<unsigned>(T), threads, 0, stream>>>(
-      reinterpret_cast<const uint4*>(x), slot, d8, K, reinterpret_cast<uint4*>(Xp));
-  return cudaGetLastError();
+  return launch_pdl(permute_kernel, dim3(static_cast<unsigned>(T)), dim3(threads), 0, stream,
+                    reinterpret_cast<const uint4*>(x), slot, d8, K, reinterpret_cast<uint4*>(Xp));
 }
 
 }  // namespace moezc

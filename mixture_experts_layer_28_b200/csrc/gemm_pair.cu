@@ -122,6 +122,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
   __syncthreads();
   cluster_sync_all();   // both CTAs' barriers exist before any cross-CTA use
   tc_fence_after();
+  griddep_wait();       // the previous kernel's results are visible from here
+  griddep_launch_dependents();
   const uint32_t tmem = tmem_base_sh;
   const int ntiles = __ldg(p.grp_ttp + p.G) * p.mblocks;
   const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
@@ -295,13 +297,15 @@ cudaError_t launch_gemm_pair(GemmMode mode, const CUtensorMap& a0, const CUtenso
   cfg.blockDim = dim3(PAIR_THREADS, 1, 1);
   cfg.dynamicSmemBytes = PAIR_SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e;
   if (mode == MODE_GATEUP) {
     e = cudaFuncSetAttribute(gemm_pair_kernel<MODE_GATEUP>,

@@ -150,6 +150,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the prologue above overlaps the previous kernel; from here on its
+  // results (routing, offsets, activations) are read
+  griddep_wait();
+  griddep_launch_dependents();
   const uint32_t tmem = tmem_base_sh;
   const int ntiles = total_tiles<MODE>(p);
 
@@ -320,21 +324,25 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
       e = cudaFuncSetAttribute(gemm_kernel<MODE_ROUTER>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
       if (e != cudaSuccess) return e;
-      gemm_kernel<MODE_ROUTER><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(a0, a1, b, p);
+      e = launch_pdl(gemm_kernel<MODE_ROUTER>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES, stream,
+                     a0, a1, b, p);
       break;
     case MODE_GATEUP:
       e = cudaFuncSetAttribute(gemm_kernel<MODE_GATEUP>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
       if (e != cudaSuccess) return e;
-      gemm_kernel<MODE_GATEUP><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(a0, a1, b, p);
+      e = launch_pdl(gemm_kernel<MODE_GATEUP>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES, stream,
+                     a0, a1, b, p);
       break;
     case MODE_DOWN:
       e = cudaFuncSetAttribute(gemm_kernel<MODE_DOWN>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
       if (e != cudaSuccess) return e;
-      gemm_kernel<MODE_DOWN><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(a0, a1, b, p);
+      e = launch_pdl(gemm_kernel<MODE_DOWN>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES, stream,
+                     a0, a1, b, p);
       break;
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

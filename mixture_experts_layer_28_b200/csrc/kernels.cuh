@@ -10,6 +10,24 @@ namespace moezc {
 
 constexpr int MOE_MAX_K_INTERNAL = 32;   // most picks per token
 
+// Launch with programmatic stream serialisation (the kernel overlaps its
+// predecessor's tail and orders itself with griddepcontrol.wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ------------------------------------------------------------------ GEMM
 // One tcgen05 engine serves the three contractions of the layer.  Weights are
 // the A operand (M = 128 rows per MMA, two A blocks per tile -> two fp32

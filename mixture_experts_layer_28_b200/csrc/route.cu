@@ -24,6 +24,7 @@
 #include <climits>
 
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace moezc {
 namespace {
@@ -59,7 +60,7 @@ __device__ __forceinline__ void lane_best(const uint32_t (&key)[VPL], const floa
   bp = pv[0];
 }
 
-template <int VPL>  // logits per lane: E <= 32 * VPL
+template <int VPL, bool SPLIT>  // logits per lane: E <= 32 * VPL; SPLIT: sum K slices
 __global__ void __launch_bounds__(ROUTE_WARPS * 32)
 route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
              const float* __restrict__ offset, int64_t T, int E, int N, int K,
@@ -67,6 +68,8 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
              int* __restrict__ cnt, int splits) {
   extern __shared__ int hist[];  // [E]
   for (int j = threadIdx.x; j < E; j += blockDim.x) hist[j] = 0;
+  griddep_wait();
+  griddep_launch_dependents();
   __syncthreads();
 
   const int warp = threadIdx.x >> 5;
@@ -82,7 +85,10 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
       const int j = lane + 32 * i;
       l[i] = (j < E) ? lrow[j] : 0.f;
     }
-    for (int sp = 1; sp < splits; ++sp) {
+    // (unrolled by 4 so that several slices' loads are in flight at once;
+    // the sum is still taken in slice order)
+#pragma unroll 4
+    for (int sp = 1; SPLIT && sp < splits; ++sp) {
       const float* srow = lrow + sp * split_stride;
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
@@ -155,20 +161,36 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
     if (hist[j]) atomicAdd(&cnt[j], hist[j]);
 }
 
+template <int VPL, bool SPLIT>
+cudaError_t launch_route_kernel(const float* logits, const float* b, const float* offset,
+                               int64_t T, int E, int N, int K, int* idx, float* gate,
+                               float* zsum, int* cnt, cudaStream_t stream, int splits) {
+  int dev = 0, sms = 148, per_sm = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // one wave of resident blocks, each warp walking many tokens, so the
+  // per-block histogram zeroing and flush are paid once per block
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_kernel<VPL, SPLIT>,
+                                                    ROUTE_WARPS * 32, E * sizeof(int)) !=
+          cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const int64_t want = (T + ROUTE_WARPS - 1) / ROUTE_WARPS;
+  const int64_t cap = static_cast<int64_t>(sms) * per_sm;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  return launch_pdl(route_kernel<VPL, SPLIT>, dim3(grid), dim3(ROUTE_WARPS * 32), E * sizeof(int),
+                    stream, logits, b, offset, T, E, N, K, idx, gate, zsum, cnt, splits);
+}
+
 template <int VPL>
 cudaError_t launch_route_vpl(const float* logits, const float* b, const float* offset, int64_t T,
                              int E, int N, int K, int* idx, float* gate, float* zsum, int* cnt,
                              cudaStream_t stream, int splits) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t want = (T + ROUTE_WARPS - 1) / ROUTE_WARPS;
-  // a few tokens per warp so the per-block histogram flush is amortised
-  const int64_t cap = static_cast<int64_t>(sms) * 8;
-  const int grid = static_cast<int>(want < cap ? want : cap);
-  route_kernel<VPL><<<grid, ROUTE_WARPS * 32, E * sizeof(int), stream>>>(
-      logits, b, offset, T, E, N, K, idx, gate, zsum, cnt, splits);
-  return cudaGetLastError();
+  if (splits > 1)
+    return launch_route_kernel<VPL, true>(logits, b, offset, T, E, N, K, idx, gate, zsum, cnt,
+                                          stream, splits);
+  return launch_route_kernel<VPL, false>(logits, b, offset, T, E, N, K, idx, gate, zsum, cnt,
+                                         stream, splits);
 }
 
 }  // namespace
