@@ -57,9 +57,13 @@ L2_BYTES = 126 * 2 ** 20
 KERNELS_PER_FORWARD = 8   # router_gemm, route, scan, assign, permute, gateup, down, combine
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel
-# from an ncu capture of the current kernel build, per workload (None = not
-# captured for this build).
-NCU_TRAFFIC_BYTES = {}
+# from an ncu capture of the current kernel build at the full workload (one
+# pass; profiles/gemm_traffic_fullsize.md), per workload.  Clear an entry when
+# that kernel changes.
+NCU_TRAFFIC_BYTES = {
+    "prefill": 9_097_588_224 + 560_337_408,    # gate/up GEMM
+    "decode": 1_520_874_496 + 5_736_192,       # gate/up GEMM
+}
 
 
 def parse():
