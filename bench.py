@@ -61,8 +61,8 @@ KERNELS_PER_FORWARD = 8   # router_gemm, route, scan, assign, permute, gateup, d
 # pass; profiles/gemm_traffic_fullsize.md), per workload.  Clear an entry when
 # that kernel changes.
 NCU_TRAFFIC_BYTES = {
-    "prefill": 9_097_588_224 + 560_337_408,    # gate/up GEMM
-    "decode": 1_520_874_496 + 5_736_192,       # gate/up GEMM
+    "prefill": 7_902_767_872 + 560_506_624,    # gate/up GEMM
+    "decode": 1_520_840_704 + 3_909_376,       # gate/up GEMM
 }
 
 

@@ -9,15 +9,18 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "ptx.cuh"
+
 namespace moezc {
 
 // One warp's 32 features x ncol tokens of fp32 results (thread = feature,
 // v[i] = token i) -> bf16 rows out[i * ld + 0..31] for i < rows, through a
 // [32 tokens][32 features] staging tile: 2-byte shared stores by feature,
-// then 16-byte loads and global stores, four lanes per 64-byte row.
+// then 16-byte loads and global stores, four lanes per 64-byte row; a
+// non-zero l2_policy (createpolicy) is attached to the global stores.
 __device__ __forceinline__ void stage_store_bf16(uint8_t* stg, int lane, const uint32_t (&v)[32],
                                                  int ncol, int rows, __nv_bfloat16* out,
-                                                 int64_t ld) {
+                                                 int64_t ld, uint64_t l2_policy) {
   __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(stg);
 #pragma unroll
   for (int i = 0; i < 32; ++i)
@@ -29,7 +32,10 @@ __device__ __forceinline__ void stage_store_bf16(uint8_t* stg, int lane, const u
     const int part = lane & 3;
     if (r < rows) {
       const uint4 val = *reinterpret_cast<const uint4*>(stg + r * 64 + part * 16);
-      *reinterpret_cast<uint4*>(out + r * ld + part * 8) = val;
+      if (l2_policy)
+        st_global_v4_hint(out + r * ld + part * 8, val, l2_policy);
+      else
+        *reinterpret_cast<uint4*>(out + r * ld + part * 8) = val;
     }
   }
   __syncwarp();

@@ -209,6 +209,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;             // TMEM lane quadrant
     const int half = (warp - 4) >> 2;   // which 32-column chunks
+    const uint64_t pol_out = p.l2_stream ? l2_policy_evict_first() : 0;
     const uint32_t acc_empty_cl0 = mapa_shared(smem_u32(&acc_empty_bar[0]), 0);
     const uint32_t acc_empty_cl1 = mapa_shared(smem_u32(&acc_empty_bar[1]), 0);
     int local = 0;
@@ -262,13 +263,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
           const int f = tl.m * GEMM_BM + static_cast<int>(rank) * 64 + (q & 1) * 32;
           if (rows > 0)
             stage_store_bf16(reinterpret_cast<uint8_t*>(mine), lane, h, nmine, rows,
-                             out + (row_of_tok0 + c0 + start) * p.out_ld + f, p.out_ld);
+                             out + (row_of_tok0 + c0 + start) * p.out_ld + f, p.out_ld,
+                             pol_out);
         } else {
           const int rows = min(ncol, tl.count - tok_base);
           const int f = tl.m * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM + q * 32;
           uint8_t* stg = epi + (warp - 4) * 2048;
           stage_store_bf16(stg, lane, r, ncol, rows, out + (row_of_tok0 + c0) * p.out_ld + f,
-                           p.out_ld);
+                           p.out_ld, pol_out);
         }
       }
       tc_fence_before();

@@ -64,6 +64,8 @@ struct GemmParams {
   long long split_stride;
   int single_a;           // MODE_ROUTER/MODE_DOWN: 1 = one 128-row A block per tile (no pair)
   int mgroup;             // pair kernel: weight blocks per tile group (divides mblocks; 0 = all)
+  int l2_stream;          // 1: weight and token tiles loaded, and outputs stored, with an
+                          // L2 evict-first policy (decode: every weight byte is read once)
   int mblocks;            // tiles along the weight rows of one group
   int a_rows;             // weight rows per group: E (router), I (gate/up), d (down)
   void* out;              // fp32 logits [T, E] | bf16 H [rows, I] | bf16 Y [rows, d]

@@ -396,6 +396,8 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       pg.out_ld = I;
       pg.err = err;
       pg.wait_ns = wait_ns;
+      // decode-sized batches stream every weight byte once
+      pg.l2_stream = T < 4 * GEMM_BN ? 1 : 0;
       const int64_t g_ub = tiles_ub * pg.mblocks;
       CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, pg, static_cast<int>(g_ub < c.sms ? g_ub : c.sms),
                      st));
