@@ -111,14 +111,18 @@ class Dist:
         if self.world != n_gpus:
             raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={self.world}: launch N>1 with torchrun")
         self.pg = None
+        self.cuda = torch.cuda.is_available()
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                    device_id=torch.device("cuda", self.local))
+            if self.cuda:
+                torch.cuda.set_device(self.local)
+                dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                        device_id=torch.device("cuda", self.local))
+            else:   # host-only ranks (tests of this plumbing)
+                dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
             self.pg = dist
-        elif torch.cuda.is_available():
+        elif self.cuda:
             torch.cuda.set_device(0)
 
     def barrier(self):
@@ -126,9 +130,10 @@ class Dist:
             self.pg.barrier()
 
     def max(self, v: float) -> float:
+        """The largest v over all ranks (step times: the slowest rank sets the pace)."""
         if not self.pg:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device="cuda" if self.cuda else "cpu")
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
