@@ -41,6 +41,35 @@ __device__ __forceinline__ void stage_store_bf16(uint8_t* stg, int lane, const u
   __syncwarp();
 }
 
+// As stage_store_bf16, from results already rounded to bf16 and packed in
+// pairs (v[i] holds tokens 2i and 2i+1 in its low and high halves).
+__device__ __forceinline__ void stage_store_bf16x2(uint8_t* stg, int lane, const uint32_t (&v)[16],
+                                                   int ncol, int rows, __nv_bfloat16* out,
+                                                   int64_t ld, uint64_t l2_policy) {
+  uint16_t* st = reinterpret_cast<uint16_t*>(stg);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (2 * i < ncol) {
+      st[(2 * i) * 32 + lane] = static_cast<uint16_t>(v[i] & 0xFFFFu);
+      st[(2 * i + 1) * 32 + lane] = static_cast<uint16_t>(v[i] >> 16);
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = (lane >> 2) + 8 * k;
+    const int part = lane & 3;
+    if (r < rows) {
+      const uint4 val = *reinterpret_cast<const uint4*>(stg + r * 64 + part * 16);
+      if (l2_policy)
+        st_global_v4_hint(out + r * ld + part * 8, val, l2_policy);
+      else
+        *reinterpret_cast<uint4*>(out + r * ld + part * 8) = val;
+    }
+  }
+  __syncwarp();
+}
+
 // fp32 variant for the router's logits: features ebase + 0..31 of rows
 // tok_base + i, features >= E dropped; 128-byte rows, eight lanes per row,
 // staged 16 tokens at a time (2 KB).

@@ -16,18 +16,29 @@
 // hit by a handful of decode tokens costs an N = 16 MMA rather than a padded
 // 128-row one.
 //
-// A tile is (expert g, token tile j, weight block m): two A blocks (gate and
-// up rows of block m, or two consecutive 128-row blocks of W_down / W_r)
-// against up to 256 tokens, giving two 128 x N fp32 accumulators in TMEM
-// (columns 0..255 and 256..511).
+// A tile is (expert g, token tile j, weight block m): one or two A blocks
+// (gate and up rows of block m; two consecutive 128-row blocks of W_down or
+// W_r; or a single block) against up to 256 tokens.  Each A block gives one
+// 128 x N fp32 accumulator in TMEM; 256-token tiles keep the MMA at N = 256,
+// the shape whose operand traffic the tensor core and L2 sustain (128-token
+// tiles and single-block down tiles were measured slower).
 //
-// Persistent, warp-specialised CTA (384 threads, one per SM):
-//   warp 0      TMA producer: A blocks [128 x 64] and B boxes [32 x 64],
-//               128-byte swizzle, into a 3-stage shared-memory ring
+// Persistent, warp-specialised CTA (512 threads, one per SM):
+//   warp 0      TMA producer: A blocks [128 x 64] and B boxes (one [256 x 64]
+//               box for a full token tile, else [32 x 64] boxes), 128-byte
+//               swizzle, into a 3-stage shared-memory ring
 //   warp 1      MMA issuer: tcgen05.mma kind::f16, commits free the stage
-//   warp 2      TMEM allocator
-//   warps 4..11 epilogue: tcgen05.ld -> fp32 math -> shared staging ->
+//   warp 2      TMEM allocator (512 columns)
+//   warps 4..15 epilogue, three per TMEM lane quadrant: tcgen05.ld ->
+//               fp32 math -> bf16 in registers -> shared staging ->
 //               coalesced 16-byte global stores
+// The epilogue hands TMEM back as soon as it has read it, before it stores:
+//   * one-block tiles use 256 columns, so two accumulator buffers alternate
+//     and a tile's epilogue overlaps the next tile's MMAs;
+//   * two-block tiles fill all 512 columns; the epilogue releases the first
+//     accumulator, then the second, and the issuer starts the next tile's
+//     first-block MMAs on up to GEMM_STAGES loaded stages before it needs
+//     the second accumulator back.
 // Every wait is time-bounded (ptx.cuh); on running out the CTA drains its
 // in-flight copies and MMAs, frees TMEM and returns with the error flag set.
 #include "epilogue.cuh"
@@ -110,15 +121,108 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   return tl;
 }
 
+
+// One 64-wide K step of one A block: four K = 16 MMAs into accumulator d.
+__device__ __forceinline__ void mma_kstep(uint32_t d, uint32_t a_smem, uint32_t b_smem,
+                                          uint32_t idesc, bool first) {
+  const uint64_t ad = smem_desc_sw128(a_smem);
+  const uint64_t bd = smem_desc_sw128(b_smem);
+#pragma unroll
+  for (int kk = 0; kk < GEMM_BK / 16; ++kk)
+    umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (first && kk == 0) ? 0u : 1u);
+}
+
+// The epilogue chunks of warp group `group` (0..2) in its lane quadrant:
+// columns group * 32 + j * 96 (j = 0..2) below nmma, 32 wide (16 for a
+// ragged last chunk).
+//
+// Reads this warp's chunks of the accumulator at tacc (for gate/up also the
+// up accumulator 256 columns on), applies the epilogue math and rounds to
+// bf16: hp[j][i] holds tokens 2i and 2i+1 of chunk j.
+template <int MODE>
+__device__ __forceinline__ void epi_read_bf16(uint32_t tacc, int group, int nmma,
+                                              uint32_t (&hp)[3][16]) {
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    const int c0 = group * 32 + j * 32 * GEMM_EPI_GROUPS;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int cc = c0 + 16 * hh;
+      if (cc < nmma) {
+        uint32_t r0[16], r1[16];
+        tmem_ld16(tacc + cc, r0);
+        if (MODE == MODE_GATEUP) tmem_ld16(tacc + 256 + cc, r1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float v[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float g = __uint_as_float(r0[2 * i + h]);
+            if (MODE == MODE_GATEUP) {
+              const float u = __uint_as_float(r1[2 * i + h]);
+              // SiLU(g) * u; the exponent is clamped so 1 + e^-g stays finite
+              v[h] = __fdividef(g, 1.0f + __expf(-fmaxf(g, -80.0f))) * u;
+            } else {
+              v[h] = g;
+            }
+          }
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[0], v[1]);
+          hp[j][8 * hh + i] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+      }
+    }
+  }
+}
+
+// Stores the chunks epi_read_bf16 produced: token rows of the tile's slots,
+// 32 bf16 columns each from out (already offset to this warp's features).
+__device__ __forceinline__ void epi_store_bf16(uint8_t* stg, int lane, int group, const Tile& tl,
+                                               const uint32_t (&hp)[3][16], __nv_bfloat16* out,
+                                               int64_t ld, uint64_t pol) {
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    const int c0 = group * 32 + j * 32 * GEMM_EPI_GROUPS;
+    if (c0 < tl.nmma) {
+      const int ncol = c0 + 32 <= tl.nmma ? 32 : 16;
+      const int tok_base = tl.tok0 + c0;
+      const int rows = min(ncol, tl.count - tok_base);
+      const int64_t row0 = tl.brow0 - tl.tok0 + tok_base;   // first output row
+      stage_store_bf16x2(stg, lane, hp[j], ncol, rows, out + row0 * ld, ld, pol);
+    }
+  }
+}
+
+// Router logits (fp32) of one accumulator: weight rows ebase + 0..31 of this
+// warp's quadrant, chunk by chunk straight from TMEM to global memory.
+__device__ __forceinline__ void epi_router_f32(uint32_t tacc, uint8_t* stg, int lane, int group,
+                                               const Tile& tl, const GemmParams& p, int ebase) {
+  float* out = static_cast<float*>(p.out) + tl.split * p.split_stride;
+  for (int c0 = group * 32; c0 < tl.nmma; c0 += 32 * GEMM_EPI_GROUPS) {
+    const bool wide = c0 + 32 <= tl.nmma;
+    uint32_t r[32];
+    tmem_ld16(tacc + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+    if (wide) tmem_ld16(tacc + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+    tmem_ld_wait();
+    const int ncol = wide ? 32 : 16;
+    const int tok_base = tl.tok0 + c0;
+    const int rows = min(ncol, tl.count - tok_base);
+    stage_store_f32(stg, lane, r, ncol, rows, out, tok_base, p.out_ld, ebase, p.a_rows);
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-            const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+            const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBf,
+            const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[GEMM_STAGES];
   __shared__ __align__(8) uint64_t empty_bar[GEMM_STAGES];
-  __shared__ __align__(8) uint64_t acc_full_bar;
-  __shared__ __align__(8) uint64_t acc_empty_bar;
+  // Accumulator hand-over.  One-block tiles: [b] = buffer b (TMEM columns
+  // 256 b ..).  Two-block tiles: [0] / [1] = first / second accumulator.
+  __shared__ __align__(8) uint64_t acc_full_bar[2];
+  __shared__ __align__(8) uint64_t acc_empty_bar[2];
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
@@ -133,14 +237,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    mbar_init(&acc_full_bar, 1);
-    mbar_init(&acc_empty_bar, GEMM_EPI_THREADS);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full_bar[b], 1);
+      mbar_init(&acc_empty_bar[b], GEMM_EPI_THREADS);
+    }
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA0);
     tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmBf);
   }
   __syncwarp();
   if (warp == 2) {
@@ -156,6 +263,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   griddep_launch_dependents();
   const uint32_t tmem = tmem_base_sh;
   const int ntiles = total_tiles<MODE>(p);
+  // gate/up tiles always hold two blocks; router and down tiles hold one
+  // when p.single_a is set (1 buffer of 512 columns, or 2 of 256)
+  const int nbuf = (MODE == MODE_GATEUP || !p.single_a) ? 1 : 2;
 
   // Single-thread roles run on lane 0; the other lanes of their warp wait at
   // a __syncwarp so that every warp reaches the final CTA barrier converged.
@@ -170,6 +280,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x) {
       const Tile tl = decode_tile<MODE>(p, t);
       const int nbox = (tl.nmma + GEMM_B_BOX_ROWS - 1) / GEMM_B_BOX_ROWS;
+      const bool full_box = p.b_box_full && tl.nmma == GEMM_BN;   // one [256 x 64] copy
       const uint32_t bytes = GEMM_A_BYTES * (tl.has_a1 ? 2 : 1) +
                              nbox * GEMM_B_BOX_ROWS * GEMM_BK * 2;
       for (int ks = tl.k0; ks < tl.k1; ++ks) {
@@ -191,15 +302,23 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
           if (tl.has_a1)
             tma_load_2d_hint(st + GEMM_A_BYTES, &tmA1, &full_bar[stage], kc, tl.a1_row,
                              pol_stream);
-          for (int bx = 0; bx < nbox; ++bx)
-            tma_load_2d_hint(sb + bx * GEMM_B_BOX_ROWS * GEMM_BK * 2, &tmB, &full_bar[stage], kc,
-                             tl.brow0 + bx * GEMM_B_BOX_ROWS, pol_stream);
+          if (full_box) {
+            tma_load_2d_hint(sb, &tmBf, &full_bar[stage], kc, tl.brow0, pol_stream);
+          } else {
+            for (int bx = 0; bx < nbox; ++bx)
+              tma_load_2d_hint(sb + bx * GEMM_B_BOX_ROWS * GEMM_BK * 2, &tmB, &full_bar[stage],
+                               kc, tl.brow0 + bx * GEMM_B_BOX_ROWS, pol_stream);
+          }
         } else {
           tma_load_2d(st, &tmA0, &full_bar[stage], kc, tl.a0_row);
           if (tl.has_a1) tma_load_2d(st + GEMM_A_BYTES, &tmA1, &full_bar[stage], kc, tl.a1_row);
-          for (int bx = 0; bx < nbox; ++bx)
-            tma_load_2d(sb + bx * GEMM_B_BOX_ROWS * GEMM_BK * 2, &tmB, &full_bar[stage], kc,
-                        tl.brow0 + bx * GEMM_B_BOX_ROWS);
+          if (full_box) {
+            tma_load_2d(sb, &tmBf, &full_bar[stage], kc, tl.brow0);
+          } else {
+            for (int bx = 0; bx < nbox; ++bx)
+              tma_load_2d(sb + bx * GEMM_B_BOX_ROWS * GEMM_BK * 2, &tmB, &full_bar[stage], kc,
+                          tl.brow0 + bx * GEMM_B_BOX_ROWS);
+          }
         }
         if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
       }
@@ -217,31 +336,56 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     int local = 0;
     for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x, ++local) {
       const Tile tl = decode_tile<MODE>(p, t);
-      if (local > 0 && !mbar_wait(&acc_empty_bar, (local - 1) & 1, p.wait_ns, p.err)) {
+      const int buf = local % nbuf;
+      const int use = local / nbuf;
+      const uint32_t par = static_cast<uint32_t>(use - 1) & 1u;
+      const uint32_t acc0 = tmem + buf * 256;
+      if (use > 0 && !mbar_wait(&acc_empty_bar[buf], par, p.wait_ns, p.err)) {
         abort_sh = 1;
         break;
       }
       tc_fence_after();
       const uint32_t idesc = idesc_bf16_f32(GEMM_BM, tl.nmma);
+      const int nk = tl.k1 - tl.k0;
+      // Two-block tile after the first: the first npre loaded stages feed the
+      // first accumulator alone; they are freed once the second accumulator
+      // is back and has had its MMAs on them too.
+      const bool stagger = nbuf == 1 && use > 0;
+      const int npre = stagger ? min(nk, GEMM_STAGES) : 0;
       bool ok = true;
-      for (int ks = tl.k0; ks < tl.k1; ++ks) {
+      const int stage0 = stage;
+      for (int i = 0; i < npre; ++i) {
         if (!mbar_wait(&full_bar[stage], phase, p.wait_ns, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = smem_u32(smem + stage * GEMM_STAGE_BYTES);
-        const uint64_t a0 = smem_desc_sw128(st);
-        const uint64_t a1 = smem_desc_sw128(st + GEMM_A_BYTES);
-        const uint64_t bd = smem_desc_sw128(st + 2 * GEMM_A_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-          const uint32_t acc = (ks != tl.k0 || kk != 0) ? 1u : 0u;
-          umma_bf16(tmem, a0 + 2 * kk, bd + 2 * kk, idesc, acc);
-          if (tl.has_a1) umma_bf16(tmem + 256, a1 + 2 * kk, bd + 2 * kk, idesc, acc);
+        mma_kstep(acc0, st, st + 2 * GEMM_A_BYTES, idesc, i == 0);
+        if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (ok && stagger) {
+        if (!mbar_wait(&acc_empty_bar[1], par, p.wait_ns, p.err)) {
+          ok = false;
+        } else {
+          tc_fence_after();
+          int s = stage0;
+          for (int i = 0; i < npre; ++i) {
+            const uint32_t st = smem_u32(smem + s * GEMM_STAGE_BYTES);
+            if (tl.has_a1) mma_kstep(acc0 + 256, st + GEMM_A_BYTES, st + 2 * GEMM_A_BYTES, idesc, i == 0);
+            umma_commit(&empty_bar[s]);
+            if (++s == GEMM_STAGES) s = 0;
+          }
         }
+      }
+      for (int i = npre; ok && i < nk; ++i) {
+        if (!mbar_wait(&full_bar[stage], phase, p.wait_ns, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + stage * GEMM_STAGE_BYTES);
+        mma_kstep(acc0, st, st + 2 * GEMM_A_BYTES, idesc, i == 0);
+        if (tl.has_a1) mma_kstep(acc0 + 256, st + GEMM_A_BYTES, st + 2 * GEMM_A_BYTES, idesc, i == 0);
         umma_commit(&empty_bar[stage]);
         if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
       }
       if (!ok) { abort_sh = 1; break; }
-      umma_commit(&acc_full_bar);
+      umma_commit(&acc_full_bar[buf]);
     }
     // Drain: all MMAs issued by this thread finish before TMEM is freed.
     umma_commit(&drain_bar);
@@ -252,13 +396,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     // ------------------------------------------------------------ epilogue
     // Twelve warps: warp w drains TMEM lanes (w % 4) * 32 .. +31 (the quadrant
     // its warp id may access) and every third 32-column chunk of the tile
-    // (group = 0, 1 or 2).  Each chunk goes TMEM -> registers (one wait per
-    // chunk) -> math -> a per-warp staging tile in shared memory -> 16-byte
-    // coalesced global stores, one output row of 64 (bf16) or 128 (fp32)
-    // bytes per 4 or 8 lanes.
+    // (group = 0, 1 or 2), leaving through a per-warp staging tile in shared
+    // memory as 16-byte coalesced stores of 64-byte (bf16) or 128-byte
+    // (fp32) row pieces.
     const int q = warp & 3;
     const int group = (warp - 4) >> 2;
-    const int row_in_blk = q * 32 + lane;
     const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
     uint8_t* stg = smem + GEMM_STAGES * GEMM_STAGE_BYTES + (warp - 4) * GEMM_STG_BYTES;
     // H / Y rows are written once here; hint them only for streaming batches
@@ -266,59 +408,47 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     int local = 0;
     for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x, ++local) {
       const Tile tl = decode_tile<MODE>(p, t);
-      if (!mbar_wait(&acc_full_bar, local & 1, p.wait_ns, p.err)) {
+      const int buf = local % nbuf;
+      if (!mbar_wait(&acc_full_bar[buf], (local / nbuf) & 1, p.wait_ns, p.err)) {
         abort_sh = 1;
         break;
       }
       tc_fence_after();
-      for (int c0 = group * 32; c0 < tl.nmma; c0 += 32 * GEMM_EPI_GROUPS) {
-        const bool wide = c0 + 32 <= tl.nmma;   // 32 columns, else 16
-        uint32_t r0[32], r1[32];
-        tmem_ld16(tq + c0, *reinterpret_cast<uint32_t(*)[16]>(&r0[0]));
-        if (wide) tmem_ld16(tq + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r0[16]));
-        if (tl.has_a1) {
-          tmem_ld16(tq + 256 + c0, *reinterpret_cast<uint32_t(*)[16]>(&r1[0]));
-          if (wide) tmem_ld16(tq + 256 + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r1[16]));
+      const uint32_t tacc = tq + buf * 256;
+      const int row_blk = tl.m * (p.single_a ? 1 : 2) * GEMM_BM + q * 32;   // router / down
+      if (MODE == MODE_ROUTER) {
+        epi_router_f32(tacc, stg, lane, group, tl, p, row_blk);
+        tc_fence_before();
+        mbar_arrive(&acc_empty_bar[buf]);
+        if (nbuf == 1) {
+          if (tl.has_a1) epi_router_f32(tacc + 256, stg, lane, group, tl, p, row_blk + GEMM_BM);
+          tc_fence_before();
+          mbar_arrive(&acc_empty_bar[1]);
         }
-        tmem_ld_wait();
-        const int ncol = wide ? 32 : 16;
-        const int tok_base = tl.tok0 + c0;              // token index in group of column 0
-        const int rows = min(ncol, tl.count - tok_base);  // valid output rows
-        if (MODE == MODE_ROUTER) {
-          const int ebase = tl.m * (p.single_a ? 1 : 2) * GEMM_BM + q * 32;
-          float* out = static_cast<float*>(p.out) + tl.split * p.split_stride;
-          stage_store_f32(stg, lane, r0, ncol, rows, out, tok_base, p.out_ld, ebase, p.a_rows);
-          if (tl.has_a1)
-            stage_store_f32(stg, lane, r1, ncol, rows, out, tok_base, p.out_ld, ebase + GEMM_BM,
-                            p.a_rows);
-        } else if (MODE == MODE_GATEUP) {
-          uint32_t h[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float g = __uint_as_float(r0[i]);
-            const float u = __uint_as_float(r1[i]);
-            // SiLU(g) * u; the exponent is clamped so 1 + e^-g stays finite
-            h[i] = __float_as_uint(__fdividef(g, 1.0f + __expf(-fmaxf(g, -80.0f))) * u);
-          }
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-          const int64_t row0 = tl.brow0 - tl.tok0 + tok_base;   // first output row
-          stage_store_bf16(stg, lane, h, ncol, rows, out + row0 * p.out_ld + tl.m * GEMM_BM + q * 32,
-                           p.out_ld, pol_out);
-        } else {
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-          const int64_t row0 = tl.brow0 - tl.tok0 + tok_base;
-          const int f0 = tl.m * (p.single_a ? 1 : 2) * GEMM_BM + q * 32;
-          stage_store_bf16(stg, lane, r0, ncol, rows, out + row0 * p.out_ld + f0, p.out_ld,
-                           pol_out);
-          if (tl.has_a1)
-            stage_store_bf16(stg, lane, r1, ncol, rows, out + row0 * p.out_ld + f0 + GEMM_BM,
-                             p.out_ld, pol_out);
+      } else if (MODE == MODE_GATEUP) {
+        uint32_t hp[3][16];
+        epi_read_bf16<MODE_GATEUP>(tacc, group, tl.nmma, hp);
+        tc_fence_before();
+        mbar_arrive(&acc_empty_bar[0]);
+        mbar_arrive(&acc_empty_bar[1]);
+        epi_store_bf16(stg, lane, group, tl, hp,
+                       static_cast<__nv_bfloat16*>(p.out) + tl.m * GEMM_BM + q * 32, p.out_ld,
+                       pol_out);
+      } else {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row_blk;
+        uint32_t hp[3][16];
+        epi_read_bf16<MODE_DOWN>(tacc, group, tl.nmma, hp);
+        tc_fence_before();
+        mbar_arrive(&acc_empty_bar[buf]);
+        epi_store_bf16(stg, lane, group, tl, hp, out, p.out_ld, pol_out);
+        if (nbuf == 1) {
+          if (tl.has_a1) epi_read_bf16<MODE_DOWN>(tacc + 256, group, tl.nmma, hp);
+          tc_fence_before();
+          mbar_arrive(&acc_empty_bar[1]);
+          if (tl.has_a1) epi_store_bf16(stg, lane, group, tl, hp, out + GEMM_BM, p.out_ld, pol_out);
         }
       }
-      tc_fence_before();
-      mbar_arrive(&acc_empty_bar);
     }
-    (void)row_in_blk;
   }
 
   tc_fence_before();
@@ -332,8 +462,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
 }  // namespace
 
 cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap& a1,
-                        const CUtensorMap& b, const GemmParams& p, int grid,
-                        cudaStream_t stream) {
+                        const CUtensorMap& b, const CUtensorMap& b_full, const GemmParams& p,
+                        int grid, cudaStream_t stream) {
   if (grid <= 0) return cudaSuccess;
   cudaError_t e = cudaSuccess;
   switch (mode) {
@@ -341,22 +471,22 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
       e = cudaFuncSetAttribute(gemm_kernel<MODE_ROUTER>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
       if (e != cudaSuccess) return e;
-      e = launch_pdl(gemm_kernel<MODE_ROUTER>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES, stream,
-                     a0, a1, b, p);
+      e = launch_pdl(gemm_kernel<MODE_ROUTER>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES,
+                     stream, a0, a1, b, b_full, p);
       break;
     case MODE_GATEUP:
       e = cudaFuncSetAttribute(gemm_kernel<MODE_GATEUP>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
       if (e != cudaSuccess) return e;
-      e = launch_pdl(gemm_kernel<MODE_GATEUP>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES, stream,
-                     a0, a1, b, p);
+      e = launch_pdl(gemm_kernel<MODE_GATEUP>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES,
+                     stream, a0, a1, b, b_full, p);
       break;
     case MODE_DOWN:
       e = cudaFuncSetAttribute(gemm_kernel<MODE_DOWN>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
       if (e != cudaSuccess) return e;
-      e = launch_pdl(gemm_kernel<MODE_DOWN>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES, stream,
-                     a0, a1, b, p);
+      e = launch_pdl(gemm_kernel<MODE_DOWN>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES,
+                     stream, a0, a1, b, b_full, p);
       break;
   }
   if (e != cudaSuccess) return e;

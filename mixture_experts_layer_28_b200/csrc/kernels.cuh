@@ -66,6 +66,7 @@ struct GemmParams {
   int mgroup;             // pair kernel: weight blocks per tile group (divides mblocks; 0 = all)
   int l2_stream;          // 1: weight and token tiles loaded, and outputs stored, with an
                           // L2 evict-first policy (decode: every weight byte is read once)
+  int b_box_full;         // 1: a full token tile's B rows come in one GEMM_BN-row copy
   int mblocks;            // tiles along the weight rows of one group
   int a_rows;             // weight rows per group: E (router), I (gate/up), d (down)
   void* out;              // fp32 logits [T, E] | bf16 H [rows, I] | bf16 Y [rows, d]
@@ -74,9 +75,11 @@ struct GemmParams {
   long long wait_ns;      // bound of every pipeline wait
 };
 
+// b: B map with GEMM_B_BOX_ROWS-row boxes; b_full: with GEMM_BN-row boxes,
+// used for full token tiles when p.b_box_full is set.
 cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap& a1,
-                        const CUtensorMap& b, const GemmParams& p, int grid,
-                        cudaStream_t stream);
+                        const CUtensorMap& b, const CUtensorMap& b_full, const GemmParams& p,
+                        int grid, cudaStream_t stream);
 
 // The FFN expert GEMMs on CTA pairs (cta_group::2, M = 256 per MMA), for
 // batches with many tokens per expert; `clusters` pairs are launched.

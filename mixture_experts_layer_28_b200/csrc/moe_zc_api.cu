@@ -301,7 +301,9 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   if (T > 0) {
     // 1  router GEMM
     CUtensorMap mWr, mX;
-    if (!make_map(&mWr, W_r, E, d, GEMM_BM) || !make_map(&mX, x, T, d, GEMM_B_BOX_ROWS))
+    CUtensorMap mXf;   // full 256-token boxes of x
+    if (!make_map(&mWr, W_r, E, d, GEMM_BM) || !make_map(&mX, x, T, d, GEMM_B_BOX_ROWS) ||
+        !make_map(&mXf, x, T, d, T >= GEMM_BN ? GEMM_BN : GEMM_B_BOX_ROWS))
       return MOE_ZC_ERR_CUDA;
     GemmParams pr{};
     pr.G = 1;
@@ -322,7 +324,8 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     pr.ksplit = splits;
     pr.split_stride = T * E;
     const int64_t rgrid = rp.tiles * splits;
-    CK(launch_gemm(MODE_ROUTER, mWr, mWr, mX, pr,
+    pr.b_box_full = T >= GEMM_BN ? 1 : 0;
+    CK(launch_gemm(MODE_ROUTER, mWr, mWr, mX, mXf, pr,
                    static_cast<int>(rgrid < c.sms ? rgrid : c.sms), st));
     rec.mark(1);
     // 2  route
@@ -384,6 +387,13 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
           !make_map(&mWu, W_up, static_cast<uint64_t>(N) * I, d, GEMM_BM) ||
           !make_map(&mXp, c.Xp.p, c.rows_cap, d, GEMM_B_BOX_ROWS))
         return MOE_ZC_ERR_CUDA;
+      // full 256-token boxes of the permuted tokens and of H
+      CUtensorMap mXpf, mHf;
+      const bool full_ok = c.rows_cap >= GEMM_BN;
+      const uint32_t fbox = full_ok ? GEMM_BN : GEMM_B_BOX_ROWS;
+      if (!make_map(&mXpf, c.Xp.p, c.rows_cap, d, fbox) ||
+          !make_map(&mHf, c.H.p, c.rows_cap, I, fbox))
+        return MOE_ZC_ERR_CUDA;
       GemmParams pg{};
       pg.grp_count = cnt;
       pg.grp_off = grp_off;
@@ -397,9 +407,10 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       pg.err = err;
       pg.wait_ns = wait_ns;
       // decode-sized batches stream every weight byte once
-      pg.l2_stream = T < 4 * GEMM_BN ? 1 : 0;
+      pg.l2_stream = T < 1024 ? 1 : 0;
+      pg.b_box_full = full_ok ? 1 : 0;
       const int64_t g_ub = tiles_ub * pg.mblocks;
-      CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, pg, static_cast<int>(g_ub < c.sms ? g_ub : c.sms),
+      CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg, static_cast<int>(g_ub < c.sms ? g_ub : c.sms),
                      st));
       rec.mark(6);
       // 7  down GEMM
@@ -414,7 +425,7 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       pd.out = c.Y.p;
       pd.out_ld = d;
       const int64_t d_ub = tiles_ub * pd.mblocks;
-      CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, pd, static_cast<int>(d_ub < c.sms ? d_ub : c.sms),
+      CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd, static_cast<int>(d_ub < c.sms ? d_ub : c.sms),
                      st));
       rec.mark(7);
       }

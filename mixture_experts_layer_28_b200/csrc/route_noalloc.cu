@@ -148,7 +148,7 @@ extern "C" int moe_zc_route_noalloc(const void* x, const void* W_r, const float*
   pr.err = err;
   pr.wait_ns = kNoallocWaitNs;
   const int64_t tiles = ((T + GEMM_BN - 1) / GEMM_BN) * pr.mblocks;
-  if (launch_gemm(MODE_ROUTER, mWr, mWr, mX, pr, static_cast<int>(tiles < s->sms ? tiles : s->sms),
+  if (launch_gemm(MODE_ROUTER, mWr, mWr, mX, mX, pr, static_cast<int>(tiles < s->sms ? tiles : s->sms),
                   cs) != cudaSuccess ||
       launch_route(logits, b, logit_offset, T, static_cast<int>(E), N, K, idx, gate, zsum, counts,
                    cs) != cudaSuccess) {
