@@ -269,7 +269,8 @@ def cpu_baseline(w, ri, b, ew, target_s=12.0):
 # ----------------------------------------------------------------- arms
 def config_of(w, extra=None):
     c = {"workload": w.name, "T": w.T, "d": w.d, "N": w.N, "Z": w.Z, "K": w.K, "I": w.I,
-         "target_zero_frac": w.zero_frac, "zipf_s": w.zipf_s, "seed": w.seed}
+         "target_zero_frac": w.zero_frac, "zipf_s": w.zipf_s, "seed": w.seed,
+         "ffn_bias": "U[-0.1,0.1]" if w.bias == "random" else "0"}
     if extra:
         c.update(extra)
     return c

@@ -11,6 +11,14 @@ to every zero-computation expert's entry so that a stated share of all picks
 lands on zero experts.  The skewed workload also gives each FFN expert a
 Zipf(s) router-logit offset (offset_i = -s * ln(rank_i)).
 
+Because |b| (up to 0.1) is far above a typical softmax score (~1/E), that
+bias decides most picks and the FFN load is concentrated on a few dozen
+experts.  Two balanced companions of the LongCat-shaped workloads
+(``prefill_balanced``, ``decode_balanced``: same seeds, x and W_r) set the
+FFN experts' bias to zero instead, so the softmax scores decide among the
+FFN experts and every expert gets about the same expected load -- the state
+the bias controller steers towards.
+
 Where the numbers come from:
   * x, W_r, b and the Zipf ranks come from a CPU ``torch.Generator`` seeded
     with the workload seed, in that order.  Routing depends only on these, so
@@ -45,6 +53,7 @@ class Workload:
     zero_frac: Optional[float] = None   # target share of picks on zero experts
     zipf_s: Optional[float] = None      # Zipf exponent of the logit offset
     delta: float = 0.0                  # shift added to the zero experts' bias
+    bias: str = "random"                # b0: "random" U[-0.1, 0.1], or "zero"
 
     @property
     def E(self) -> int:
@@ -70,6 +79,10 @@ WORKLOADS = {
                  seed=2, zero_frac=0.30),
         Workload("decode", T=64, d=6144, N=512, Z=256, K=12, I=2048, w_std=0.01,
                  seed=3, zero_frac=0.40),
+        Workload("prefill_balanced", T=16384, d=6144, N=512, Z=256, K=12, I=2048,
+                 w_std=0.01, seed=2, zero_frac=0.30, bias="zero"),
+        Workload("decode_balanced", T=64, d=6144, N=512, Z=256, K=12, I=2048, w_std=0.01,
+                 seed=3, zero_frac=0.40, bias="zero"),
         Workload("skewed20", T=32768, d=4096, N=256, Z=128, K=8, I=1536, w_std=0.02,
                  seed=4, zero_frac=0.20, zipf_s=1.1),
         Workload("skewed40", T=32768, d=4096, N=256, Z=128, K=8, I=1536, w_std=0.02,
@@ -109,6 +122,8 @@ def routing_inputs(w: Workload, T: Optional[int] = None) -> RoutingInputs:
     x = torch.randn(w.T, w.d, generator=g, dtype=torch.float32).to(torch.bfloat16)
     W_r = (torch.randn(w.E, w.d, generator=g, dtype=torch.float32) * w.w_std).to(torch.bfloat16)
     b0 = torch.rand(w.E, generator=g, dtype=torch.float32) * 0.2 - 0.1
+    if w.bias == "zero":        # drawn all the same, so later draws do not move
+        b0 = torch.zeros_like(b0)
     off = None
     if w.zipf_s is not None:
         rank = torch.randperm(w.N, generator=g) + 1           # rank 1..N per FFN expert

@@ -170,7 +170,7 @@ def test_logit_offset_moves_routing():
     _full_check(Case(w))
 
 
-@pytest.mark.parametrize("name", ["decode", "prefill"])
+@pytest.mark.parametrize("name", ["decode", "prefill", "decode_balanced", "prefill_balanced"])
 def test_full_size_longcat_shaped(name):
     _sampled_check(Case(wl.get(name)))
 

@@ -43,10 +43,33 @@ def test_zipf_offset():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["prefill", "decode", "skewed20", "skewed40", "skewed60"])
+@pytest.mark.parametrize("name", ["prefill", "decode", "skewed20", "skewed40", "skewed60",
+                                  "prefill_balanced", "decode_balanced"])
 def test_calibrated_zero_share(name):
     """The stored bias shift gives the workload's zero-expert share (fp64 router)."""
     w = wl.get(name)
     ri = wl.routing_inputs(w)
     r = ref.route(ri.x, ri.W_r, ri.bias(w.N, w.delta), w.N, w.K, ri.logit_offset)
     assert abs(ref.zero_pick_fraction(r.idx, w.N) - w.zero_frac) <= 0.005
+
+
+def test_balanced_companions_share_x_and_router():
+    """The balanced workloads differ from their LongCat-shaped twins only in b:
+    same x and W_r, FFN bias zero, and one shift on the zero experts."""
+    for name in ["prefill", "decode"]:
+        w, wb = wl.get(name, T=32), wl.get(name + "_balanced", T=32)
+        a, b = wl.routing_inputs(w), wl.routing_inputs(wb)
+        assert torch.equal(a.x, b.x) and torch.equal(a.W_r, b.W_r)
+        bb = b.bias(wb.N, wb.delta)
+        assert torch.all(bb[: wb.N] == 0) and torch.all(bb[wb.N:] == wb.delta)
+
+
+@pytest.mark.slow
+def test_balanced_prefill_spreads_load():
+    """With no FFN bias every FFN expert is hit and none takes more than a
+    few times the mean load (fp64 router)."""
+    w = wl.get("prefill_balanced")
+    ri = wl.routing_inputs(w)
+    r = ref.route(ri.x, ri.W_r, ri.bias(w.N, w.delta), w.N, w.K)
+    ffn = ref.expert_load(r.idx, w.E)[: w.N]
+    assert (ffn > 0).all() and ffn.max() < 2 * ffn.mean()
