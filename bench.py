@@ -58,11 +58,11 @@ KERNELS_PER_FORWARD = 8   # router_gemm, route, scan, assign, permute, gateup, d
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel
 # from an ncu capture of the current kernel build at the full workload (one
-# pass; profiles/gemm_traffic_fullsize.md), per workload.  Clear an entry when
-# that kernel changes.
+# pass; the full-size GEMM traffic summary under profiles/), per workload.
+# Clear an entry when that kernel changes.
 NCU_TRAFFIC_BYTES = {
-    "prefill": 7_902_767_872 + 560_506_624,    # gate/up GEMM
-    "decode": 1_520_840_704 + 3_909_376,       # gate/up GEMM
+    "prefill": 8_755_961_088 + 561_242_624,    # gate/up GEMM
+    "decode": 1_520_849_408 + 4_829_696,       # gate/up GEMM
 }
 
 
