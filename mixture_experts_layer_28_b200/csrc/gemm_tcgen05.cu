@@ -104,8 +104,20 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
     tl.count = __ldg(p.grp_count + lo);
     tl.brow0 = __ldg(p.grp_off + lo);
   }
-  tl.tok0 = j * GEMM_BN;
-  tl.ntok = min(GEMM_BN, tl.count - tl.tok0);
+  // An expert's ntt = ceil(count / 256) token tiles share its tokens evenly
+  // (sizes a multiple of 16): two tiles of similar size run side by side in
+  // one round of the persistent grid and read the same weight blocks at the
+  // same pace, so the second read of a block is an L2 hit.
+  int tsz = GEMM_BN;
+  if (MODE != MODE_ROUTER) {
+    const int ntt = __ldg(p.grp_ttp + tl.g + 1) - __ldg(p.grp_ttp + tl.g);
+    if (ntt > 1) {
+      const int even = (((tl.count + ntt - 1) / ntt) + 15) & ~15;
+      if (static_cast<long long>(ntt - 1) * even < tl.count) tsz = even;   // last tile non-empty
+    }
+  }
+  tl.tok0 = j * tsz;
+  tl.ntok = min(tsz, tl.count - tl.tok0);
   tl.nmma = (tl.ntok + 15) & ~15;
   tl.brow0 += tl.tok0;
   if (MODE == MODE_GATEUP) {
