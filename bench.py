@@ -77,6 +77,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--chunk-tokens", type=int, default=0,
                     help="chunk size of the host-buffer forward (0: library default)")
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of one forward captured into a CUDA graph")
     ap.add_argument("--shape", default="",
                     help="override workload sizes, e.g. T=4096,N=32,Z=16 (for profiling runs)")
     return ap.parse_args()
@@ -296,6 +298,24 @@ def run_ours(args, dist, w):
     st = routing_stats(w, mz.expert_load(w.E))
     rf = roofline_numbers(w, st, pk)
 
+    # --graph: the forward captured once into a CUDA graph (its launches on
+    # the capture stream), each timed step one replay
+    graph = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            mz.forward(dev["x"], dev["W_r"], dev["b"], ew.W_gate, ew.W_up, ew.W_down,
+                       w.N, w.Z, w.K, out=out, logit_offset=dev["off"])
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+
+    def timed_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
+
     # ---- device-resident timed region (no per-stage events: they would
     # separate the kernels and undo the overlap of dependent launches)
     clocks = ClockSampler(dist.local) if dist.rank == 0 else None
@@ -306,7 +326,7 @@ def run_ours(args, dist, w):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        step()
+        timed_step()
     e1.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
@@ -402,6 +422,7 @@ def run_ours(args, dist, w):
         "data": "synthetic: seeded inputs, random-init weights of the workload's shapes",
         "config": config_of(w, {
             "global_batch": w.T * dist.world, "parallelism": f"replicas{dist.world}",
+            "cuda_graph": bool(args.graph),
             "l2": f"no flush: expert weights touched per step {touched / 1e9:.2f} GB > L2 126 MB"}),
         "e2e": {"value": dist.world * w.T / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": int(x_host.numel() * 2),

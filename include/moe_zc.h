@@ -73,6 +73,10 @@ typedef enum moe_zc_status {
  * W_gate/W_up/W_down may be NULL only when N == 0.
  * Asynchronous on `stream`; the expert-load histogram and routing of this
  * call stay available through moe_zc_expert_load / moe_zc_last_routing.
+ * The call may be captured into a CUDA graph (stream capture on `stream`,
+ * after moe_zc_reserve has sized the workspace, so that the captured call
+ * allocates nothing): each replay recomputes the layer from the buffers the
+ * call was given, and the result queries then wait for the whole device.
  */
 int moe_zc_forward(const void* x, const void* W_r, const float* b,
                    const void* W_gate, const void* W_up, const void* W_down,

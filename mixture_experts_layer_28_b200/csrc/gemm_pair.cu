@@ -310,13 +310,11 @@ cudaError_t launch_gemm_pair(GemmMode mode, const CUtensorMap& a0, const CUtenso
   cfg.numAttrs = 2;
   cudaError_t e;
   if (mode == MODE_GATEUP) {
-    e = cudaFuncSetAttribute(gemm_pair_kernel<MODE_GATEUP>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, PAIR_SMEM_BYTES);
+    e = smem_limit<gemm_pair_kernel<MODE_GATEUP>>(PAIR_SMEM_BYTES);
     if (e != cudaSuccess) return e;
     e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<MODE_GATEUP>, a0, a1, b, p);
   } else if (mode == MODE_DOWN) {
-    e = cudaFuncSetAttribute(gemm_pair_kernel<MODE_DOWN>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, PAIR_SMEM_BYTES);
+    e = smem_limit<gemm_pair_kernel<MODE_DOWN>>(PAIR_SMEM_BYTES);
     if (e != cudaSuccess) return e;
     e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<MODE_DOWN>, a0, a1, b, p);
   } else {

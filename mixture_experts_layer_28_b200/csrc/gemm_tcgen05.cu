@@ -64,10 +64,16 @@ struct Tile {
   int a0_row, a1_row;
 };
 
+__device__ __forceinline__ int router_tok_tile(const GemmParams& p) {
+  return p.tok_tile > 0 ? p.tok_tile : GEMM_BN;
+}
+
 template <int MODE>
 __device__ __forceinline__ int total_tiles(const GemmParams& p) {
-  if (MODE == MODE_ROUTER)
-    return ((p.T + GEMM_BN - 1) / GEMM_BN) * p.mblocks * (p.ksplit > 1 ? p.ksplit : 1);
+  if (MODE == MODE_ROUTER) {
+    const int tt = router_tok_tile(p);
+    return ((p.T + tt - 1) / tt) * p.mblocks * (p.ksplit > 1 ? p.ksplit : 1);
+  }
   return __ldg(p.grp_ttp + p.G) * p.mblocks;
 }
 
@@ -78,7 +84,7 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   tl.k0 = 0;
   tl.k1 = p.ksteps;
   if (MODE == MODE_ROUTER && p.ksplit > 1) {
-    const int per = ((p.T + GEMM_BN - 1) / GEMM_BN) * p.mblocks;
+    const int per = ((p.T + router_tok_tile(p) - 1) / router_tok_tile(p)) * p.mblocks;
     tl.split = t / per;
     t -= tl.split * per;
     tl.k0 = static_cast<int>(static_cast<long long>(p.ksteps) * tl.split / p.ksplit);
@@ -108,7 +114,7 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   // (sizes a multiple of 16): two tiles of similar size run side by side in
   // one round of the persistent grid and read the same weight blocks at the
   // same pace, so the second read of a block is an L2 hit.
-  int tsz = GEMM_BN;
+  int tsz = MODE == MODE_ROUTER ? router_tok_tile(p) : GEMM_BN;
   if (MODE != MODE_ROUTER) {
     const int ntt = __ldg(p.grp_ttp + tl.g + 1) - __ldg(p.grp_ttp + tl.g);
     if (ntt > 1) {
@@ -292,9 +298,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x) {
       const Tile tl = decode_tile<MODE>(p, t);
       const int nbox = (tl.nmma + GEMM_B_BOX_ROWS - 1) / GEMM_B_BOX_ROWS;
-      const bool full_box = p.b_box_full && tl.nmma == GEMM_BN;   // one [256 x 64] copy
+      // a full token tile (256 tokens; the router's tile size) in one copy
+      // of the b_full map, whose box has exactly that many rows
+      const int full_rows = MODE == MODE_ROUTER ? router_tok_tile(p) : GEMM_BN;
+      const bool full_box = p.b_box_full && tl.nmma == full_rows;
       const uint32_t bytes = GEMM_A_BYTES * (tl.has_a1 ? 2 : 1) +
-                             nbox * GEMM_B_BOX_ROWS * GEMM_BK * 2;
+                             (full_box ? tl.nmma : nbox * GEMM_B_BOX_ROWS) * GEMM_BK * 2;
       for (int ks = tl.k0; ks < tl.k1; ++ks) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1, p.wait_ns, p.err)) {
           abort_sh = 1;
@@ -480,22 +489,19 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
   cudaError_t e = cudaSuccess;
   switch (mode) {
     case MODE_ROUTER:
-      e = cudaFuncSetAttribute(gemm_kernel<MODE_ROUTER>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+      e = smem_limit<gemm_kernel<MODE_ROUTER>>(GEMM_SMEM_BYTES);
       if (e != cudaSuccess) return e;
       e = launch_pdl(gemm_kernel<MODE_ROUTER>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES,
                      stream, a0, a1, b, b_full, p);
       break;
     case MODE_GATEUP:
-      e = cudaFuncSetAttribute(gemm_kernel<MODE_GATEUP>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+      e = smem_limit<gemm_kernel<MODE_GATEUP>>(GEMM_SMEM_BYTES);
       if (e != cudaSuccess) return e;
       e = launch_pdl(gemm_kernel<MODE_GATEUP>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES,
                      stream, a0, a1, b, b_full, p);
       break;
     case MODE_DOWN:
-      e = cudaFuncSetAttribute(gemm_kernel<MODE_DOWN>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+      e = smem_limit<gemm_kernel<MODE_DOWN>>(GEMM_SMEM_BYTES);
       if (e != cudaSuccess) return e;
       e = launch_pdl(gemm_kernel<MODE_DOWN>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES,
                      stream, a0, a1, b, b_full, p);

@@ -28,6 +28,55 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once: later calls only read a per-device cache, so a forward makes
+// no attribute calls after its first (e.g. while a caller captures it into a
+// CUDA graph).
+template <auto Kernel>
+inline cudaError_t smem_limit(int bytes) {
+  static int done[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = bytes;
+  return e;
+}
+
+// Resident blocks per SM of a kernel at (threads, smem), cached per device
+// for the last smem asked.
+template <auto Kernel>
+inline int blocks_per_sm(int threads, size_t smem) {
+  static int cached[64] = {0};
+  static size_t cached_smem[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = -1;
+  if (dev >= 0 && cached[dev] > 0 && cached_smem[dev] == smem) return cached[dev];
+  int n = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, threads, smem) != cudaSuccess ||
+      n < 1)
+    n = 1;
+  if (dev >= 0) {
+    cached[dev] = n;
+    cached_smem[dev] = smem;
+  }
+  return n;
+}
+
+// Multiprocessors of the current device (cached).
+inline int device_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 // ------------------------------------------------------------------ GEMM
 // One tcgen05 engine serves the three contractions of the layer.  Weights are
 // the A operand (M = 128 rows per MMA, two A blocks per tile -> two fp32
@@ -67,6 +116,7 @@ struct GemmParams {
   int l2_stream;          // 1: weight and token tiles loaded, and outputs stored, with an
                           // L2 evict-first policy (decode: every weight byte is read once)
   int b_box_full;         // 1: a full token tile's B rows come in one GEMM_BN-row copy
+  int tok_tile;           // MODE_ROUTER: tokens per tile (multiple of 16, <= GEMM_BN; 0: GEMM_BN)
   int mblocks;            // tiles along the weight rows of one group
   int a_rows;             // weight rows per group: E (router), I (gate/up), d (down)
   void* out;              // fp32 logits [T, E] | bf16 H [rows, I] | bf16 Y [rows, d]

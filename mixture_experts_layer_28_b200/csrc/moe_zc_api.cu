@@ -53,6 +53,7 @@ struct Ctx {
   bool counts_total = false;   // last forward was chunked: report cnt_total
   cudaEvent_t done = nullptr;
   bool has_result = false;
+  bool done_valid = false;     // `done` marks the last forward (false: it was captured)
   int64_t T = 0;
   int d = 0, N = 0, Z = 0, K = 0, I = 0;
   int64_t rows_cap = 0;
@@ -152,12 +153,29 @@ int get_ctx(Ctx** out) {
 // blocks and K is not split.
 struct RouterPlan {
   int single_a, mblocks, splits;
+  int tok_tile;    // tokens per tile
   int64_t tiles;   // token tiles x weight blocks (per slice)
 };
 RouterPlan router_plan(int64_t T, int E, int ksteps, int sms) {
-  RouterPlan rp{0, (E + 2 * GEMM_BM - 1) / (2 * GEMM_BM), 1, 0};
+  RouterPlan rp{0, (E + 2 * GEMM_BM - 1) / (2 * GEMM_BM), 1, GEMM_BN, 0};
   const int64_t ttiles = (T + GEMM_BN - 1) / GEMM_BN;
   rp.tiles = ttiles * rp.mblocks;
+  if (rp.tiles >= sms) {
+    // Many tiles: the token tile size (176..256 tokens) that finishes in the
+    // least time, taking each wave of `sms` tiles to last as long as its
+    // tile size (e.g. T = 16384, E = 768: 282 tiles of 176 tokens in two
+    // waves rather than 192 of 256 in two, the second a third full).
+    int64_t best = -1;
+    for (int tt = GEMM_BN; tt >= 176; tt -= 16) {
+      const int64_t tiles = (T + tt - 1) / tt * rp.mblocks;
+      const int64_t cost = (tiles + sms - 1) / sms * tt;
+      if (best < 0 || cost < best) {
+        best = cost;
+        rp.tok_tile = tt;
+        rp.tiles = tiles;
+      }
+    }
+  }
   if (rp.tiles > 0 && rp.tiles < sms / 2) {
     rp.single_a = 1;
     rp.mblocks = (E + GEMM_BM - 1) / GEMM_BM;
@@ -289,10 +307,15 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   int* grp_ttp = static_cast<int*>(c.grp_ttp.p);
   int* fill = static_cast<int*>(c.fill.p);
 
+  // A forward captured into a CUDA graph by the caller records no events:
+  // an event recorded during capture cannot be waited on afterwards.
+  cudaStreamCaptureStatus capturing = cudaStreamCaptureStatusNone;
+  CK(cudaStreamIsCapturing(st, &capturing));
+  const bool captured = capturing != cudaStreamCaptureStatusNone;
   StageRec rec;
   int dev_now = -1;
   cudaGetDevice(&dev_now);
-  if (g_prof.on && g_prof.device == dev_now && g_prof.n < kRing) {
+  if (!captured && g_prof.on && g_prof.device == dev_now && g_prof.n < kRing) {
     rec.ev = g_prof.ev[g_prof.n];
     rec.st = st;
   }
@@ -301,9 +324,12 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   if (T > 0) {
     // 1  router GEMM
     CUtensorMap mWr, mX;
-    CUtensorMap mXf;   // full 256-token boxes of x
+    const RouterPlan rp = router_plan(T, E, d / GEMM_BK, c.sms);
+    // x in boxes of 32 tokens, and of one full token tile (rp.tok_tile)
+    CUtensorMap mXf;
+    const bool full_ok = T >= rp.tok_tile;
     if (!make_map(&mWr, W_r, E, d, GEMM_BM) || !make_map(&mX, x, T, d, GEMM_B_BOX_ROWS) ||
-        !make_map(&mXf, x, T, d, T >= GEMM_BN ? GEMM_BN : GEMM_B_BOX_ROWS))
+        !make_map(&mXf, x, T, d, full_ok ? rp.tok_tile : GEMM_B_BOX_ROWS))
       return MOE_ZC_ERR_CUDA;
     GemmParams pr{};
     pr.G = 1;
@@ -317,14 +343,14 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     // Few token tiles (decode): single blocks and K slices so that every SM
     // streams a part of W_r; the slices' partial logits are summed in slice
     // order by the route kernel.
-    const RouterPlan rp = router_plan(T, E, pr.ksteps, c.sms);
     pr.mblocks = rp.mblocks;
     pr.single_a = rp.single_a;
+    pr.tok_tile = rp.tok_tile;
     const int splits = rp.splits;
     pr.ksplit = splits;
     pr.split_stride = T * E;
     const int64_t rgrid = rp.tiles * splits;
-    pr.b_box_full = T >= GEMM_BN ? 1 : 0;
+    pr.b_box_full = full_ok ? 1 : 0;
     CK(launch_gemm(MODE_ROUTER, mWr, mWr, mX, mXf, pr,
                    static_cast<int>(rgrid < c.sms ? rgrid : c.sms), st));
     rec.mark(1);
@@ -443,7 +469,8 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   }
   rec.mark(8);
   if (rec.ev) ++g_prof.n;
-  CK(cudaEventRecord(c.done, st));
+  if (!captured) CK(cudaEventRecord(c.done, st));
+  c.done_valid = !captured;
   c.has_result = true;
   c.counts_total = false;
   c.T = T;
@@ -535,6 +562,7 @@ int forward_host_impl(const void* x_host, const void* W_r, const float* b, const
   // the caller's stream completes only after every copy out
   for (int i = 0; i < 2 && i < nchunks; ++i) CK(cudaStreamWaitEvent(st, c.ev_out[i], 0));
   CK(cudaEventRecord(c.done, st));
+  c.done_valid = true;
   c.has_result = true;
   c.counts_total = true;
   c.N = N;
@@ -544,7 +572,12 @@ int forward_host_impl(const void* x_host, const void* W_r, const float* b, const
 
 int sync_impl(Ctx& c) {
   if (!c.has_result) return MOE_ZC_ERR_NO_RESULT;
-  CK(cudaEventSynchronize(c.done));
+  // after a captured forward its replays are the caller's: wait for the device
+  if (c.done_valid) {
+    CK(cudaEventSynchronize(c.done));
+  } else {
+    CK(cudaDeviceSynchronize());
+  }
   int e = 0;
   CK(cudaMemcpy(&e, c.err.p, sizeof(int), cudaMemcpyDeviceToHost));
   if (e != 0) {

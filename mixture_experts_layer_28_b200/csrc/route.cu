@@ -246,9 +246,7 @@ template <int VPL, bool SLICED>
 cudaError_t launch_route_kernel(const float* logits, const float* b, const float* offset,
                                 int64_t T, int E, int N, int K, int* idx, float* gate,
                                 float* zsum, int* cnt, cudaStream_t stream, int splits) {
-  int dev = 0, sms = 148, per_sm = 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sms();
   // tokens per block step: ROUTE_WARPS, or for sliced logits of few tokens
   // fewer, so that about two blocks per SM share the slice sums
   int tps = ROUTE_WARPS;
@@ -259,17 +257,12 @@ cudaError_t launch_route_kernel(const float* logits, const float* b, const float
   const size_t smem =
       E * sizeof(int) + (SLICED && tps < ROUTE_WARPS ? static_cast<size_t>(tps) * E * sizeof(float) : 0);
   if (smem > 48 * 1024) {
-    const cudaError_t e = cudaFuncSetAttribute(route_kernel<VPL, SLICED>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem));
+    const cudaError_t e = smem_limit<route_kernel<VPL, SLICED>>(static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
   // one wave of resident blocks, each walking many token steps, so the
   // per-block histogram zeroing and flush are paid once per block
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_kernel<VPL, SLICED>,
-                                                    ROUTE_WARPS * 32, smem) != cudaSuccess ||
-      per_sm < 1)
-    per_sm = 1;
+  const int per_sm = blocks_per_sm<route_kernel<VPL, SLICED>>(ROUTE_WARPS * 32, smem);
   const int64_t want = (T + tps - 1) / tps;
   const int64_t cap = static_cast<int64_t>(sms) * per_sm;
   const int grid = static_cast<int>(want < cap ? want : cap);

@@ -136,6 +136,14 @@ def test_odd_weight_blocks():
     _full_check(Case(w))
 
 
+def test_router_token_tiles_sized_to_waves():
+    """40000 tokens fill more than one wave of router tiles, so the router
+    GEMM takes 176-token tiles (two full waves instead of 157 tiles of 256):
+    ragged last tile and a one-copy box of 176 rows."""
+    w = wl.get("tiny", d=128, I=128, T=40000)
+    _full_check(Case(w))
+
+
 def test_empty_batch_is_noop():
     w = wl.get("tiny")
     case = Case(wl.get("tiny", T=1))
