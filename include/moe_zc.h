@@ -77,6 +77,10 @@ typedef enum moe_zc_status {
  * after moe_zc_reserve has sized the workspace, so that the captured call
  * allocates nothing): each replay recomputes the layer from the buffers the
  * call was given, and the result queries then wait for the whole device.
+ * Batches of 1024 tokens or more leave a copy of their expert-load histogram
+ * in pinned host memory (asynchronously); a later forward on the device uses
+ * it to choose how the expert GEMMs are launched.  That choice changes speed
+ * only: every launch gives the same bits.
  */
 int moe_zc_forward(const void* x, const void* W_r, const float* b,
                    const void* W_gate, const void* W_up, const void* W_down,

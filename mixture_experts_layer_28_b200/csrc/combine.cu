@@ -10,7 +10,9 @@
 // with zsum_t the router's sum of zero-expert gates.  fp32 accumulation in a
 // fixed order (zero experts first, then picks k = 0..K-1), one rounding to
 // bf16: the result does not depend on where the dispatch put a token's rows.
-// One CTA per token; each thread handles 8 features with 16-byte loads.
+// One CTA per token and part of the row (few tokens: several parts, so that
+// more SMs keep loads in flight); each thread handles 8 features at a time
+// with 16-byte loads.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -31,6 +33,9 @@ __global__ void combine_kernel(const uint4* __restrict__ x, const uint4* __restr
                                const float* __restrict__ zsum, int d8, int K,
                                uint4* __restrict__ out) {
   const int64_t t = blockIdx.x;
+  const int part = blockIdx.y, parts = gridDim.y;   // this CTA's share of the row
+  const int c_begin = static_cast<int>(static_cast<int64_t>(d8) * part / parts);
+  const int c_end = static_cast<int>(static_cast<int64_t>(d8) * (part + 1) / parts);
   __shared__ int sl[MOE_MAX_K_INTERNAL];
   __shared__ float gt[MOE_MAX_K_INTERNAL];
   __shared__ int nffn;
@@ -47,7 +52,7 @@ __global__ void combine_kernel(const uint4* __restrict__ x, const uint4* __restr
   __syncthreads();
   const float z = zsum[t];
   const int n = nffn;
-  for (int c = threadIdx.x; c < d8; c += blockDim.x) {
+  for (int c = c_begin + threadIdx.x; c < c_end; c += blockDim.x) {
     float a[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) a[i] = 0.f;
@@ -71,8 +76,15 @@ cudaError_t launch_combine(const __nv_bfloat16* x, const __nv_bfloat16* Y, const
                            __nv_bfloat16* out, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
   const int d8 = d / 8;
-  const int threads = d8 < 256 ? ((d8 + 31) / 32) * 32 : 256;
-  return launch_pdl(combine_kernel, dim3(static_cast<unsigned>(T)), dim3(threads), 0, stream,
+  // few tokens: split each row over up to 8 CTAs (at least 128 vectors each)
+  // so that about two CTAs per SM are busy
+  const int64_t want = (2LL * device_sms() + T - 1) / T;
+  int parts = static_cast<int>(want < 8 ? want : 8);
+  while (parts > 1 && d8 / parts < 128) --parts;
+  if (parts < 1) parts = 1;
+  const int per = (d8 + parts - 1) / parts;
+  const int threads = per < 256 ? ((per + 31) / 32) * 32 : 256;
+  return launch_pdl(combine_kernel, dim3(static_cast<unsigned>(T), parts), dim3(threads), 0, stream,
                     reinterpret_cast<const uint4*>(x), reinterpret_cast<const uint4*>(Y), slot,
                     gate, zsum, d8, K, reinterpret_cast<uint4*>(out));
 }

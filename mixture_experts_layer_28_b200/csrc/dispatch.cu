@@ -12,8 +12,9 @@
 //   assign    one thread per (token, pick): lanes of a warp that picked the
 //             same expert are grouped with __match_any_sync and take their
 //             slots with one atomicAdd per group (warp-aggregated atomics).
-//   permute   one CTA per token: copies x_t (16-byte vectors) to each of its
-//             FFN slots of Xp, the B operand of the gate/up GEMM.
+//   permute   one CTA per token (per part of its row for few tokens): copies
+//             x_t (16-byte vectors) to each of its FFN slots of Xp, the B
+//             operand of the gate/up GEMM.
 // The histogram itself is integer and comes from the router, so it is exact.
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -108,13 +109,16 @@ __global__ void assign_slots_kernel(const int* __restrict__ idx, int64_t pairs, 
 __global__ void permute_kernel(const uint4* __restrict__ x, const int* __restrict__ slot,
                                int d8, int K, uint4* __restrict__ Xp) {
   const int64_t t = blockIdx.x;
+  const int part = blockIdx.y, parts = gridDim.y;   // this CTA's share of the row
+  const int c_begin = static_cast<int>(static_cast<int64_t>(d8) * part / parts);
+  const int c_end = static_cast<int>(static_cast<int64_t>(d8) * (part + 1) / parts);
   __shared__ int sl[MOE_MAX_K_INTERNAL];
   griddep_wait();
   griddep_launch_dependents();
   if (threadIdx.x < K) sl[threadIdx.x] = slot[t * K + threadIdx.x];
   __syncthreads();
   const uint4* src = x + t * d8;
-  for (int c = threadIdx.x; c < d8; c += blockDim.x) {
+  for (int c = c_begin + threadIdx.x; c < c_end; c += blockDim.x) {
     const uint4 v = src[c];
     for (int k = 0; k < K; ++k) {
       const int s = sl[k];
@@ -155,8 +159,14 @@ cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, i
                            __nv_bfloat16* Xp, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
   const int d8 = d / 8;
-  const int threads = d8 < 256 ? ((d8 + 31) / 32) * 32 : 256;
-  return launch_pdl(permute_kernel, dim3(static_cast<unsigned>(T)), dim3(threads), 0, stream,
+  // few tokens: split each row over up to 8 CTAs (at least 128 vectors each)
+  const int64_t want = (2LL * device_sms() + T - 1) / T;
+  int parts = static_cast<int>(want < 8 ? want : 8);
+  while (parts > 1 && d8 / parts < 128) --parts;
+  if (parts < 1) parts = 1;
+  const int per = (d8 + parts - 1) / parts;
+  const int threads = per < 256 ? ((per + 31) / 32) * 32 : 256;
+  return launch_pdl(permute_kernel, dim3(static_cast<unsigned>(T), parts), dim3(threads), 0, stream,
                     reinterpret_cast<const uint4*>(x), slot, d8, K, reinterpret_cast<uint4*>(Xp));
 }
 

@@ -49,6 +49,7 @@ namespace moezc {
 namespace {
 
 constexpr long long DRAIN_NS = 2000000000LL;  // bound of the drain waits at exit
+constexpr long long PACE_NS = 50000LL;        // longest wait for the partner CTA's tile start
 
 struct Tile {
   int k0, k1;   // k-step range of this tile
@@ -60,6 +61,7 @@ struct Tile {
   int nmma;     // MMA N: ntok rounded up to 16
   int brow0;    // first B row
   int count;    // tokens in the group
+  int ntt;      // token tiles of the group
   bool has_a1;  // second A block present
   int a0_row, a1_row;
 };
@@ -75,6 +77,18 @@ __device__ __forceinline__ int total_tiles(const GemmParams& p) {
     return ((p.T + tt - 1) / tt) * p.mblocks * (p.ksplit > 1 ? p.ksplit : 1);
   }
   return __ldg(p.grp_ttp + p.G) * p.mblocks;
+}
+
+// Group (expert) of expert-GEMM tile t: the largest g with ttp[g] <= t / mblocks
+// (a group's tiles start at ttp[g] * mblocks).
+__device__ __forceinline__ int group_of_tile(const GemmParams& p, int t) {
+  const int tt = t / p.mblocks;
+  int lo = 0, hi = p.G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.grp_ttp + mid) <= tt) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
 template <int MODE>
@@ -95,18 +109,29 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   int j;
   if (MODE == MODE_ROUTER) {
     tl.g = 0;
+    tl.ntt = 0;
     j = tt;
     tl.count = p.T;
     tl.brow0 = 0;
   } else {
-    // largest g with ttp[g] <= tt
-    int lo = 0, hi = p.G - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (__ldg(p.grp_ttp + mid) <= tt) lo = mid; else hi = mid - 1;
-    }
+    const int lo = group_of_tile(p, t);
     tl.g = lo;
-    j = tt - __ldg(p.grp_ttp + lo);
+    // Order inside the group: weight block fastest, so that the tiles of a
+    // round of the persistent grid share a few weight blocks and token
+    // tiles; but an expert with two token tiles goes weight block by weight
+    // block with its two token tiles adjacent (tiles 2i and 2i + 1 read the
+    // same weight block).
+    const int ttp0 = __ldg(p.grp_ttp + lo);
+    const int ntt = __ldg(p.grp_ttp + lo + 1) - ttp0;
+    tl.ntt = ntt;
+    const int u = t - ttp0 * p.mblocks;
+    if (ntt == 2) {
+      tl.m = u >> 1;
+      j = u & 1;
+    } else {
+      j = u / p.mblocks;
+      tl.m = u - j * p.mblocks;
+    }
     tl.count = __ldg(p.grp_count + lo);
     tl.brow0 = __ldg(p.grp_off + lo);
   }
@@ -244,6 +269,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
+  __shared__ uint32_t peer_tile_sh;   // p.pair_tiles: paced tiles the partner CTA has begun
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -261,6 +287,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     }
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
+    peer_tile_sh = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA0);
     tma_prefetch_desc(&tmA1);
@@ -274,6 +301,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   }
   tc_fence_before();
   __syncthreads();
+  if (p.pair_tiles) cluster_sync_all();   // the partner's pacing word exists before any store
   tc_fence_after();
   // the prologue above overlaps the previous kernel; from here on its
   // results (routing, offsets, activations) are read
@@ -295,8 +323,29 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     uint32_t armed = 0;          // stages armed at least once
     uint32_t last_par = 0;       // parity each stage was last armed with
     const uint64_t pol_stream = l2_policy_evict_first();
+    // p.pair_tiles: the grid runs as 2-CTA clusters (the two SMs of a TPC),
+    // CTA rank r of a cluster taking tiles t with t % 2 == r.  When tiles t
+    // and t ^ 1 are the two token tiles of one weight block of an expert with
+    // two token tiles (the common case when experts get a few hundred tokens
+    // each), the CTAs start them together, so the weight bytes one of them
+    // loads from DRAM are an L2 hit for the other: each stores into the
+    // partner's shared memory how many such tiles it has begun and waits
+    // until the partner has begun the same one -- for at most PACE_NS, after
+    // which it goes on alone (pacing is only a hint: it never holds up or
+    // fails the GEMM).  Experts with many token tiles share weight blocks
+    // across each round of the grid anyway and are not paced.
+    const uint32_t peer_word =
+        p.pair_tiles ? mapa_shared(smem_u32(&peer_tile_sh), cluster_ctarank() ^ 1u) : 0u;
+    uint32_t begun = 0;
     for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x) {
       const Tile tl = decode_tile<MODE>(p, t);
+      // both CTAs evaluate the same predicate on the pair (t, t ^ 1)
+      if (MODE != MODE_ROUTER && p.pair_tiles && tl.ntt == 2 && (t ^ 1) < ntiles &&
+          group_of_tile(p, t ^ 1) == tl.g) {
+        ++begun;
+        st_cluster_u32(peer_word, begun);
+        pace_until_shared(&peer_tile_sh, begun, PACE_NS);
+      }
       const int nbox = (tl.nmma + GEMM_B_BOX_ROWS - 1) / GEMM_B_BOX_ROWS;
       // a full token tile (256 tokens; the router's tile size) in one copy
       // of the b_full map, whose box has exactly that many rows
@@ -474,10 +523,29 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
 
   tc_fence_before();
   __syncthreads();
+  // no CTA leaves while its partner may still store into its shared memory
+  if (p.pair_tiles) cluster_sync_all();
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+template <int MODE>
+cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                        const CUtensorMap& b_full, GemmParams p, int grid, cudaStream_t stream) {
+  const cudaError_t e = smem_limit<gemm_kernel<MODE>>(GEMM_SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  // pacing runs the grid as 2-CTA clusters: an even grid of at least two
+  if (p.pair_tiles) {
+    if (grid >= 2) {
+      return launch_pdl_pairs(gemm_kernel<MODE>, dim3(grid & ~1), dim3(GEMM_THREADS),
+                              GEMM_SMEM_BYTES, stream, a0, a1, b, b_full, p);
+    }
+    p.pair_tiles = 0;
+  }
+  return launch_pdl(gemm_kernel<MODE>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES, stream,
+                    a0, a1, b, b_full, p);
 }
 
 }  // namespace
@@ -488,23 +556,17 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
   if (grid <= 0) return cudaSuccess;
   cudaError_t e = cudaSuccess;
   switch (mode) {
-    case MODE_ROUTER:
-      e = smem_limit<gemm_kernel<MODE_ROUTER>>(GEMM_SMEM_BYTES);
-      if (e != cudaSuccess) return e;
-      e = launch_pdl(gemm_kernel<MODE_ROUTER>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES,
-                     stream, a0, a1, b, b_full, p);
+    case MODE_ROUTER: {
+      GemmParams q = p;
+      q.pair_tiles = 0;
+      e = launch_mode<MODE_ROUTER>(a0, a1, b, b_full, q, grid, stream);
       break;
+    }
     case MODE_GATEUP:
-      e = smem_limit<gemm_kernel<MODE_GATEUP>>(GEMM_SMEM_BYTES);
-      if (e != cudaSuccess) return e;
-      e = launch_pdl(gemm_kernel<MODE_GATEUP>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES,
-                     stream, a0, a1, b, b_full, p);
+      e = launch_mode<MODE_GATEUP>(a0, a1, b, b_full, p, grid, stream);
       break;
     case MODE_DOWN:
-      e = smem_limit<gemm_kernel<MODE_DOWN>>(GEMM_SMEM_BYTES);
-      if (e != cudaSuccess) return e;
-      e = launch_pdl(gemm_kernel<MODE_DOWN>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES,
-                     stream, a0, a1, b, b_full, p);
+      e = launch_mode<MODE_DOWN>(a0, a1, b, b_full, p, grid, stream);
       break;
   }
   if (e != cudaSuccess) return e;

@@ -64,6 +64,28 @@ inline int blocks_per_sm(int threads, size_t smem) {
   return n;
 }
 
+// Launch with programmatic dependent launch (as launch_pdl) as clusters of
+// two CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_pairs(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Multiprocessors of the current device (cached).
 inline int device_sms() {
   static int cached[64] = {0};
@@ -117,6 +139,7 @@ struct GemmParams {
                           // L2 evict-first policy (decode: every weight byte is read once)
   int b_box_full;         // 1: a full token tile's B rows come in one GEMM_BN-row copy
   int tok_tile;           // MODE_ROUTER: tokens per tile (multiple of 16, <= GEMM_BN; 0: GEMM_BN)
+  int pair_tiles;         // gate/up, down: 2-CTA clusters pace tiles t, t ^ 1 (even grid)
   int mblocks;            // tiles along the weight rows of one group
   int a_rows;             // weight rows per group: E (router), I (gate/up), d (down)
   void* out;              // fp32 logits [T, E] | bf16 H [rows, I] | bf16 Y [rows, d]
@@ -126,7 +149,8 @@ struct GemmParams {
 };
 
 // b: B map with GEMM_B_BOX_ROWS-row boxes; b_full: with GEMM_BN-row boxes,
-// used for full token tiles when p.b_box_full is set.
+// used for full token tiles when p.b_box_full is set.  With p.pair_tiles the
+// grid (rounded down to even) runs as 2-CTA clusters.
 cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap& a1,
                         const CUtensorMap& b, const CUtensorMap& b_full, const GemmParams& p,
                         int grid, cudaStream_t stream);

@@ -57,6 +57,15 @@ struct Ctx {
   int64_t T = 0;
   int d = 0, N = 0, Z = 0, K = 0, I = 0;
   int64_t rows_cap = 0;
+  // Expert-load shape seen by earlier forwards, to choose the expert GEMMs'
+  // launch without a host sync: after each prefill-sized forward its FFN
+  // histogram is copied to pinned host memory behind an event; a later
+  // forward reads it once the event has completed.
+  int* hist_host = nullptr;          // pinned [MOE_ZC_MAX_E]
+  cudaEvent_t hist_ev = nullptr;
+  bool hist_pending = false;
+  int hist_N = 0;
+  bool pair_hint = false;            // most FFN pairs sit in experts with two token tiles
 };
 
 Ctx g_ctx[kMaxDevices];
@@ -141,6 +150,12 @@ int get_ctx(Ctx** out) {
       return MOE_ZC_ERR_CUDA;
     if (cudaEventCreateWithFlags(&c.done, cudaEventDisableTiming) != cudaSuccess)
       return MOE_ZC_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&c.hist_ev, cudaEventDisableTiming) != cudaSuccess)
+      return MOE_ZC_ERR_CUDA;
+    if (cudaMallocHost(&c.hist_host, sizeof(int) * MOE_ZC_MAX_E) != cudaSuccess) {
+      cudaGetLastError();
+      c.hist_host = nullptr;   // the launch choice then keeps its default
+    }
     c.init = true;
   }
   *out = &c;
@@ -321,6 +336,30 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   }
   rec.mark(0);
   CK(cudaMemsetAsync(cnt, 0, sizeof(int) * E, st));
+  // Prefill-sized batches whose experts mostly get two token tiles (a few
+  // hundred tokens each, as under balanced load) run the expert GEMMs as
+  // 2-CTA clusters that pace those tiles; batches concentrated on a few
+  // experts do better without (measured: +10% on balanced gate/up, -3% on
+  // concentrated).  The choice follows the histogram of an earlier forward.
+  if (!captured && c.hist_pending) {
+    const cudaError_t q = cudaEventQuery(c.hist_ev);
+    if (q == cudaErrorNotReady) {
+      cudaGetLastError();   // not an error: the copy is still on its way
+    } else {
+      CK(q);
+      if (c.hist_N == N) {
+        long long two = 0, all = 0;
+        for (int e = 0; e < N; ++e) {
+          const int n = c.hist_host[e];
+          all += n;
+          if (n > GEMM_BN && n <= 2 * GEMM_BN) two += n;
+        }
+        c.pair_hint = all > 0 && 2 * two >= all;
+      }
+      c.hist_pending = false;
+    }
+  }
+  const bool pace_tiles = N > 0 && T >= 1024 && c.pair_hint;
   if (T > 0) {
     // 1  router GEMM
     CUtensorMap mWr, mX;
@@ -435,6 +474,9 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       // decode-sized batches stream every weight byte once
       pg.l2_stream = T < 1024 ? 1 : 0;
       pg.b_box_full = full_ok ? 1 : 0;
+      // prefill-sized batches: CTA pairs pace the two token tiles of a weight
+      // block so that its second read is an L2 hit
+      pg.pair_tiles = pace_tiles ? 1 : 0;
       const int64_t g_ub = tiles_ub * pg.mblocks;
       CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg, static_cast<int>(g_ub < c.sms ? g_ub : c.sms),
                      st));
@@ -469,6 +511,12 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   }
   rec.mark(8);
   if (rec.ev) ++g_prof.n;
+  if (!captured && !c.hist_pending && c.hist_host && N > 0 && T >= 1024) {
+    CK(cudaMemcpyAsync(c.hist_host, cnt, sizeof(int) * N, cudaMemcpyDeviceToHost, st));
+    CK(cudaEventRecord(c.hist_ev, st));
+    c.hist_pending = true;
+    c.hist_N = N;
+  }
   if (!captured) CK(cudaEventRecord(c.done, st));
   c.done_valid = !captured;
   c.has_result = true;

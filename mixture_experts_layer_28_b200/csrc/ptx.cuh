@@ -237,6 +237,29 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
                : "memory");
 }
 
+// A 32-bit store into a cluster-window shared-memory address (may be a
+// peer CTA's), and a poll of this CTA's word that such stores update: wait
+// until it is at least `target` for at most limit_ns, then go on either way
+// (for pacing only -- nothing may depend on the wait having succeeded).
+__device__ __forceinline__ void st_cluster_u32(uint32_t cl_addr, uint32_t v) {
+  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(cl_addr), "r"(v)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t ld_cluster_u32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p))
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void pace_until_shared(const void* p, uint32_t target,
+                                                  long long limit_ns) {
+  if (ld_cluster_u32(p) >= target) return;
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_cluster_u32(p) < target) {
+    if (static_cast<long long>(globaltimer_ns() - t0) > limit_ns) return;
+  }
+}
+
 // Named barrier over `nthreads` threads (multiple of 32) of this CTA.
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -144,6 +144,22 @@ def test_router_token_tiles_sized_to_waves():
     _full_check(Case(w))
 
 
+def test_paired_tile_launch_matches_plain():
+    """Balanced load (experts of ~270 tokens, two token tiles each): once a
+    forward has seen such a histogram, the next ones run the expert GEMMs as
+    paced 2-CTA clusters.  Every forward gives the same bits, and the oracle
+    agrees."""
+    w = wl.get("prefill_balanced", T=2048, N=64, Z=32, d=1024, I=256)
+    case = Case(w)
+    o1, i1, g1, c1 = _gpu_result(case)
+    for _ in range(2):
+        o2, i2, g2, c2 = _gpu_result(case)
+        assert np.array_equal(o1, o2) and np.array_equal(i1, i2) and np.array_equal(c1, c2)
+    ffn = c2[: w.N]
+    assert 2 * ffn[(ffn > 256) & (ffn <= 512)].sum() >= ffn.sum()   # the balanced shape
+    _full_check(case)
+
+
 def test_empty_batch_is_noop():
     w = wl.get("tiny")
     case = Case(wl.get("tiny", T=1))
