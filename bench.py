@@ -61,8 +61,9 @@ KERNELS_PER_FORWARD = 8   # router_gemm, route, scan, assign, permute, gateup, d
 # pass; the full-size GEMM traffic summary under profiles/), per workload.
 # Clear an entry when that kernel changes.
 NCU_TRAFFIC_BYTES = {
-    "prefill": 8_755_961_088 + 561_242_624,    # gate/up GEMM
-    "decode": 1_520_849_408 + 4_829_696,       # gate/up GEMM
+    "prefill": 9_217_720_576 + 561_846_016,    # gate/up GEMM
+    "decode": 1_520_860_672 + 4_152_064,       # gate/up GEMM
+    "prefill_balanced": 30_004_439_040 + 564_574_976,   # gate/up GEMM, paired tiles
 }
 
 
