@@ -66,6 +66,7 @@ struct Ctx {
   bool hist_pending = false;
   int hist_N = 0;
   bool pair_hint = false;            // most FFN pairs sit in experts with two token tiles
+  bool spread_hint = false;          // at least half of the N FFN experts were hit
 };
 
 Ctx g_ctx[kMaxDevices];
@@ -354,7 +355,10 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
           all += n;
           if (n > GEMM_BN && n <= 2 * GEMM_BN) two += n;
         }
+        int hit = 0;
+        for (int e = 0; e < N; ++e) hit += c.hist_host[e] > 0;
         c.pair_hint = all > 0 && 2 * two >= all;
+        c.spread_hint = 2 * hit >= N;
       }
       c.hist_pending = false;
     }
@@ -556,17 +560,24 @@ int forward_host_impl(const void* x_host, const void* W_r, const float* b, const
   int s = check_args(reinterpret_cast<const void*>(16), W_r, b, W_gate, W_up, W_down, T, d, N,
                      Z, K, I, off, reinterpret_cast<void*>(16));
   if (s != MOE_ZC_OK) return s;
-  if (chunk <= 0) {
-    // four chunks: measured best at the prefill workload (2048: 13.0 ms,
-    // 4096: 12.1 ms, 8192: 12.8 ms per step, B200)
-    chunk = (T + 3) / 4;
-    chunk = ((chunk + 255) / 256) * 256;
-    if (chunk < 1024) chunk = 1024;
-  }
-  if (chunk > T) chunk = T;
   Ctx* cp = nullptr;
   if ((s = get_ctx(&cp)) != MOE_ZC_OK) return s;
   Ctx& c = *cp;
+  if (chunk <= 0) {
+    // Four chunks: measured best at the prefill workload (2048: 13.0 ms,
+    // 4096: 12.1 ms, 8192: 12.8 ms per step, B200).  But when earlier
+    // forwards spread their tokens over most FFN experts, every chunk would
+    // stream nearly all expert weights again: one chunk then (balanced
+    // prefill: 18.3 ms per step against 27 ms in four).
+    if (c.spread_hint && c.hist_N == N) {
+      chunk = T;
+    } else {
+      chunk = (T + 3) / 4;
+      chunk = ((chunk + 255) / 256) * 256;
+      if (chunk < 1024) chunk = 1024;
+    }
+  }
+  if (chunk > T) chunk = T;
   const int E = N + Z;
   if ((s = host_streams(c)) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.cnt_total, sizeof(int) * E)) != MOE_ZC_OK) return s;
