@@ -40,7 +40,6 @@ __global__ void combine_kernel(const uint4* __restrict__ x, const uint4* __restr
   __shared__ float gt[MOE_MAX_K_INTERNAL];
   __shared__ int nffn;
   griddep_wait();
-  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     int n = 0;
     for (int k = 0; k < K; ++k) {
@@ -67,6 +66,8 @@ __global__ void combine_kernel(const uint4* __restrict__ x, const uint4* __restr
     }
     out[t * d8 + c] = o;
   }
+  // many waves of CTAs: let dependents launch only as the last ones finish
+  griddep_launch_dependents();
 }
 
 }  // namespace

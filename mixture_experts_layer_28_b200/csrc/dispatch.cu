@@ -86,7 +86,6 @@ __global__ void assign_slots_kernel(const int* __restrict__ idx, int64_t pairs, 
                                     const int* __restrict__ grp_off, int* __restrict__ fill,
                                     int* __restrict__ slot) {
   griddep_wait();
-  griddep_launch_dependents();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
   const bool valid = i < pairs;
@@ -104,6 +103,7 @@ __global__ void assign_slots_kernel(const int* __restrict__ idx, int64_t pairs, 
     s = grp_off[e] + base + rank;
   }
   if (valid) slot[i] = s;
+  griddep_launch_dependents();   // as the last CTAs finish (several waves)
 }
 
 __global__ void permute_kernel(const uint4* __restrict__ x, const int* __restrict__ slot,
@@ -114,7 +114,6 @@ __global__ void permute_kernel(const uint4* __restrict__ x, const int* __restric
   const int c_end = static_cast<int>(static_cast<int64_t>(d8) * (part + 1) / parts);
   __shared__ int sl[MOE_MAX_K_INTERNAL];
   griddep_wait();
-  griddep_launch_dependents();
   if (threadIdx.x < K) sl[threadIdx.x] = slot[t * K + threadIdx.x];
   __syncthreads();
   const uint4* src = x + t * d8;
@@ -125,6 +124,10 @@ __global__ void permute_kernel(const uint4* __restrict__ x, const int* __restric
       if (s >= 0) Xp[static_cast<int64_t>(s) * d8 + c] = v;
     }
   }
+  // Many waves of CTAs: the dependent GEMM (one 216 KB CTA per SM) may
+  // launch only as the last CTAs finish, or its early CTAs would take SMs
+  // from this kernel's later waves.
+  griddep_launch_dependents();
 }
 
 __global__ void add_counts_kernel(const int* __restrict__ cnt, int E, int* __restrict__ total) {
