@@ -54,7 +54,7 @@ from mixture_experts_layer_28_b200 import workloads as wl  # noqa: E402
 METRIC = "MoE-layer tokens/s; executed-FFN TFLOPS as % of B200 bf16 peak (HBM % at decode)"
 UNIT = "tokens/s"
 L2_BYTES = 126 * 2 ** 20
-KERNELS_PER_FORWARD = 8   # router_gemm, route, scan, assign, permute, gateup, down, combine
+KERNELS_PER_FORWARD = 7   # router_gemm, route, assign, permute, gateup, down, combine
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel
 # from an ncu capture of the current kernel build at the full workload (one

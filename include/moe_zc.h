@@ -198,9 +198,9 @@ const char* moe_zc_status_string(int status);
  * recording on the current device -- at most 256 forwards are kept --
  * moe_zc_profile(0) stops.  moe_zc_profile_read waits for the last recorded
  * forward and writes, for each stage i < max_stages, the milliseconds summed
- * over the recorded forwards (stage_ms: host float[max_stages]; 8 stages,
- * named by moe_zc_stage_name: router_gemm, route, scan, assign_slots,
- * permute, gateup_gemm, down_gemm, combine) and their count to *n_forwards.
+ * over the recorded forwards (stage_ms: host float[max_stages]; 7 stages,
+ * named by moe_zc_stage_name: router_gemm, route, assign_slots, permute,
+ * gateup_gemm, down_gemm, combine) and their count to *n_forwards.
  */
 int moe_zc_profile(int32_t enable);
 int moe_zc_profile_read(float* stage_ms, int32_t max_stages, int32_t* n_forwards);

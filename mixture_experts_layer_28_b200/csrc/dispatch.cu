@@ -5,13 +5,16 @@
 // for its speed", section "Zero-computation experts"), so its picks were
 // already folded into zsum by the router and get slot -1 here.
 //
-//   scan      one CTA: per expert, rows = count rounded up to 16 and token
-//             tiles = ceil(count / 256); exclusive prefix sums give each
-//             expert's first row in the permuted buffers (grp_off) and its
-//             first GEMM token tile (grp_ttp); the GEMM grid walks grp_ttp.
-//   assign    one thread per (token, pick): lanes of a warp that picked the
-//             same expert are grouped with __match_any_sync and take their
-//             slots with one atomicAdd per group (warp-aggregated atomics).
+//   assign    first every CTA takes, from the expert-load histogram, each
+//             FFN expert's rows (count rounded up to 16) and token tiles
+//             (ceil(count / 256)); exclusive prefix sums give the expert's
+//             first row in the permuted buffers (grp_off) and its first GEMM
+//             token tile (grp_ttp), which CTA 0 also stores for the GEMMs
+//             (the GEMM grid walks grp_ttp).  Then one thread per (token,
+//             pick): lanes of a warp that picked the same expert are grouped
+//             with __match_any_sync and take their slots with one atomicAdd
+//             per group (warp-aggregated atomics) on per-expert fill
+//             counters that the router GEMM zeroed.
 //   permute   one CTA per token (per part of its row for few tokens): copies
 //             x_t (16-byte vectors) to each of its FFN slots of Xp, the B
 //             operand of the gate/up GEMM.
@@ -22,9 +25,12 @@
 namespace moezc {
 namespace {
 
-constexpr int SCAN_THREADS = 1024;
+constexpr int ASSIGN_THREADS = 256;
 
+// Exclusive prefix sum of v over the CTA (ASSIGN_THREADS threads), with the
+// CTA's total in *total.
 __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total) {
+  constexpr int W = ASSIGN_THREADS / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = v;
 #pragma unroll
@@ -35,57 +41,52 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = (lane < SCAN_THREADS / 32) ? warp_sums[lane] : 0;
+    int w = lane < W ? warp_sums[lane] : 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
+    for (int o = 1; o < W; o <<= 1) {
       const int u = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += u;
     }
-    warp_sums[lane] = w;  // inclusive prefix over warps
+    if (lane < W) warp_sums[lane] = w;   // inclusive prefix over warps
   }
   __syncthreads();
   const int base = warp ? warp_sums[warp - 1] : 0;
-  *total = warp_sums[SCAN_THREADS / 32 - 1];
+  *total = warp_sums[W - 1];
   __syncthreads();
   return base + incl - v;
 }
 
-__global__ void __launch_bounds__(SCAN_THREADS)
-scan_kernel(const int* __restrict__ cnt, int N, int* __restrict__ grp_off,
-            int* __restrict__ grp_ttp, int* __restrict__ fill) {
+__global__ void __launch_bounds__(ASSIGN_THREADS)
+assign_slots_kernel(const int* __restrict__ cnt, const int* __restrict__ idx, int64_t pairs,
+                    int N, int* __restrict__ grp_off, int* __restrict__ grp_ttp,
+                    int* __restrict__ fill, int* __restrict__ slot) {
+  __shared__ int off_s[MOE_MAX_E_INTERNAL];
   __shared__ int warp_sums[32];
-  __shared__ int carry_rows, carry_tiles;
   griddep_wait();
-  griddep_launch_dependents();
-  if (threadIdx.x == 0) { carry_rows = 0; carry_tiles = 0; }
-  __syncthreads();
-  for (int base = 0; base < N; base += SCAN_THREADS) {
+  // experts' first rows (and, in CTA 0, first token tiles) from the histogram
+  int carry_rows = 0, carry_tiles = 0;
+  for (int base = 0; base < N; base += ASSIGN_THREADS) {
     const int g = base + threadIdx.x;
-    const int c = (g < N) ? cnt[g] : 0;
-    const int rows = (c + 15) & ~15;
-    const int tiles = (c + GEMM_BN - 1) / GEMM_BN;
-    int tot_rows, tot_tiles;
-    const int off = block_excl_scan(rows, warp_sums, &tot_rows);
-    const int ttp = block_excl_scan(tiles, warp_sums, &tot_tiles);
-    if (g < N) {
-      grp_off[g] = carry_rows + off;
-      grp_ttp[g] = carry_tiles + ttp;
-      fill[g] = 0;
+    const int c = g < N ? cnt[g] : 0;
+    int tot_rows, tot_tiles = 0;
+    const int off = block_excl_scan((c + 15) & ~15, warp_sums, &tot_rows);
+    if (g < N) off_s[g] = carry_rows + off;
+    if (blockIdx.x == 0) {
+      const int ttp = block_excl_scan((c + GEMM_BN - 1) / GEMM_BN, warp_sums, &tot_tiles);
+      if (g < N) {
+        grp_off[g] = carry_rows + off;
+        grp_ttp[g] = carry_tiles + ttp;
+      }
     }
-    __syncthreads();
-    if (threadIdx.x == 0) { carry_rows += tot_rows; carry_tiles += tot_tiles; }
-    __syncthreads();
+    carry_rows += tot_rows;
+    carry_tiles += tot_tiles;
   }
-  if (threadIdx.x == 0) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
     grp_off[N] = carry_rows;
     grp_ttp[N] = carry_tiles;
   }
-}
+  __syncthreads();
 
-__global__ void assign_slots_kernel(const int* __restrict__ idx, int64_t pairs, int N,
-                                    const int* __restrict__ grp_off, int* __restrict__ fill,
-                                    int* __restrict__ slot) {
-  griddep_wait();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
   const bool valid = i < pairs;
@@ -100,7 +101,7 @@ __global__ void assign_slots_kernel(const int* __restrict__ idx, int64_t pairs, 
     int base = 0;
     if (lane == leader) base = atomicAdd(&fill[e], __popc(peers));
     base = __shfl_sync(peers, base, leader);
-    s = grp_off[e] + base + rank;
+    s = off_s[e] + base + rank;
   }
   if (valid) slot[i] = s;
   griddep_launch_dependents();   // as the last CTAs finish (several waves)
@@ -143,19 +144,12 @@ cudaError_t launch_add_counts(const int* cnt, int E, int* total, cudaStream_t st
   return launch_pdl(add_counts_kernel, dim3((E + 255) / 256), dim3(256), 0, stream, cnt, E, total);
 }
 
-cudaError_t launch_scan(const int* cnt, int N, int* grp_off, int* grp_ttp, int* fill,
-                        cudaStream_t stream) {
-  return launch_pdl(scan_kernel, dim3(1), dim3(SCAN_THREADS), 0, stream, cnt, N, grp_off, grp_ttp,
-                    fill);
-}
-
-cudaError_t launch_assign_slots(const int* idx, int64_t pairs, int N, const int* grp_off,
-                                int* fill, int* slot, cudaStream_t stream) {
-  if (pairs <= 0) return cudaSuccess;
-  const int threads = 256;
-  const int64_t blocks = (pairs + threads - 1) / threads;
-  return launch_pdl(assign_slots_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0,
-                    stream, idx, pairs, N, grp_off, fill, slot);
+cudaError_t launch_assign_slots(const int* cnt, const int* idx, int64_t pairs, int N,
+                                int* grp_off, int* grp_ttp, int* fill, int* slot,
+                                cudaStream_t stream) {
+  const int64_t blocks = pairs > 0 ? (pairs + ASSIGN_THREADS - 1) / ASSIGN_THREADS : 1;
+  return launch_pdl(assign_slots_kernel, dim3(static_cast<unsigned>(blocks)), dim3(ASSIGN_THREADS),
+                    0, stream, cnt, idx, pairs, N, grp_off, grp_ttp, fill, slot);
 }
 
 cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, int d, int K,

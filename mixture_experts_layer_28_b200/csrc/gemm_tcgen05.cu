@@ -307,6 +307,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   // results (routing, offsets, activations) are read
   griddep_wait();
   griddep_launch_dependents();
+  if (MODE == MODE_ROUTER && blockIdx.x == 0) {
+    // this forward's expert-load histogram and slot counters start at zero
+    // (the previous forward's readers are done: griddep_wait)
+    for (int i = threadIdx.x; i < p.nzero0; i += blockDim.x) p.zero0[i] = 0;
+    for (int i = threadIdx.x; i < p.nzero1; i += blockDim.x) p.zero1[i] = 0;
+  }
   const uint32_t tmem = tmem_base_sh;
   const int ntiles = total_tiles<MODE>(p);
   // gate/up tiles always hold two blocks; router and down tiles hold one

@@ -9,6 +9,7 @@
 namespace moezc {
 
 constexpr int MOE_MAX_K_INTERNAL = 32;   // most picks per token
+constexpr int MOE_MAX_E_INTERNAL = 1024; // most experts (FFN + zero)
 
 // Launch with programmatic stream serialisation (the kernel overlaps its
 // predecessor's tail and orders itself with griddepcontrol.wait).
@@ -140,6 +141,9 @@ struct GemmParams {
   int b_box_full;         // 1: a full token tile's B rows come in one GEMM_BN-row copy
   int tok_tile;           // MODE_ROUTER: tokens per tile (multiple of 16, <= GEMM_BN; 0: GEMM_BN)
   int pair_tiles;         // gate/up, down: 2-CTA clusters pace tiles t, t ^ 1 (even grid)
+  int* zero0;             // MODE_ROUTER: CTA 0 clears zero0[0, nzero0) and zero1[0, nzero1)
+  int* zero1;             //   once the previous kernel is done (the next forward's counters)
+  int nzero0, nzero1;
   int mblocks;            // tiles along the weight rows of one group
   int a_rows;             // weight rows per group: E (router), I (gate/up), d (down)
   void* out;              // fp32 logits [T, E] | bf16 H [rows, I] | bf16 Y [rows, d]
@@ -180,10 +184,12 @@ cudaError_t launch_route(const float* logits, const float* b, const float* offse
                          cudaStream_t stream, int splits = 1);
 
 // ------------------------------------------------------------------ dispatch
-cudaError_t launch_scan(const int* cnt, int N, int* grp_off, int* grp_ttp, int* fill,
-                        cudaStream_t stream);
-cudaError_t launch_assign_slots(const int* idx, int64_t pairs, int N, const int* grp_off,
-                                int* fill, int* slot, cudaStream_t stream);
+// Slot assignment with the experts' row and tile offsets (grp_off, grp_ttp
+// [N + 1], written by CTA 0) computed from the histogram cnt; fill [N] must
+// be zero on entry (the router GEMM clears it).
+cudaError_t launch_assign_slots(const int* cnt, const int* idx, int64_t pairs, int N,
+                                int* grp_off, int* grp_ttp, int* fill, int* slot,
+                                cudaStream_t stream);
 // total[j] += cnt[j] for j < E (histogram summed over the chunks of a forward)
 cudaError_t launch_add_counts(const int* cnt, int E, int* total, cudaStream_t stream);
 cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, int d, int K,

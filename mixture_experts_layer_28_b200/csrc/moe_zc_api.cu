@@ -73,11 +73,11 @@ Ctx g_ctx[kMaxDevices];
 std::mutex g_mu;
 
 // Per-stage CUDA-event timing of forwards (moe_zc_profile / moe_zc_profile_read).
-constexpr int kStages = 8;
+constexpr int kStages = 7;
 constexpr int kRing = 256;
-const char* const kStageNames[kStages] = {"router_gemm", "route",        "scan",
-                                          "assign_slots", "permute",     "gateup_gemm",
-                                          "down_gemm",    "combine"};
+const char* const kStageNames[kStages] = {"router_gemm", "route",       "assign_slots",
+                                          "permute",     "gateup_gemm", "down_gemm",
+                                          "combine"};
 struct Prof {
   bool on = false;
   int device = -1;
@@ -336,7 +336,8 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     rec.st = st;
   }
   rec.mark(0);
-  CK(cudaMemsetAsync(cnt, 0, sizeof(int) * E, st));
+  // (a batch with tokens clears its histogram in the router GEMM)
+  if (T == 0) CK(cudaMemsetAsync(cnt, 0, sizeof(int) * E, st));
   // Prefill-sized batches whose experts mostly get two token tiles (a few
   // hundred tokens each, as under balanced load) run the expert GEMMs as
   // 2-CTA clusters that pace those tiles; batches concentrated on a few
@@ -394,6 +395,10 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     pr.split_stride = T * E;
     const int64_t rgrid = rp.tiles * splits;
     pr.b_box_full = full_ok ? 1 : 0;
+    pr.zero0 = cnt;
+    pr.nzero0 = E;
+    pr.zero1 = fill;
+    pr.nzero1 = N;
     CK(launch_gemm(MODE_ROUTER, mWr, mWr, mX, mXf, pr,
                    static_cast<int>(rgrid < c.sms ? rgrid : c.sms), st));
     rec.mark(1);
@@ -402,17 +407,15 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
                     cnt, st, splits));
     rec.mark(2);
     if (N > 0) {
-      // 3-5  dispatch
-      CK(launch_scan(cnt, N, grp_off, grp_ttp, fill, st));
+      // 3-4  dispatch
+      CK(launch_assign_slots(cnt, idx, T * K, N, grp_off, grp_ttp, fill, slot, st));
       rec.mark(3);
-      CK(launch_assign_slots(idx, T * K, N, grp_off, fill, slot, st));
-      rec.mark(4);
       CK(launch_permute(static_cast<const __nv_bfloat16*>(x), slot, T, d, K,
                         static_cast<__nv_bfloat16*>(c.Xp.p), st));
-      rec.mark(5);
+      rec.mark(4);
       const int64_t tiles_ub = (T * K + GEMM_BN - 1) / GEMM_BN + N;
       if (use_pair_gemm(T, K, d)) {
-        // 6-7 on CTA pairs
+        // 5-6 on CTA pairs
         CUtensorMap mWg, mWu, mXp, mWd, mH;
         if (!make_map(&mWg, W_gate, static_cast<uint64_t>(N) * I, d, 64) ||
             !make_map(&mWu, W_up, static_cast<uint64_t>(N) * I, d, 64) ||
@@ -437,7 +440,7 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
         const int64_t g_ub = tiles_ub * pg.mblocks;
         CK(launch_gemm_pair(MODE_GATEUP, mWg, mWu, mXp, pg,
                             static_cast<int>(g_ub < pairs_max ? g_ub : pairs_max), st));
-        rec.mark(6);
+        rec.mark(5);
         GemmParams pd = pg;
         pd.ksteps = I / GEMM_BK;
         pd.mblocks = d / (2 * GEMM_BM);
@@ -448,9 +451,9 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
         const int64_t d_ub = tiles_ub * pd.mblocks;
         CK(launch_gemm_pair(MODE_DOWN, mWd, mWd, mH, pd,
                             static_cast<int>(d_ub < pairs_max ? d_ub : pairs_max), st));
-        rec.mark(7);
+        rec.mark(6);
       } else {
-      // 6  gate/up GEMM
+      // 5  gate/up GEMM
       CUtensorMap mWg, mWu, mXp;
       if (!make_map(&mWg, W_gate, static_cast<uint64_t>(N) * I, d, GEMM_BM) ||
           !make_map(&mWu, W_up, static_cast<uint64_t>(N) * I, d, GEMM_BM) ||
@@ -484,8 +487,8 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       const int64_t g_ub = tiles_ub * pg.mblocks;
       CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg, static_cast<int>(g_ub < c.sms ? g_ub : c.sms),
                      st));
-      rec.mark(6);
-      // 7  down GEMM
+      rec.mark(5);
+      // 6  down GEMM
       CUtensorMap mWd, mH;
       if (!make_map(&mWd, W_down, static_cast<uint64_t>(N) * d, I, GEMM_BM) ||
           !make_map(&mH, c.H.p, c.rows_cap, I, GEMM_B_BOX_ROWS))
@@ -499,21 +502,20 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       const int64_t d_ub = tiles_ub * pd.mblocks;
       CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd, static_cast<int>(d_ub < c.sms ? d_ub : c.sms),
                      st));
-      rec.mark(7);
+      rec.mark(6);
       }
     } else {
-      rec.mark(3);
-      CK(launch_assign_slots(idx, T * K, N, grp_off, fill, slot, st));
-      for (int i = 4; i <= 7; ++i) rec.mark(i);
+      CK(launch_assign_slots(cnt, idx, T * K, N, grp_off, grp_ttp, fill, slot, st));
+      for (int i = 3; i <= 6; ++i) rec.mark(i);
     }
-    // 8  combine
+    // 7  combine
     CK(launch_combine(static_cast<const __nv_bfloat16*>(x),
                       static_cast<const __nv_bfloat16*>(c.Y.p), slot, gate, zsum, T, d, K,
                       static_cast<__nv_bfloat16*>(out), st));
   } else {
-    for (int i = 1; i <= 7; ++i) rec.mark(i);
+    for (int i = 1; i <= 6; ++i) rec.mark(i);
   }
-  rec.mark(8);
+  rec.mark(7);
   if (rec.ev) ++g_prof.n;
   if (!captured && !c.hist_pending && c.hist_host && N > 0 && T >= 1024) {
     CK(cudaMemcpyAsync(c.hist_host, cnt, sizeof(int) * N, cudaMemcpyDeviceToHost, st));

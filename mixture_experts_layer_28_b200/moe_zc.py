@@ -229,7 +229,7 @@ def route_noalloc(x: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor, N: int, Z
     _check(st, "moe_zc_route_noalloc")
 
 
-STAGES = 8
+STAGES = 7
 
 
 def profile(enable: bool) -> None:
