@@ -6,13 +6,14 @@
 // "Zero-computation experts") is, all on the caller's stream:
 //
 //   1  router GEMM        logits = x W_r^T              tcgen05, fp32 out
+//                         (and clears this forward's histogram and counters)
 //   2  route              softmax, + b, top-K, zsum, histogram
-//   3  scan               per-expert row offsets and GEMM token tiles
-//   4  assign slots       warp-aggregated atomics, FFN picks only
-//   5  permute            x rows -> Xp (grouped by expert)
-//   6  gate/up GEMM       H = SiLU(Xp W_gate^T) * (Xp W_up^T)
-//   7  down GEMM          Y = H W_down^T
-//   8  combine            out = zsum x + sum gate * Y
+//   3  assign slots       per-expert row offsets and GEMM token tiles from
+//                         the histogram; warp-aggregated atomics, FFN picks
+//   4  permute            x rows -> Xp (grouped by expert)
+//   5  gate/up GEMM       H = SiLU(Xp W_gate^T) * (Xp W_up^T)
+//   6  down GEMM          Y = H W_down^T
+//   7  combine            out = zsum x + sum gate * Y
 //
 // No step reads anything back to the host: the GEMM tile lists are built on
 // the device and walked by persistent kernels.
