@@ -160,6 +160,26 @@ def test_paired_tile_launch_matches_plain():
     _full_check(case)
 
 
+@pytest.mark.parametrize("T,d", [(300, 2048), (4096, 2048), (20000, 256)])
+def test_exact_ties_pick_lowest_indices(T, d):
+    """W_r = 0 and b = 0: every expert scores exactly 1/E, so each token picks
+    experts 0..K-1 (ties go to the lower index) with gates 1/E -- through the
+    router's K-sliced (few and many tokens) and unsliced route kernels."""
+    w = wl.get("small", T=T, d=d, I=128)
+    case = Case(w, bias=torch.zeros(w.E))
+    case.W_r = torch.zeros_like(case.W_r)
+    case.dev["W_r"] = case.W_r.cuda()
+    out_g, idx, gate, cnt = _gpu_result(case)
+    assert (idx == np.arange(w.K)[None, :]).all()
+    assert (gate == np.float32(1.0) / np.float32(w.E)).all()
+    want = np.zeros(w.E, dtype=np.int64)
+    want[: w.K] = T
+    assert np.array_equal(cnt, want)
+    r = case.oracle_routing()
+    assert (r.idx == np.arange(w.K)[None, :]).all()
+    check_output(out_g, ref.forward_rows(case.x, r, case.expert))
+
+
 def test_empty_batch_is_noop():
     w = wl.get("tiny")
     case = Case(wl.get("tiny", T=1))
