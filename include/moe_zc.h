@@ -102,10 +102,11 @@ int moe_zc_forward_ex(const void* x, const void* W_r, const float* b,
  * moe_zc_forward_ex on HOST buffers: x_host [T, d] bf16 in, out_host [T, d]
  * bf16 out (page-locked memory for overlap; pageable memory works but its
  * copies do not overlap).  The weights, b and logit_offset stay device
- * memory.  The tokens go in chunks of chunk_tokens (<= 0: T/4 rounded up to
- * 256, at least 1024 -- or all T at once when earlier forwards on the device
- * hit at least half of the FFN experts, as each chunk would then stream
- * nearly all expert weights again): while the kernels of one chunk run on
+ * memory.  The tokens go in chunks of chunk_tokens (<= 0: about T/4,
+ * rounded up to 256 and at least 1024, with the first and the last chunk
+ * half as long -- or all T at once when earlier forwards on the device hit
+ * at least half of the FFN experts, as each chunk would then stream nearly
+ * all expert weights again): while the kernels of one chunk run on
  * `stream`, the next chunk is copied in and the previous one out on two
  * streams of the library's own, so copies overlap compute.  Tokens are independent, so the
  * result equals moe_zc_forward_ex's bit for bit.  Asynchronous: out_host is

@@ -301,6 +301,47 @@ struct StageRec {
   }
 };
 
+// Expert-load hints for later launch choices, without a host sync: a copy
+// of the FFN histogram goes to pinned memory behind an event
+// (queue_load_hints), and a later forward reads it once the event has
+// completed (read_load_hints):
+//   pair_hint    at least half of the FFN pairs sat in experts with two token
+//                tiles (257..512 tokens): pace those tiles on 2-CTA clusters
+//   spread_hint  at least half of the FFN experts were hit: a host-buffer
+//                forward takes the batch in one chunk
+int read_load_hints(Ctx& c, int N) {
+  if (!c.hist_pending) return MOE_ZC_OK;
+  const cudaError_t q = cudaEventQuery(c.hist_ev);
+  if (q == cudaErrorNotReady) {
+    cudaGetLastError();   // not an error: the copy is still on its way
+    return MOE_ZC_OK;
+  }
+  CK(q);
+  if (c.hist_N == N) {
+    long long two = 0, all = 0;
+    int hit = 0;
+    for (int e = 0; e < N; ++e) {
+      const int n = c.hist_host[e];
+      all += n;
+      hit += n > 0;
+      if (n > GEMM_BN && n <= 2 * GEMM_BN) two += n;
+    }
+    c.pair_hint = all > 0 && 2 * two >= all;
+    c.spread_hint = 2 * hit >= N;
+  }
+  c.hist_pending = false;
+  return MOE_ZC_OK;
+}
+
+int queue_load_hints(Ctx& c, const int* cnt, int N, cudaStream_t st) {
+  if (c.hist_pending || !c.hist_host) return MOE_ZC_OK;
+  CK(cudaMemcpyAsync(c.hist_host, cnt, sizeof(int) * N, cudaMemcpyDeviceToHost, st));
+  CK(cudaEventRecord(c.hist_ev, st));
+  c.hist_pending = true;
+  c.hist_N = N;
+  return MOE_ZC_OK;
+}
+
 int forward_impl(const void* x, const void* W_r, const float* b, const void* W_gate,
                  const void* W_up, const void* W_down, int64_t T, int32_t d, int32_t N,
                  int32_t Z, int32_t K, int32_t I, const float* off, void* out, void* stream) {
@@ -344,27 +385,7 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   // 2-CTA clusters that pace those tiles; batches concentrated on a few
   // experts do better without (measured: +10% on balanced gate/up, -3% on
   // concentrated).  The choice follows the histogram of an earlier forward.
-  if (!captured && c.hist_pending) {
-    const cudaError_t q = cudaEventQuery(c.hist_ev);
-    if (q == cudaErrorNotReady) {
-      cudaGetLastError();   // not an error: the copy is still on its way
-    } else {
-      CK(q);
-      if (c.hist_N == N) {
-        long long two = 0, all = 0;
-        for (int e = 0; e < N; ++e) {
-          const int n = c.hist_host[e];
-          all += n;
-          if (n > GEMM_BN && n <= 2 * GEMM_BN) two += n;
-        }
-        int hit = 0;
-        for (int e = 0; e < N; ++e) hit += c.hist_host[e] > 0;
-        c.pair_hint = all > 0 && 2 * two >= all;
-        c.spread_hint = 2 * hit >= N;
-      }
-      c.hist_pending = false;
-    }
-  }
+  if (!captured && (s = read_load_hints(c, N)) != MOE_ZC_OK) return s;
   const bool pace_tiles = N > 0 && T >= 1024 && c.pair_hint;
   if (T > 0) {
     // 1  router GEMM
@@ -518,12 +539,8 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   }
   rec.mark(7);
   if (rec.ev) ++g_prof.n;
-  if (!captured && !c.hist_pending && c.hist_host && N > 0 && T >= 1024) {
-    CK(cudaMemcpyAsync(c.hist_host, cnt, sizeof(int) * N, cudaMemcpyDeviceToHost, st));
-    CK(cudaEventRecord(c.hist_ev, st));
-    c.hist_pending = true;
-    c.hist_N = N;
-  }
+  if (!captured && N > 0 && T >= 1024 && (s = queue_load_hints(c, cnt, N, st)) != MOE_ZC_OK)
+    return s;
   if (!captured) CK(cudaEventRecord(c.done, st));
   c.done_valid = !captured;
   c.has_result = true;
@@ -566,21 +583,39 @@ int forward_host_impl(const void* x_host, const void* W_r, const float* b, const
   Ctx* cp = nullptr;
   if ((s = get_ctx(&cp)) != MOE_ZC_OK) return s;
   Ctx& c = *cp;
-  if (chunk <= 0) {
-    // Four chunks: measured best at the prefill workload (2048: 13.0 ms,
-    // 4096: 12.1 ms, 8192: 12.8 ms per step, B200).  But when earlier
-    // forwards spread their tokens over most FFN experts, every chunk would
-    // stream nearly all expert weights again: one chunk then (balanced
-    // prefill: 18.3 ms per step against 27 ms in four).
-    if (c.spread_hint && c.hist_N == N) {
-      chunk = T;
-    } else {
-      chunk = (T + 3) / 4;
-      chunk = ((chunk + 255) / 256) * 256;
-      if (chunk < 1024) chunk = 1024;
+  // Chunk sizes.  Given: chunk_tokens each.  Default: about T/4 (measured
+  // best of uniform sizes at the prefill workload: 2048: 13.0 ms, 4096:
+  // 12.1 ms, 8192: 12.8 ms per step), with the first and the last chunk
+  // half as long, since the first copy in and the last copy out overlap
+  // nothing (prefill: 2048, 4096, 4096, 4096, 2048).  But when earlier
+  // forwards spread their tokens over most FFN experts, every chunk would
+  // stream nearly all expert weights again: one chunk then (balanced
+  // prefill: 18.3 ms per step against 27 ms in four).
+  std::vector<int64_t> sizes;
+  if (chunk > 0 || (c.spread_hint && c.hist_N == N)) {
+    const int64_t step = chunk > 0 ? chunk : (T > 0 ? T : 1);
+    for (int64_t t0 = 0; t0 < T; t0 += step) sizes.push_back(T - t0 < step ? T - t0 : step);
+  } else {
+    int64_t mid = ((T + 3) / 4 + 255) / 256 * 256;
+    if (mid < 1024) mid = 1024;
+    const int64_t end = mid / 2 / 256 * 256 >= 512 ? mid / 2 / 256 * 256 : 512;
+    int64_t rem = T;
+    if (rem > mid + end) {
+      sizes.push_back(end);
+      rem -= end;
+      while (rem > mid + end) {
+        sizes.push_back(mid);
+        rem -= mid;
+      }
+      if (rem > mid) {
+        sizes.push_back(rem - end);
+        rem = end;
+      }
     }
+    if (rem > 0) sizes.push_back(rem);
   }
-  if (chunk > T) chunk = T;
+  chunk = 0;
+  for (int64_t n : sizes) chunk = n > chunk ? n : chunk;
   const int E = N + Z;
   if ((s = host_streams(c)) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.cnt_total, sizeof(int) * E)) != MOE_ZC_OK) return s;
@@ -596,11 +631,11 @@ int forward_host_impl(const void* x_host, const void* W_r, const float* b, const
   CK(cudaStreamWaitEvent(c.s_out, c.ev_start, 0));
   const char* xh = static_cast<const char*>(x_host);
   char* oh = static_cast<char*>(out_host);
-  const int64_t nchunks = T > 0 ? (T + chunk - 1) / chunk : 0;
-  for (int64_t ci = 0; ci < nchunks; ++ci) {
+  const int64_t nchunks = static_cast<int64_t>(sizes.size());
+  int64_t t0 = 0;
+  for (int64_t ci = 0; ci < nchunks; t0 += sizes[ci], ++ci) {
     const int bi = static_cast<int>(ci & 1);
-    const int64_t t0 = ci * chunk;
-    const int64_t n = (T - t0) < chunk ? (T - t0) : chunk;
+    const int64_t n = sizes[ci];
     // copy in once the kernels of chunk ci-2 are done with this buffer
     if (ci >= 2) CK(cudaStreamWaitEvent(c.s_in, c.ev_comp[bi], 0));
     CK(cudaMemcpyAsync(c.xin[bi].p, xh + t0 * row_bytes, n * row_bytes, cudaMemcpyHostToDevice,
