@@ -254,14 +254,18 @@ __device__ __forceinline__ void epi_router_f32(uint32_t tacc, uint8_t* stg, int 
   }
 }
 
-template <int MODE>
+// NST stages of SB bytes: two A blocks (2 * GEMM_A_BYTES), then the B rows
+// (up to (SB - 2 * GEMM_A_BYTES) / 128 tokens).  The prefill shape has 3
+// stages of 64 KB (256 tokens); batches of at most 64 tokens have 5 stages of
+// 40 KB, so that more weight bytes are in flight per SM while they stream.
+template <int MODE, int NST, int SB>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
             const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBf,
             const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[GEMM_STAGES];
-  __shared__ __align__(8) uint64_t empty_bar[GEMM_STAGES];
+  __shared__ __align__(8) uint64_t full_bar[NST];
+  __shared__ __align__(8) uint64_t empty_bar[NST];
   // Accumulator hand-over.  One-block tiles: [b] = buffer b (TMEM columns
   // 256 b ..).  Two-block tiles: [0] / [1] = first / second accumulator.
   __shared__ __align__(8) uint64_t acc_full_bar[2];
@@ -277,7 +281,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < GEMM_STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
@@ -364,7 +368,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
           abort_sh = 1;
           break;
         }
-        uint8_t* st = smem + stage * GEMM_STAGE_BYTES;
+        uint8_t* st = smem + stage * SB;
         mbar_arrive_expect_tx(&full_bar[stage], bytes);
         armed |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -396,11 +400,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                           tl.brow0 + bx * GEMM_B_BOX_ROWS);
           }
         }
-        if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+        if (++stage == NST) { stage = 0; phase ^= 1; }
       }
     }
     // Drain: every copy this thread started must land before the CTA exits.
-    for (int s = 0; s < GEMM_STAGES; ++s)
+    for (int s = 0; s < NST; ++s)
       if (armed & (1u << s)) mbar_wait(&full_bar[s], (last_par >> s) & 1, DRAIN_NS, p.err);
    }
    __syncwarp();
@@ -427,15 +431,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       // first accumulator alone; they are freed once the second accumulator
       // is back and has had its MMAs on them too.
       const bool stagger = nbuf == 1 && use > 0;
-      const int npre = stagger ? min(nk, GEMM_STAGES) : 0;
+      const int npre = stagger ? min(nk, NST) : 0;
       bool ok = true;
       const int stage0 = stage;
       for (int i = 0; i < npre; ++i) {
         if (!mbar_wait(&full_bar[stage], phase, p.wait_ns, p.err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t st = smem_u32(smem + stage * GEMM_STAGE_BYTES);
+        const uint32_t st = smem_u32(smem + stage * SB);
         mma_kstep(acc0, st, st + 2 * GEMM_A_BYTES, idesc, i == 0);
-        if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+        if (++stage == NST) { stage = 0; phase ^= 1; }
       }
       if (ok && stagger) {
         if (!mbar_wait(&acc_empty_bar[1], par, p.wait_ns, p.err)) {
@@ -444,21 +448,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
           tc_fence_after();
           int s = stage0;
           for (int i = 0; i < npre; ++i) {
-            const uint32_t st = smem_u32(smem + s * GEMM_STAGE_BYTES);
+            const uint32_t st = smem_u32(smem + s * SB);
             if (tl.has_a1) mma_kstep(acc0 + 256, st + GEMM_A_BYTES, st + 2 * GEMM_A_BYTES, idesc, i == 0);
             umma_commit(&empty_bar[s]);
-            if (++s == GEMM_STAGES) s = 0;
+            if (++s == NST) s = 0;
           }
         }
       }
       for (int i = npre; ok && i < nk; ++i) {
         if (!mbar_wait(&full_bar[stage], phase, p.wait_ns, p.err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t st = smem_u32(smem + stage * GEMM_STAGE_BYTES);
+        const uint32_t st = smem_u32(smem + stage * SB);
         mma_kstep(acc0, st, st + 2 * GEMM_A_BYTES, idesc, i == 0);
         if (tl.has_a1) mma_kstep(acc0 + 256, st + GEMM_A_BYTES, st + 2 * GEMM_A_BYTES, idesc, i == 0);
         umma_commit(&empty_bar[stage]);
-        if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+        if (++stage == NST) { stage = 0; phase ^= 1; }
       }
       if (!ok) { abort_sh = 1; break; }
       umma_commit(&acc_full_bar[buf]);
@@ -478,7 +482,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     const int q = warp & 3;
     const int group = (warp - 4) >> 2;
     const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    uint8_t* stg = smem + GEMM_STAGES * GEMM_STAGE_BYTES + (warp - 4) * GEMM_STG_BYTES;
+    uint8_t* stg = smem + NST * SB + (warp - 4) * GEMM_STG_BYTES;
     // H / Y rows are written once here; hint them only for streaming batches
     const uint64_t pol_out = p.l2_stream ? l2_policy_evict_first() : 0;
     int local = 0;
@@ -537,21 +541,33 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   }
 }
 
-template <int MODE>
+template <int MODE, int NST, int SB>
 cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                         const CUtensorMap& b_full, GemmParams p, int grid, cudaStream_t stream) {
-  const cudaError_t e = smem_limit<gemm_kernel<MODE>>(GEMM_SMEM_BYTES);
+  constexpr int smem = NST * SB + GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024;
+  const cudaError_t e = smem_limit<gemm_kernel<MODE, NST, SB>>(smem);
   if (e != cudaSuccess) return e;
   // pacing runs the grid as 2-CTA clusters: an even grid of at least two
   if (p.pair_tiles) {
     if (grid >= 2) {
-      return launch_pdl_pairs(gemm_kernel<MODE>, dim3(grid & ~1), dim3(GEMM_THREADS),
-                              GEMM_SMEM_BYTES, stream, a0, a1, b, b_full, p);
+      return launch_pdl_pairs(gemm_kernel<MODE, NST, SB>, dim3(grid & ~1), dim3(GEMM_THREADS),
+                              smem, stream, a0, a1, b, b_full, p);
     }
     p.pair_tiles = 0;
   }
-  return launch_pdl(gemm_kernel<MODE>, dim3(grid), dim3(GEMM_THREADS), GEMM_SMEM_BYTES, stream,
+  return launch_pdl(gemm_kernel<MODE, NST, SB>, dim3(grid), dim3(GEMM_THREADS), smem, stream,
                     a0, a1, b, b_full, p);
+}
+
+// The stage shapes: prefill (3 x 64 KB) and at most 64 tokens (5 x 40 KB).
+template <int MODE>
+cudaError_t launch_shape(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                         const CUtensorMap& b_full, const GemmParams& p, int grid,
+                         cudaStream_t stream) {
+  if (p.small_b)
+    return launch_mode<MODE, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>(a0, a1, b, b_full, p, grid,
+                                                                         stream);
+  return launch_mode<MODE, GEMM_STAGES, GEMM_STAGE_BYTES>(a0, a1, b, b_full, p, grid, stream);
 }
 
 }  // namespace
@@ -565,14 +581,14 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
     case MODE_ROUTER: {
       GemmParams q = p;
       q.pair_tiles = 0;
-      e = launch_mode<MODE_ROUTER>(a0, a1, b, b_full, q, grid, stream);
+      e = launch_shape<MODE_ROUTER>(a0, a1, b, b_full, q, grid, stream);
       break;
     }
     case MODE_GATEUP:
-      e = launch_mode<MODE_GATEUP>(a0, a1, b, b_full, p, grid, stream);
+      e = launch_shape<MODE_GATEUP>(a0, a1, b, b_full, p, grid, stream);
       break;
     case MODE_DOWN:
-      e = launch_mode<MODE_DOWN>(a0, a1, b, b_full, p, grid, stream);
+      e = launch_shape<MODE_DOWN>(a0, a1, b, b_full, p, grid, stream);
       break;
   }
   if (e != cudaSuccess) return e;

@@ -121,6 +121,14 @@ constexpr int GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;
 constexpr int GEMM_STAGE_BYTES = 2 * GEMM_A_BYTES + GEMM_B_BYTES;
 constexpr int GEMM_SMEM_BYTES =
     GEMM_STAGES * GEMM_STAGE_BYTES + GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024;
+// Stage shape for batches of at most GEMM_SMALL_B tokens (decode): B rows
+// need 8 KB, so five 40 KB stages keep twice the weight bytes in flight.
+constexpr int GEMM_SMALL_B = 64;
+constexpr int GEMM_SMALL_STAGES = 5;
+constexpr int GEMM_SMALL_STAGE_BYTES = 2 * GEMM_A_BYTES + GEMM_SMALL_B * GEMM_BK * 2;
+static_assert(GEMM_SMALL_STAGES * GEMM_SMALL_STAGE_BYTES + GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024 <=
+                  227 * 1024 - 256,
+              "small-batch stages exceed shared memory");
 
 struct GemmParams {
   // Token groups (FFN experts).  For MODE_ROUTER there is one group of T
@@ -141,6 +149,7 @@ struct GemmParams {
   int b_box_full;         // 1: a full token tile's B rows come in one GEMM_BN-row copy
   int tok_tile;           // MODE_ROUTER: tokens per tile (multiple of 16, <= GEMM_BN; 0: GEMM_BN)
   int pair_tiles;         // gate/up, down: 2-CTA clusters pace tiles t, t ^ 1 (even grid)
+  int small_b;            // every token tile has at most GEMM_SMALL_B tokens: small-B stages
   int* zero0;             // MODE_ROUTER: CTA 0 clears zero0[0, nzero0) and zero1[0, nzero1)
   int* zero1;             //   once the previous kernel is done (the next forward's counters)
   int nzero0, nzero1;

@@ -417,6 +417,7 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     pr.split_stride = T * E;
     const int64_t rgrid = rp.tiles * splits;
     pr.b_box_full = full_ok ? 1 : 0;
+    pr.small_b = T <= GEMM_SMALL_B ? 1 : 0;
     pr.zero0 = cnt;
     pr.nzero0 = E;
     pr.zero1 = fill;
@@ -502,6 +503,8 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       pg.wait_ns = wait_ns;
       // decode-sized batches stream every weight byte once
       pg.l2_stream = T < 1024 ? 1 : 0;
+      // at most 64 tokens per expert: five smaller stages, more weights in flight
+      pg.small_b = T <= GEMM_SMALL_B ? 1 : 0;
       pg.b_box_full = full_ok ? 1 : 0;
       // prefill-sized batches: CTA pairs pace the two token tiles of a weight
       // block so that its second read is an L2 hit
