@@ -62,7 +62,7 @@ KERNELS_PER_FORWARD = 7   # router_gemm, route, assign, permute, gateup, down, c
 # Clear an entry when that kernel changes.
 NCU_TRAFFIC_BYTES = {
     "prefill": 9_217_720_576 + 561_846_016,    # gate/up GEMM
-    "decode": 1_520_860_672 + 4_152_064,       # gate/up GEMM
+    "decode": 1_520_890_112 + 4_314_112,       # gate/up GEMM (five-stage shape)
     "prefill_balanced": 30_004_439_040 + 564_574_976,   # gate/up GEMM, paired tiles
 }
 
