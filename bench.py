@@ -447,10 +447,19 @@ def run_reference(args, dist, w):
     b = ri.bias(w.N, w.delta)
     ew = wl.expert_weights(w, "cuda" if torch.cuda.is_available() else "cpu")
     cores = len(os.sched_getaffinity(0))
-    # size the per-step sample so the whole run stays within about two minutes
-    dt1, n1 = oracle_sample_time(w, ri, b, ew, 4, 100)
-    per_tok = dt1 / n1
-    n = int(max(1, min(w.T, 120.0 / max(args.steps + args.warmup, 1) / max(per_tok, 1e-6))))
+    # Size the per-step sample so the whole run stays within about two
+    # minutes: grow it from 16 tokens (doubling, then scaling) while a step
+    # takes under the per-step share; the oracle's cost per token falls as
+    # more tokens share the widened expert weights, so a probe of a few
+    # tokens would overstate it.
+    per_step = 120.0 / max(args.steps + args.warmup, 1)
+    n = min(w.T, 16)
+    dt, n = oracle_sample_time(w, ri, b, ew, n, 100)
+    for i in range(8):
+        if dt >= 0.5 * per_step or n >= w.T:
+            break
+        n = int(min(w.T, max(2 * n, n * 0.8 * per_step / max(dt, 1e-3))))
+        dt, n = oracle_sample_time(w, ri, b, ew, n, 101 + i)
     for i in range(args.warmup):
         oracle_sample_time(w, ri, b, ew, n, 200 + i)
     tot = 0.0
