@@ -108,8 +108,11 @@ int moe_zc_forward_ex(const void* x, const void* W_r, const float* b,
  * at least half of the FFN experts, as each chunk would then stream nearly
  * all expert weights again): while the kernels of one chunk run on
  * `stream`, the next chunk is copied in and the previous one out on two
- * streams of the library's own, so copies overlap compute.  Tokens are independent, so the
- * result equals moe_zc_forward_ex's bit for bit.  Asynchronous: out_host is
+ * streams of the library's own, so copies overlap compute.  Tokens are
+ * independent, so each chunk's rows equal those of moe_zc_forward_ex on the
+ * same chunk bit for bit (and those of one call on all T tokens wherever
+ * the router GEMM slices K the same way for both batch sizes; where it does
+ * not, logits differ in rounding only).  Asynchronous: out_host is
  * complete when `stream` is.  Afterwards moe_zc_expert_load reports the
  * histogram of all T tokens; moe_zc_last_routing and moe_zc_last_expert
  * describe the last chunk only.  Uses device staging for two chunks in and
