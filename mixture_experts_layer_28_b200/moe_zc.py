@@ -26,6 +26,9 @@ ERR_OOM = -4
 ERR_TIMEOUT = -5
 ERR_NO_RESULT = -6
 
+MAX_K = 32      # largest K the library accepts
+MAX_E = 1024    # largest N + Z the library accepts
+
 
 class MoeZcError(RuntimeError):
     def __init__(self, status: int, what: str):

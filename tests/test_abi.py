@@ -22,6 +22,12 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, n), n
 
 
+def test_size_limits_match_header():
+    text = open(mz.HEADER).read()
+    assert f"#define MOE_ZC_MAX_K {mz.MAX_K}" in text
+    assert f"#define MOE_ZC_MAX_E {mz.MAX_E}" in text
+
+
 def test_status_strings(L):
     for code in (mz.OK, mz.ERR_INVALID_ARG, mz.ERR_UNSUPPORTED, mz.ERR_CUDA, mz.ERR_OOM,
                  mz.ERR_TIMEOUT, mz.ERR_NO_RESULT):
@@ -54,6 +60,7 @@ def _fwd(L, x=FAKE, W_r=FAKE, b=FAKE, Wg=FAKE, Wu=FAKE, Wd=FAKE, T=16, d=128, N=
     (dict(I=64), mz.ERR_UNSUPPORTED),             # I % 128
     (dict(N=40, Z=0, K=33), mz.ERR_UNSUPPORTED),  # K > 32
     (dict(N=1000, Z=100, K=2), mz.ERR_UNSUPPORTED),  # E > 1024
+    (dict(N=1000, Z=25, K=2), mz.ERR_UNSUPPORTED),   # E = 1025, one past the largest
     (dict(x=FAKE + 8), mz.ERR_UNSUPPORTED),       # misaligned
     (dict(Wd=FAKE + 2), mz.ERR_UNSUPPORTED),
 ])

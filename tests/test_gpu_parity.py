@@ -125,6 +125,20 @@ def test_dense_limit_k_equals_e():
     _full_check(Case(w), n_expert_checks=6)
 
 
+@pytest.mark.parametrize("N,Z,K,over", [
+    # E and K both at their largest supported values; with the bias at zero
+    # the scores spread the picks over every FFN expert
+    (768, 256, 32, dict(bias="zero", w_std=0.05)),
+    # every one of the largest expert count is an FFN expert
+    (1024, 0, 8, dict(bias="zero", w_std=0.05)),
+    (20, 12, 32, {}),   # K = E = 32: dense at the largest K
+])
+def test_maximum_sizes(N, Z, K, over):
+    w = wl.get("tiny", T=300, d=256, I=128, N=N, Z=Z, K=K, **over)
+    assert w.E <= mz.MAX_E and w.K <= mz.MAX_K
+    _full_check(Case(w), n_expert_checks=6)
+
+
 def test_minimum_widths():
     w = wl.get("tiny", d=128, I=128, T=200)
     _full_check(Case(w))
