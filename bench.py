@@ -55,15 +55,23 @@ METRIC = "MoE-layer tokens/s; executed-FFN TFLOPS as % of B200 bf16 peak (HBM % 
 UNIT = "tokens/s"
 L2_BYTES = 126 * 2 ** 20
 KERNELS_PER_FORWARD = 7   # router_gemm, route, assign, permute, gateup, down, combine
+SMALL_BATCH = 64          # batches of at most this many tokens run gate/up and down as one kernel
+
+
+def kernels_per_forward(w):
+    if w.N == 0:
+        return 4          # router_gemm, route, assign, combine
+    return KERNELS_PER_FORWARD - 1 if w.T <= SMALL_BATCH else KERNELS_PER_FORWARD
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel
 # from an ncu capture of the current kernel build at the full workload (one
-# pass; the full-size GEMM traffic summary under profiles/), per workload.
+# pass; mean over the captured launches; the full-size GEMM traffic summary
+# under profiles/), per workload.
 # Clear an entry when that kernel changes.
 NCU_TRAFFIC_BYTES = {
-    "prefill": 9_217_720_576 + 561_846_016,    # gate/up GEMM
-    "decode": 1_520_890_112 + 4_314_112,       # gate/up GEMM (five-stage shape)
-    "prefill_balanced": 30_004_439_040 + 564_574_976,   # gate/up GEMM, paired tiles
+    "prefill": 8_885_600_000 + 558_700_000,    # gate/up GEMM
+    "decode": 2_278_000_000 + 5_900_000,       # gate/up + down GEMMs in one kernel
+    "prefill_balanced": 30_013_700_000 + 565_300_000,   # gate/up GEMM, paired tiles
 }
 
 
@@ -378,7 +386,11 @@ def run_ours(args, dist, w):
     # ---- roofline of the dominant kernel (largest share of the step)
     per = {k: v / max(nfw, 1) for k, v in stage_ms.items()}
     dom = max(per, key=per.get)
-    kern = {"gateup_gemm": (rf["F_gateup"], rf["B_gateup"]),
+    # (batches of at most SMALL_BATCH tokens: the gate/up stage is the one
+    # kernel that runs both expert GEMMs)
+    fused = w.N > 0 and w.T <= SMALL_BATCH
+    kern = {"gateup_gemm": ((rf["F_gateup"] + rf["F_down"], rf["B_gateup"] + rf["B_down"])
+                            if fused else (rf["F_gateup"], rf["B_gateup"])),
             "down_gemm": (rf["F_down"], rf["B_down"])}.get(dom)
     roof = None
     if kern and per[dom] > 0:
@@ -394,7 +406,7 @@ def run_ours(args, dist, w):
             ach = B / sec / 1e9
             roof = {"bound": "hbm", "achieved": ach, "peak": pk["hbm"], "unit": "GB/s",
                     "frac": ach / pk["hbm"], "peak_kind": f"HBM copy ({pk['src']})"}
-        roof["kernel"] = dom
+        roof["kernel"] = "gateup_down_gemm (one kernel)" if fused and dom == "gateup_gemm" else dom
         roof["ms_per_launch"] = per[dom]
         tr = NCU_TRAFFIC_BYTES.get(w.name)
         roof["traffic"] = tr
@@ -431,7 +443,7 @@ def run_ours(args, dist, w):
         "roofline": roof,
         "layer_roofline": layer,
         "cpu_baseline": cpu,
-        "gpu_launches": KERNELS_PER_FORWARD * args.steps if w.N > 0 else 4 * args.steps,
+        "gpu_launches": kernels_per_forward(w) * args.steps,
         "clocks": clk,
         "routing": st,
         "stage_ms": {k: round(v, 5) for k, v in per.items()},

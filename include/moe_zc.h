@@ -204,7 +204,9 @@ const char* moe_zc_status_string(int status);
  * forward and writes, for each stage i < max_stages, the milliseconds summed
  * over the recorded forwards (stage_ms: host float[max_stages]; 7 stages,
  * named by moe_zc_stage_name: router_gemm, route, assign_slots, permute,
- * gateup_gemm, down_gemm, combine) and their count to *n_forwards.
+ * gateup_gemm, down_gemm, combine) and their count to *n_forwards.  A batch
+ * of at most 64 tokens runs both expert GEMMs as one kernel: its time is
+ * under gateup_gemm, and down_gemm covers no kernel.
  */
 int moe_zc_profile(int32_t enable);
 int moe_zc_profile_read(float* stage_ms, int32_t max_stages, int32_t* n_forwards);

@@ -39,6 +39,10 @@
 //     accumulator, then the second, and the issuer starts the next tile's
 //     first-block MMAs on up to GEMM_STAGES loaded stages before it needs
 //     the second accumulator back.
+// Batches of at most 64 tokens (decode) stream weights: there the gate/up and
+// down tiles run in one persistent grid (MODE_FUSED, see gemm_kernel), so the
+// SMs that the last, part-filled round of gate/up tiles leaves idle stream
+// down weights of the experts whose H rows are already complete.
 // Every wait is time-bounded (ptx.cuh); on running out the CTA drains its
 // in-flight copies and MMAs, frees TMEM and returns with the error flag set.
 #include "epilogue.cuh"
@@ -164,6 +168,47 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   return tl;
 }
 
+// Tile `it` of this CTA's list: phase 0 tiles are the mode's own (for
+// MODE_FUSED the gate/up tiles), phase 1 the down tiles of MODE_FUSED.
+// One-phase modes and the gate/up phase take tiles blockIdx.x + i * G of the
+// n0.  The n1 down tiles then go out so that the CTAs finish together: the
+// r = n0 % G CTAs that hold one gate/up tile more join p.down_lead down tiles
+// later.  With F = G - r, down tile j belongs to
+//   j <  L * F:  CTA r + j % F (its (j / F)-th down tile),
+//   j >= L * F:  CTA (j - L * F) % G,
+// so that every CTA meets its down tiles, and the groups, in increasing
+// order: the earliest finished gate/up results are read first.
+template <int MODE>
+__device__ __forceinline__ bool tile_at(const GemmParams& p, int it, int n0, int n1, int& tph,
+                                        int& t) {
+  const int c = blockIdx.x;
+  const int G = gridDim.x;
+  if (MODE != MODE_FUSED || it < (c < n0 ? (n0 - 1 - c) / G + 1 : 0)) {
+    tph = 0;
+    t = c + it * G;
+    return t < n0;
+  }
+  const int k = it - (c < n0 ? (n0 - 1 - c) / G + 1 : 0);
+  const int r = n0 % G;
+  const int F = G - r;
+  const int L = p.down_lead;
+  tph = 1;
+  if (c >= r && k < L) {
+    t = k * F + (c - r);
+  } else {
+    t = L * F + (c >= r ? k - L : k) * G + c;
+  }
+  return t < n1;
+}
+
+// Tile t of the given phase (see tile_at).
+template <int MODE>
+__device__ __forceinline__ Tile phase_tile(const GemmParams& p, const GemmParams& p2, int tph,
+                                           int t) {
+  if (MODE == MODE_FUSED) return tph ? decode_tile<MODE_DOWN>(p2, t) : decode_tile<MODE_GATEUP>(p, t);
+  return decode_tile<MODE>(p, t);
+}
+
 
 // One 64-wide K step of one A block: four K = 16 MMAs into accumulator d.
 __device__ __forceinline__ void mma_kstep(uint32_t d, uint32_t a_smem, uint32_t b_smem,
@@ -258,11 +303,23 @@ __device__ __forceinline__ void epi_router_f32(uint32_t tacc, uint8_t* stg, int 
 // (up to (SB - 2 * GEMM_A_BYTES) / 128 tokens).  The prefill shape has 3
 // stages of 64 KB (256 tokens); batches of at most 64 tokens have 5 stages of
 // 40 KB, so that more weight bytes are in flight per SM while they stream.
+//
+// MODE_FUSED runs the gate/up tiles (maps tmA0, tmA1, tmB; parameters p) and
+// then the down tiles (maps tmA2 for both A blocks, tmB2; parameters p2) of
+// one forward in one grid, so that the SMs left idle in the last, part-filled
+// round of gate/up tiles already stream down weights.  A down tile of group g
+// reads H rows that other CTAs write: its producer waits (bounded) until all
+// GEMM_EPI_WARPS * mblocks * ntt epilogue warps of g's gate/up tiles have
+// counted themselves in p.done[g].  No wait can close a cycle: every CTA
+// holds all its gate/up tiles before its down tiles, gate/up tiles wait on
+// nothing outside their CTA, and the grid (one CTA per SM, at most one per
+// SM of the device) is resident as a whole.
 template <int MODE, int NST, int SB>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
             const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBf,
-            const GemmParams p) {
+            const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+            const GemmParams p, const GemmParams p2) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[NST];
   __shared__ __align__(8) uint64_t empty_bar[NST];
@@ -297,6 +354,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmBf);
+    if (MODE == MODE_FUSED) {
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB2);
+    }
   }
   __syncwarp();
   if (warp == 2) {
@@ -318,10 +379,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     for (int i = threadIdx.x; i < p.nzero1; i += blockDim.x) p.zero1[i] = 0;
   }
   const uint32_t tmem = tmem_base_sh;
-  const int ntiles = total_tiles<MODE>(p);
+  const int ntiles = total_tiles<MODE == MODE_FUSED ? MODE_GATEUP : MODE>(p);
+  const int ntiles2 = MODE == MODE_FUSED ? total_tiles<MODE_DOWN>(p2) : 0;
   // gate/up tiles always hold two blocks; router and down tiles hold one
   // when p.single_a is set (1 buffer of 512 columns, or 2 of 256)
-  const int nbuf = (MODE == MODE_GATEUP || !p.single_a) ? 1 : 2;
+  // (MODE_FUSED: both phases hold two blocks)
+  const int nbuf = (MODE == MODE_GATEUP || MODE == MODE_FUSED || !p.single_a) ? 1 : 2;
 
   // Single-thread roles run on lane 0; the other lanes of their warp wait at
   // a __syncwarp so that every warp reaches the final CTA barrier converged.
@@ -347,10 +410,28 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     const uint32_t peer_word =
         p.pair_tiles ? mapa_shared(smem_u32(&peer_tile_sh), cluster_ctarank() ^ 1u) : 0u;
     uint32_t begun = 0;
-    for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x) {
-      const Tile tl = decode_tile<MODE>(p, t);
+    for (int it = 0; !abort_sh; ++it) {
+      int tph, t;
+      if (!tile_at<MODE>(p, it, ntiles, ntiles2, tph, t)) break;
+      const Tile tl = phase_tile<MODE>(p, p2, tph, t);
+      const bool down_ph = MODE == MODE_FUSED && tph == 1;
+      if (down_ph) {
+        // group tl.g's H rows are all stored once every epilogue warp of its
+        // gate/up tiles has counted itself; the acquire and the proxy fence
+        // order this CTA's bulk copies of them after those stores
+        const int need = GEMM_EPI_WARPS * p.mblocks * tl.ntt;
+        if (!wait_count_geq(p.done + tl.g, need, p.wait_ns, p.err)) {
+          abort_sh = 1;
+          break;
+        }
+        fence_proxy_async_global();
+      }
+      const CUtensorMap* mA0 = down_ph ? &tmA2 : &tmA0;
+      const CUtensorMap* mA1 = down_ph ? &tmA2 : &tmA1;
+      const CUtensorMap* mB = down_ph ? &tmB2 : &tmB;
       // both CTAs evaluate the same predicate on the pair (t, t ^ 1)
-      if (MODE != MODE_ROUTER && p.pair_tiles && tl.ntt == 2 && (t ^ 1) < ntiles &&
+      if (MODE != MODE_ROUTER && MODE != MODE_FUSED && p.pair_tiles && tl.ntt == 2 &&
+          (t ^ 1) < ntiles &&
           group_of_tile(p, t ^ 1) == tl.g) {
         ++begun;
         st_cluster_u32(peer_word, begun);
@@ -360,7 +441,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       // a full token tile (256 tokens; the router's tile size) in one copy
       // of the b_full map, whose box has exactly that many rows
       const int full_rows = MODE == MODE_ROUTER ? router_tok_tile(p) : GEMM_BN;
-      const bool full_box = p.b_box_full && tl.nmma == full_rows;
+      const bool full_box = MODE != MODE_FUSED && p.b_box_full && tl.nmma == full_rows;
       const uint32_t bytes = GEMM_A_BYTES * (tl.has_a1 ? 2 : 1) +
                              (full_box ? tl.nmma : nbox * GEMM_B_BOX_ROWS) * GEMM_BK * 2;
       for (int ks = tl.k0; ks < tl.k1; ++ks) {
@@ -378,25 +459,24 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         // evict-last weights or evict-first tokens there cost ~4%).
         uint8_t* sb = st + 2 * GEMM_A_BYTES;
         if (p.l2_stream) {
-          tma_load_2d_hint(st, &tmA0, &full_bar[stage], kc, tl.a0_row, pol_stream);
+          tma_load_2d_hint(st, mA0, &full_bar[stage], kc, tl.a0_row, pol_stream);
           if (tl.has_a1)
-            tma_load_2d_hint(st + GEMM_A_BYTES, &tmA1, &full_bar[stage], kc, tl.a1_row,
-                             pol_stream);
+            tma_load_2d_hint(st + GEMM_A_BYTES, mA1, &full_bar[stage], kc, tl.a1_row, pol_stream);
           if (full_box) {
             tma_load_2d_hint(sb, &tmBf, &full_bar[stage], kc, tl.brow0, pol_stream);
           } else {
             for (int bx = 0; bx < nbox; ++bx)
-              tma_load_2d_hint(sb + bx * GEMM_B_BOX_ROWS * GEMM_BK * 2, &tmB, &full_bar[stage],
-                               kc, tl.brow0 + bx * GEMM_B_BOX_ROWS, pol_stream);
+              tma_load_2d_hint(sb + bx * GEMM_B_BOX_ROWS * GEMM_BK * 2, mB, &full_bar[stage], kc,
+                               tl.brow0 + bx * GEMM_B_BOX_ROWS, pol_stream);
           }
         } else {
-          tma_load_2d(st, &tmA0, &full_bar[stage], kc, tl.a0_row);
-          if (tl.has_a1) tma_load_2d(st + GEMM_A_BYTES, &tmA1, &full_bar[stage], kc, tl.a1_row);
+          tma_load_2d(st, mA0, &full_bar[stage], kc, tl.a0_row);
+          if (tl.has_a1) tma_load_2d(st + GEMM_A_BYTES, mA1, &full_bar[stage], kc, tl.a1_row);
           if (full_box) {
             tma_load_2d(sb, &tmBf, &full_bar[stage], kc, tl.brow0);
           } else {
             for (int bx = 0; bx < nbox; ++bx)
-              tma_load_2d(sb + bx * GEMM_B_BOX_ROWS * GEMM_BK * 2, &tmB, &full_bar[stage], kc,
+              tma_load_2d(sb + bx * GEMM_B_BOX_ROWS * GEMM_BK * 2, mB, &full_bar[stage], kc,
                           tl.brow0 + bx * GEMM_B_BOX_ROWS);
           }
         }
@@ -413,11 +493,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     // ------------------------------------------------------------ MMA issuer
     int stage = 0;
     uint32_t phase = 0;
-    int local = 0;
-    for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x, ++local) {
-      const Tile tl = decode_tile<MODE>(p, t);
+    for (int local = 0; !abort_sh; ++local) {
+      int tph, t;
+      if (!tile_at<MODE>(p, local, ntiles, ntiles2, tph, t)) break;
+      const Tile tl = phase_tile<MODE>(p, p2, tph, t);
       const int buf = local % nbuf;
       const int use = local / nbuf;
+      (void)tph;
       const uint32_t par = static_cast<uint32_t>(use - 1) & 1u;
       const uint32_t acc0 = tmem + buf * 256;
       if (use > 0 && !mbar_wait(&acc_empty_bar[buf], par, p.wait_ns, p.err)) {
@@ -485,9 +567,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     uint8_t* stg = smem + NST * SB + (warp - 4) * GEMM_STG_BYTES;
     // H / Y rows are written once here; hint them only for streaming batches
     const uint64_t pol_out = p.l2_stream ? l2_policy_evict_first() : 0;
-    int local = 0;
-    for (int t = blockIdx.x; t < ntiles && !abort_sh; t += gridDim.x, ++local) {
-      const Tile tl = decode_tile<MODE>(p, t);
+    for (int local = 0; !abort_sh; ++local) {
+      int tph, t;
+      if (!tile_at<MODE>(p, local, ntiles, ntiles2, tph, t)) break;
+      const Tile tl = phase_tile<MODE>(p, p2, tph, t);
       const int buf = local % nbuf;
       if (!mbar_wait(&acc_full_bar[buf], (local / nbuf) & 1, p.wait_ns, p.err)) {
         abort_sh = 1;
@@ -495,7 +578,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       }
       tc_fence_after();
       const uint32_t tacc = tq + buf * 256;
-      const int row_blk = tl.m * (p.single_a ? 1 : 2) * GEMM_BM + q * 32;   // router / down
+      const bool down_ph = MODE == MODE_FUSED && tph == 1;
+      // router / down (MODE_FUSED's down tiles hold two blocks)
+      const int row_blk = tl.m * ((MODE == MODE_FUSED || !p.single_a) ? 2 : 1) * GEMM_BM + q * 32;
       if (MODE == MODE_ROUTER) {
         epi_router_f32(tacc, stg, lane, group, tl, p, row_blk);
         tc_fence_before();
@@ -505,27 +590,39 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
           tc_fence_before();
           mbar_arrive(&acc_empty_bar[1]);
         }
-      } else if (MODE == MODE_GATEUP) {
+      } else if (MODE == MODE_GATEUP || (MODE == MODE_FUSED && !down_ph)) {
         uint32_t hp[3][16];
         epi_read_bf16<MODE_GATEUP>(tacc, group, tl.nmma, hp);
         tc_fence_before();
         mbar_arrive(&acc_empty_bar[0]);
         mbar_arrive(&acc_empty_bar[1]);
+        // (MODE_FUSED reads H back in this grid: default L2 policy)
         epi_store_bf16(stg, lane, group, tl, hp,
                        static_cast<__nv_bfloat16*>(p.out) + tl.m * GEMM_BM + q * 32, p.out_ld,
-                       pol_out);
+                       MODE == MODE_FUSED ? 0 : pol_out);
+        if (MODE == MODE_FUSED) {
+          // publish this warp's H rows of the tile to the down tiles of
+          // tl.g: each lane's stores are made visible (also to bulk copies)
+          // before lane 0 counts the warp in
+          fence_proxy_async_global();
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) atomicAdd(p.done + tl.g, 1);
+        }
       } else {
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row_blk;
+        __nv_bfloat16* out =
+            static_cast<__nv_bfloat16*>(MODE == MODE_FUSED ? p2.out : p.out) + row_blk;
+        const int64_t out_ld = MODE == MODE_FUSED ? p2.out_ld : p.out_ld;
         uint32_t hp[3][16];
         epi_read_bf16<MODE_DOWN>(tacc, group, tl.nmma, hp);
         tc_fence_before();
         mbar_arrive(&acc_empty_bar[buf]);
-        epi_store_bf16(stg, lane, group, tl, hp, out, p.out_ld, pol_out);
+        epi_store_bf16(stg, lane, group, tl, hp, out, out_ld, pol_out);
         if (nbuf == 1) {
           if (tl.has_a1) epi_read_bf16<MODE_DOWN>(tacc + 256, group, tl.nmma, hp);
           tc_fence_before();
           mbar_arrive(&acc_empty_bar[1]);
-          if (tl.has_a1) epi_store_bf16(stg, lane, group, tl, hp, out + GEMM_BM, p.out_ld, pol_out);
+          if (tl.has_a1) epi_store_bf16(stg, lane, group, tl, hp, out + GEMM_BM, out_ld, pol_out);
         }
       }
     }
@@ -541,9 +638,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   }
 }
 
+// a2, b2, p2: MODE_FUSED's down phase (other modes: copies of a0, b, p).
 template <int MODE, int NST, int SB>
 cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
-                        const CUtensorMap& b_full, GemmParams p, int grid, cudaStream_t stream) {
+                        const CUtensorMap& b_full, const CUtensorMap& a2, const CUtensorMap& b2,
+                        GemmParams p, const GemmParams& p2, int grid, cudaStream_t stream) {
   constexpr int smem = NST * SB + GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024;
   const cudaError_t e = smem_limit<gemm_kernel<MODE, NST, SB>>(smem);
   if (e != cudaSuccess) return e;
@@ -551,12 +650,12 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   if (p.pair_tiles) {
     if (grid >= 2) {
       return launch_pdl_pairs(gemm_kernel<MODE, NST, SB>, dim3(grid & ~1), dim3(GEMM_THREADS),
-                              smem, stream, a0, a1, b, b_full, p);
+                              smem, stream, a0, a1, b, b_full, a2, b2, p, p2);
     }
     p.pair_tiles = 0;
   }
   return launch_pdl(gemm_kernel<MODE, NST, SB>, dim3(grid), dim3(GEMM_THREADS), smem, stream,
-                    a0, a1, b, b_full, p);
+                    a0, a1, b, b_full, a2, b2, p, p2);
 }
 
 // The stage shapes: prefill (3 x 64 KB) and at most 64 tokens (5 x 40 KB).
@@ -565,9 +664,10 @@ cudaError_t launch_shape(const CUtensorMap& a0, const CUtensorMap& a1, const CUt
                          const CUtensorMap& b_full, const GemmParams& p, int grid,
                          cudaStream_t stream) {
   if (p.small_b)
-    return launch_mode<MODE, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>(a0, a1, b, b_full, p, grid,
-                                                                         stream);
-  return launch_mode<MODE, GEMM_STAGES, GEMM_STAGE_BYTES>(a0, a1, b, b_full, p, grid, stream);
+    return launch_mode<MODE, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>(a0, a1, b, b_full, a0, b, p,
+                                                                         p, grid, stream);
+  return launch_mode<MODE, GEMM_STAGES, GEMM_STAGE_BYTES>(a0, a1, b, b_full, a0, b, p, p, grid,
+                                                          stream);
 }
 
 }  // namespace
@@ -591,6 +691,21 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
       e = launch_shape<MODE_DOWN>(a0, a1, b, b_full, p, grid, stream);
       break;
   }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, const CUtensorMap& xp,
+                              const CUtensorMap& wd, const CUtensorMap& h, const GemmParams& pg,
+                              const GemmParams& pd, int grid, cudaStream_t stream) {
+  if (grid <= 0) return cudaSuccess;
+  // every CTA resident at once (one per SM): a down tile may wait for
+  // gate/up tiles of any other CTA
+  if (grid > device_sms() || !pg.small_b || pg.pair_tiles || pg.b_box_full || pd.single_a ||
+      pg.done == nullptr)
+    return cudaErrorInvalidValue;
+  const cudaError_t e = launch_mode<MODE_FUSED, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>(
+      wg, wu, xp, xp, wd, h, pg, pd, grid, stream);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -104,7 +104,9 @@ inline int device_sms() {
 // One tcgen05 engine serves the three contractions of the layer.  Weights are
 // the A operand (M = 128 rows per MMA, two A blocks per tile -> two fp32
 // accumulators in TMEM); tokens are the B operand (N = 16..256 per tile).
-enum GemmMode : int { MODE_ROUTER = 0, MODE_GATEUP = 1, MODE_DOWN = 2 };
+// MODE_FUSED: the gate/up and down GEMMs of batches of at most GEMM_SMALL_B
+// tokens in one persistent grid (launch_gemm_fused).
+enum GemmMode : int { MODE_ROUTER = 0, MODE_GATEUP = 1, MODE_DOWN = 2, MODE_FUSED = 3 };
 
 constexpr int GEMM_BM = 128;           // rows of one A block
 constexpr int GEMM_BN = 256;           // tokens per tile at most
@@ -159,6 +161,13 @@ struct GemmParams {
   int out_ld;             // elements per output row
   int* err;               // device error flag
   long long wait_ns;      // bound of every pipeline wait
+  // MODE_FUSED (set in the gate/up parameters): done[g] counts the epilogue
+  // warps that have stored their part of a gate/up tile of group g (zeroed
+  // before the launch); a down tile of group g starts once all of them have.
+  // down_lead: down tiles that the CTAs with one gate/up tile fewer take
+  // first (about a gate/up tile's cost in down tiles).
+  int* done;
+  int down_lead;
 };
 
 // b: B map with GEMM_B_BOX_ROWS-row boxes; b_full: with GEMM_BN-row boxes,
@@ -167,6 +176,14 @@ struct GemmParams {
 cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap& a1,
                         const CUtensorMap& b, const CUtensorMap& b_full, const GemmParams& p,
                         int grid, cudaStream_t stream);
+
+// Gate/up then down in one persistent grid of `grid` CTAs (batches of at most
+// GEMM_SMALL_B tokens): wg, wu, xp as for the gate/up launch (parameters pg,
+// with pg.done and pg.down_lead set), wd and h as for the down launch
+// (parameters pd).
+cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, const CUtensorMap& xp,
+                              const CUtensorMap& wd, const CUtensorMap& h, const GemmParams& pg,
+                              const GemmParams& pd, int grid, cudaStream_t stream);
 
 // The FFN expert GEMMs on CTA pairs (cta_group::2, M = 256 per MMA), for
 // batches with many tokens per expert; `clusters` pairs are launched.

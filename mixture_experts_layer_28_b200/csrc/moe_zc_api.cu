@@ -248,7 +248,8 @@ int reserve_impl(Ctx& c, int64_t T, int d, int N, int Z, int K, int I) {
   if ((s = ensure(c, c.slot, static_cast<size_t>(pairs) * sizeof(int))) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.zsum, static_cast<size_t>(T) * sizeof(float))) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.cnt, static_cast<size_t>(E) * sizeof(int))) != MOE_ZC_OK) return s;
-  if ((s = ensure(c, c.fill, static_cast<size_t>(N + 1) * sizeof(int))) != MOE_ZC_OK) return s;
+  // fill: [N + 1] slot counters, then [N + 1] gate/up completion counters
+  if ((s = ensure(c, c.fill, static_cast<size_t>(2 * N + 2) * sizeof(int))) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.grp_off, static_cast<size_t>(N + 1) * sizeof(int))) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.grp_ttp, static_cast<size_t>(N + 1) * sizeof(int))) != MOE_ZC_OK) return s;
   if (N > 0) {
@@ -421,7 +422,7 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     pr.zero0 = cnt;
     pr.nzero0 = E;
     pr.zero1 = fill;
-    pr.nzero1 = N;
+    pr.nzero1 = 2 * N + 2;
     CK(launch_gemm(MODE_ROUTER, mWr, mWr, mX, mXf, pr,
                    static_cast<int>(rgrid < c.sms ? rgrid : c.sms), st));
     rec.mark(1);
@@ -509,11 +510,6 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       // prefill-sized batches: CTA pairs pace the two token tiles of a weight
       // block so that its second read is an L2 hit
       pg.pair_tiles = pace_tiles ? 1 : 0;
-      const int64_t g_ub = tiles_ub * pg.mblocks;
-      CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg, static_cast<int>(g_ub < c.sms ? g_ub : c.sms),
-                     st));
-      rec.mark(5);
-      // 6  down GEMM
       CUtensorMap mWd, mH;
       if (!make_map(&mWd, W_down, static_cast<uint64_t>(N) * d, I, GEMM_BM) ||
           !make_map(&mH, c.H.p, c.rows_cap, I, GEMM_B_BOX_ROWS))
@@ -524,10 +520,32 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       pd.a_rows = d;
       pd.out = c.Y.p;
       pd.out_ld = d;
+      const int64_t g_ub = tiles_ub * pg.mblocks;
       const int64_t d_ub = tiles_ub * pd.mblocks;
-      CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd, static_cast<int>(d_ub < c.sms ? d_ub : c.sms),
-                     st));
-      rec.mark(6);
+      if (pg.small_b) {
+        // 5-6  at most 64 tokens: both expert GEMMs in one persistent grid,
+        // the down tiles of an expert starting as soon as its H rows are
+        // stored (the SMs that the last round of gate/up tiles leaves idle
+        // stream down weights meanwhile); a gate/up tile costs about d / I
+        // down tiles
+        pg.b_box_full = 0;
+        pg.done = fill + N + 1;
+        pg.down_lead = (d + I / 2) / I;
+        const int64_t f_ub = g_ub + d_ub;
+        CK(launch_gemm_fused(mWg, mWu, mXp, mWd, mH, pg, pd,
+                             static_cast<int>(f_ub < c.sms ? f_ub : c.sms), st));
+        rec.mark(5);
+        rec.mark(6);
+      } else {
+        // 5  gate/up GEMM
+        CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg,
+                       static_cast<int>(g_ub < c.sms ? g_ub : c.sms), st));
+        rec.mark(5);
+        // 6  down GEMM
+        CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd,
+                       static_cast<int>(d_ub < c.sms ? d_ub : c.sms), st));
+        rec.mark(6);
+      }
       }
     } else {
       CK(launch_assign_slots(cnt, idx, T * K, N, grp_off, grp_ttp, fill, slot, st));

@@ -260,6 +260,34 @@ __device__ __forceinline__ void pace_until_shared(const void* p, uint32_t target
   }
 }
 
+// Counters in global memory that CTAs of one grid publish progress through:
+// the writer stores its data, fences and adds; the reader waits (bounded) for
+// the count with acquire loads and then orders its later bulk-tensor (async
+// proxy) reads after what it has seen.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Wait until *p >= target for at most limit_ns; on running out record
+// DEV_TIMEOUT in *err and return false.
+__device__ __forceinline__ bool wait_count_geq(const int* p, int target, long long limit_ns,
+                                               int* err) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(128);
+    if (ld_acquire_gpu(p) >= target) return true;
+    if (static_cast<long long>(globaltimer_ns() - t0) > limit_ns) {
+      atomicCAS(err, DEV_OK, DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Named barrier over `nthreads` threads (multiple of 32) of this CTA.
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
