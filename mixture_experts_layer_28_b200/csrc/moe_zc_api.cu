@@ -13,6 +13,7 @@
 //   4  permute            x rows -> Xp (grouped by expert)
 //   5  gate/up GEMM       H = SiLU(Xp W_gate^T) * (Xp W_up^T)
 //   6  down GEMM          Y = H W_down^T
+//                         (batches of at most 64 tokens: 5 and 6 in one grid)
 //   7  combine            out = zsum x + sum gate * Y
 //
 // No step reads anything back to the host: the GEMM tile lists are built on
