@@ -690,6 +690,8 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
     case MODE_DOWN:
       e = launch_shape<MODE_DOWN>(a0, a1, b, b_full, p, grid, stream);
       break;
+    case MODE_FUSED:   // two phases: launch_gemm_fused
+      return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
