@@ -32,6 +32,15 @@ readings are taken (each one is a test):
       their input tokens quantised), the down projection stays bf16.
 The dequantised value of a code is decode(code) * scale, exactly, in fp64;
 the layer is then the fp64 definition of moe_zc_ref on dequantised operands.
+
+A second reading, for the tensor cores' block-scaled FP8 form, replaces Q2-Q4
+(the ``mx`` functions below):
+  M1  weights and activations alike are cut into 1 x 32 blocks along the
+      contraction dimension (one weight row or one token, 32 consecutive
+      features), each with one power-of-two scale (an 8-bit exponent);
+  M2  the scale is the smallest power of two with amax / scale <= 448, so no
+      element saturates; an all-zero block gets scale 1.
+Q1, Q5-Q7 hold for it unchanged (dividing by a power of two is exact).
 """
 from __future__ import annotations
 
@@ -44,6 +53,7 @@ from oracle import moe_zc_ref as ref
 E4M3_MAX = 448.0
 WEIGHT_BLOCK = (128, 128)   # Q2
 ACT_TILE = (1, 128)         # Q3
+MX_BLOCK = (1, 32)          # M1
 
 
 def e4m3_value(code: int) -> float:
@@ -111,6 +121,41 @@ def dequantize_blocks(codes, scales, block: Tuple[int, int]) -> np.ndarray:
     return e4m3_decode(codes) * s[: codes.shape[0], : codes.shape[1]]
 
 
+def quantize_mx(W) -> Tuple[np.ndarray, np.ndarray]:
+    """(codes uint8 [R, C], scales float32 [R, ceil(C/32)]) under M1-M2: each
+    1 x 32 block's scale is 2^ceil(log2(amax / 448))."""
+    W = np.asarray(W, dtype=np.float32)
+    R, C = W.shape
+    nb = -(-C // MX_BLOCK[1])
+    scales = np.ones((R, nb), dtype=np.float32)
+    codes = np.zeros((R, C), dtype=np.uint8)
+    for j in range(nb):
+        blk = W[:, j * MX_BLOCK[1]:(j + 1) * MX_BLOCK[1]]
+        amax = np.max(np.abs(blk), axis=1).astype(np.float64)
+        e = np.zeros(R)
+        nz = amax > 0
+        e[nz] = np.ceil(np.log2(amax[nz] / E4M3_MAX))
+        # guard the log2 rounding: the smallest power of two with amax / s <= 448
+        s = np.ldexp(1.0, e.astype(int))
+        lower = nz & (amax / (s / 2) <= E4M3_MAX)
+        s[lower] /= 2
+        s[~nz] = 1.0
+        scales[:, j] = s.astype(np.float32)
+        codes[:, j * MX_BLOCK[1]:(j + 1) * MX_BLOCK[1]] = e4m3_encode(blk / s[:, None].astype(np.float32))
+    return codes, scales
+
+
+def fp8_swiglu_expert_mx(xs, Wg_q, Wu_q, Wd) -> np.ndarray:
+    """E(x) with FP8 gate/up under the block-scaled reading (M1-M2): tokens
+    and weights in 1 x 32 blocks along d; the down projection unquantised."""
+    cx, sx = quantize_mx(xs)
+    Xd = dequantize_blocks(cx, sx, MX_BLOCK)
+    Wg = dequantize_blocks(*Wg_q, MX_BLOCK)
+    Wu = dequantize_blocks(*Wu_q, MX_BLOCK)
+    H = ref.silu(Xd @ Wg.T) * (Xd @ Wu.T)
+    return H @ ref._f64(Wd).T
+
+
 def quantize_weight(W) -> Tuple[np.ndarray, np.ndarray]:
     """One expert matrix in 128 x 128 blocks (Q2)."""
     return quantize_blocks(W, WEIGHT_BLOCK)
@@ -133,17 +178,19 @@ def fp8_swiglu_expert(xs, Wg_q, Wu_q, Wd) -> np.ndarray:
     return H @ ref._f64(Wd).T
 
 
-def forward_rows_fp8(x, r: ref.Routing,
-                     expert: Callable[[int], Sequence]) -> np.ndarray:
+def forward_rows_fp8(x, r: ref.Routing, expert: Callable[[int], Sequence],
+                     mx: bool = False) -> np.ndarray:
     """out_t for the rows of x routed by r (routing as in moe_zc_ref: the
-    router stays bf16/fp32), FFN terms from fp8_swiglu_expert.  ``expert(e)``
-    returns ((codes, scales) of W_gate[e], (codes, scales) of W_up[e],
-    W_down[e])."""
+    router stays bf16/fp32), FFN terms from fp8_swiglu_expert (mx: from
+    fp8_swiglu_expert_mx).  ``expert(e)`` returns ((codes, scales) of
+    W_gate[e], (codes, scales) of W_up[e], W_down[e]), quantised with
+    quantize_weight (mx: quantize_mx)."""
     xs = ref._f64(x)
     xq = xs.astype(np.float32)      # exact: x holds bf16 values
     out = r.zsum[:, None] * xs
+    term = fp8_swiglu_expert_mx if mx else fp8_swiglu_expert
     for e in np.unique(r.idx[r.idx < r.N]):
         rows, ks = np.nonzero(r.idx == e)
         Wg_q, Wu_q, Wd = expert(int(e))
-        out[rows] += r.gate[rows, ks][:, None] * fp8_swiglu_expert(xq[rows], Wg_q, Wu_q, Wd)
+        out[rows] += r.gate[rows, ks][:, None] * term(xq[rows], Wg_q, Wu_q, Wd)
     return out

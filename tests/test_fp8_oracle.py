@@ -268,3 +268,97 @@ def test_fp8_mutant_is_caught(name, monkeypatch):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"no pin catches: {name}"
+
+
+# ------------------------------------------------- block-scaled reading (M1-M2)
+
+def test_mx_scales_are_the_smallest_powers_of_two_without_saturation():
+    W = _gauss((16, 200), 11, 0.02)                  # ragged last block of 8
+    W[3, 64:96] = 0.0                                 # an all-zero block
+    codes, scales = f8.quantize_mx(W)
+    assert scales.shape == (16, 7)
+    e = np.log2(scales.astype(np.float64))
+    assert np.array_equal(e, np.round(e))
+    assert scales[3, 2] == 1.0 and np.all(codes[3, 64:96] & 0x7F == 0)
+    for j in range(7):
+        amax = np.abs(W[:, 32 * j:32 * (j + 1)]).max(axis=1).astype(np.float64)
+        nz = amax > 0
+        s = scales[nz, j].astype(np.float64)
+        assert np.all(amax[nz] / s <= 448.0) and np.all(amax[nz] / (s / 2) > 448.0)
+    deq = f8.dequantize_blocks(codes, scales, f8.MX_BLOCK)
+    s_el = np.repeat(scales.astype(np.float64), 32, axis=1)[:, :200]
+    W64 = W.astype(np.float64)
+    normal = np.abs(W64) >= 2.0 ** -6 * s_el
+    assert np.all(np.abs(deq - W64)[normal] <= 2.0 ** -4 * np.abs(W64)[normal] * (1 + 1e-6))
+    assert np.all(np.abs(deq - W64)[~normal] <= 2.0 ** -10 * s_el[~normal] * (1 + 1e-6))
+
+
+def test_mx_blocks_run_along_the_contraction_dimension():
+    X = _gauss((5, 128), 12)
+    c1, s1 = f8.quantize_mx(X)
+    X2 = X.copy()
+    X2[2, 40] = 100.0                                 # block (row 2, features 32..63)
+    c2, s2 = f8.quantize_mx(X2)
+    diff = s1 != s2
+    assert diff.sum() == 1 and diff[2, 1]
+
+
+def test_mx_layer_equals_bf16_layer_when_quantisation_is_exact():
+    T, d, I, N, Z, K = 20, 128, 128, 3, 2, 2
+    xv = _on_grid((T, d), 13, -8, f8.MX_BLOCK)
+    x = torch.from_numpy(xv).to(torch.bfloat16)
+    assert np.array_equal(x.float().numpy(), xv)
+    Wg = [_on_grid((I, d), 14 + e, -12, f8.MX_BLOCK) for e in range(N)]
+    Wu = [_on_grid((I, d), 24 + e, -12, f8.MX_BLOCK) for e in range(N)]
+    Wd = [_gauss((d, I), 34 + e, 0.02) for e in range(N)]
+    g = torch.Generator().manual_seed(9)
+    W_r = (torch.randn(N + Z, d, generator=g) * 0.05).to(torch.bfloat16)
+    r = ref.route(x, W_r, torch.zeros(N + Z), N, K)
+    assert (r.idx < N).any()
+    q = {e: (f8.quantize_mx(Wg[e]), f8.quantize_mx(Wu[e]), Wd[e]) for e in range(N)}
+    assert all(np.all(q[e][0][1] == np.float32(2.0 ** -12)) for e in range(N))
+    out8 = f8.forward_rows_fp8(x, r, lambda e: q[e], mx=True)
+    out = ref.forward_rows(x, r, lambda e: (Wg[e], Wu[e], Wd[e]))
+    assert np.allclose(out8, out, rtol=1e-12, atol=1e-15)
+
+
+def _mx_scale_floor(W):
+    """Mutant: the OCP-style floor exponent, 2^(floor(log2 amax) - 8), which
+    lets the largest elements saturate."""
+    W = np.asarray(W, dtype=np.float32)
+    codes, scales = _orig_mx(W)
+    R, C = W.shape
+    for j in range(scales.shape[1]):
+        blk = W[:, 32 * j:32 * (j + 1)]
+        amax = np.abs(blk).max(axis=1).astype(np.float64)
+        s = np.where(amax > 0, np.ldexp(1.0, (np.floor(np.log2(np.maximum(amax, 1e-300))) - 8)
+                                        .astype(int)), 1.0)
+        scales[:, j] = s
+        codes[:, 32 * j:32 * (j + 1)] = f8.e4m3_encode(blk / s[:, None].astype(np.float32))
+    return codes, scales
+
+
+_orig_mx = f8.quantize_mx
+_MX_PINS = [test_mx_scales_are_the_smallest_powers_of_two_without_saturation,
+            test_mx_blocks_run_along_the_contraction_dimension,
+            test_mx_layer_equals_bf16_layer_when_quantisation_is_exact]
+
+
+@pytest.mark.parametrize("name,attr,val", [
+    ("floor exponent (saturating)", "quantize_mx", _mx_scale_floor),
+    ("blocks of 32 rows", "MX_BLOCK", (32, 1)),
+])
+def test_mx_mutant_is_caught(name, attr, val, monkeypatch):
+    if attr == "MX_BLOCK":
+        def by_rows(W):
+            c, s = _orig_mx(np.asarray(W, np.float32).T)
+            return c.T.copy(), s.T.copy()
+        monkeypatch.setattr(f8, "quantize_mx", by_rows)
+    monkeypatch.setattr(f8, attr, val)
+    caught = []
+    for pin in _MX_PINS:
+        try:
+            pin()
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches: {name}"
