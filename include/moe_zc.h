@@ -80,7 +80,12 @@ typedef enum moe_zc_status {
  * Batches of 1024 tokens or more leave a copy of their expert-load histogram
  * in pinned host memory (asynchronously); a later forward on the device uses
  * it to choose how the expert GEMMs are launched.  That choice changes speed
- * only: every launch gives the same bits.
+ * only: every launch gives the same bits.  Batches of at most 64 tokens run
+ * both expert GEMMs in one grid of at most one block per multiprocessor,
+ * whose down-projection tiles wait (bounded, like every device wait) for
+ * other blocks' gate/up results: should other work hold multiprocessors
+ * for longer than the wait bound (2 s), the call reports
+ * MOE_ZC_ERR_TIMEOUT instead of hanging.
  */
 int moe_zc_forward(const void* x, const void* W_r, const float* b,
                    const void* W_gate, const void* W_up, const void* W_down,
