@@ -186,6 +186,29 @@ int moe_zc_bias_controller_init(const float* b, int32_t E, float* state);
 int moe_zc_bias_controller_step(const int32_t* counts, int32_t N, int32_t Z, int64_t tokens,
                                 int32_t K, const moe_zc_pid* pid, float* state, float* b);
 
+/*
+ * FP8 (E4M3) block quantisation of one weight matrix, on the host (write-up,
+ * section "System-level optimisation": fine-grained block quantisation as in
+ * DeepSeek-V3).  For an FP8 expert path: moe_zc_forward itself still takes
+ * bf16 weights.
+ *   W       host bf16 [rows, cols], row-major (e.g. W_gate[e], [I, d])
+ *   mode    MOE_ZC_FP8_BLOCK128: 128 x 128 blocks, scale = amax / 448 in fp32;
+ *           MOE_ZC_FP8_MX32: 1 x 32 blocks along a row, scale = the smallest
+ *           power of two with amax / scale <= 448
+ *   codes   host uint8 [rows, cols]: E4M3 codes of W / scale (division in
+ *           fp32), nearest value, ties to the even code, saturating at 448;
+ *           E4M3 = sign, 4 exponent bits (bias 7), 3 mantissa bits, no
+ *           infinities, 0x7F / 0xFF NaN
+ *   scales  host float [ceil(rows/br), ceil(cols/bc)] for br x bc blocks
+ * A block of zeros, or holding a NaN or an infinity, gets scale 1.  Element (r, c)
+ * stands for decode(codes[r, c]) * scales[r / br, c / bc].
+ * Returns MOE_ZC_ERR_INVALID_ARG for null pointers, rows or cols < 1, or an
+ * unknown mode.
+ */
+enum { MOE_ZC_FP8_BLOCK128 = 0, MOE_ZC_FP8_MX32 = 1 };
+int moe_zc_fp8_quantize(const void* W, int64_t rows, int64_t cols, int32_t mode,
+                        uint8_t* codes, float* scales);
+
 /* Wait for the last forward; report (and clear) a device-side timeout. */
 int moe_zc_synchronize(void);
 

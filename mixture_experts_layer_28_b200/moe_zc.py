@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.moe_zc_bias_controller_step.restype = ctypes.c_int
         L.moe_zc_test_inject.argtypes = [i32, i64]
         L.moe_zc_test_inject.restype = None
+        L.moe_zc_fp8_quantize.argtypes = [vp, i64, i64, i32, vp, vp]
+        L.moe_zc_fp8_quantize.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -273,6 +275,25 @@ class BiasController:
                                                  self.b.ctypes.data),
                "moe_zc_bias_controller_step")
         return self.b.copy()
+
+
+FP8_BLOCK128 = 0   # 128 x 128 blocks, fp32 scale amax / 448
+FP8_MX32 = 1       # 1 x 32 blocks along a row, power-of-two scales
+
+
+def fp8_quantize(W: torch.Tensor, mode: int = FP8_BLOCK128):
+    """E4M3 codes (numpy uint8 [rows, cols]) and block scales (numpy float32)
+    of a host bf16 matrix (moe_zc_fp8_quantize)."""
+    if W.device.type != "cpu" or W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise ValueError("W must be a 2-D bf16 CPU tensor")
+    W = W.contiguous()
+    rows, cols = W.shape
+    br, bc = (128, 128) if mode == FP8_BLOCK128 else (1, 32)
+    codes = np.zeros((rows, cols), dtype=np.uint8)
+    scales = np.zeros(((rows + br - 1) // br, (cols + bc - 1) // bc), dtype=np.float32)
+    _check(lib().moe_zc_fp8_quantize(W.data_ptr(), rows, cols, mode, codes.ctypes.data,
+                                     scales.ctypes.data), "moe_zc_fp8_quantize")
+    return codes, scales
 
 
 def allreduce_expert_load(counts: np.ndarray, group=None) -> np.ndarray:

@@ -22,7 +22,7 @@ readings are taken (each one is a test):
   Q3  activations are cut into 1 x 128 tiles (one token, 128 consecutive
       features), each with one fp32 scale;
   Q4  a block's scale is amax / 448 (amax = its largest magnitude); an
-      all-zero block gets scale 1;
+      all-zero block, or one holding a NaN or an infinity, gets scale 1;
   Q5  encoding rounds to the nearest E4M3 value, ties to the even code, and
       saturates at +-448;
   Q6  the scale and the scaled value w / scale are formed in fp32 (IEEE
@@ -39,7 +39,7 @@ A second reading, for the tensor cores' block-scaled FP8 form, replaces Q2-Q4
       contraction dimension (one weight row or one token, 32 consecutive
       features), each with one power-of-two scale (an 8-bit exponent);
   M2  the scale is the smallest power of two with amax / scale <= 448, so no
-      element saturates; an all-zero block gets scale 1.
+      element saturates; an all-zero or non-finite block gets scale 1.
 Q1, Q5-Q7 hold for it unchanged (dividing by a power of two is exact).
 """
 from __future__ import annotations
@@ -107,7 +107,8 @@ def quantize_blocks(W, block: Tuple[int, int]) -> Tuple[np.ndarray, np.ndarray]:
         for j in range(nc):
             blk = W[i * br:(i + 1) * br, j * bc:(j + 1) * bc]
             amax = np.float32(np.max(np.abs(blk))) if blk.size else np.float32(0)
-            s = np.float32(amax / np.float32(E4M3_MAX)) if amax > 0 else np.float32(1.0)
+            ok = amax > 0 and np.isfinite(amax)     # NaN or infinity: scale 1
+            s = np.float32(amax / np.float32(E4M3_MAX)) if ok else np.float32(1.0)
             scales[i, j] = s
             codes[i * br:(i + 1) * br, j * bc:(j + 1) * bc] = e4m3_encode(blk / s)
     return codes, scales
@@ -133,10 +134,14 @@ def quantize_mx(W) -> Tuple[np.ndarray, np.ndarray]:
         blk = W[:, j * MX_BLOCK[1]:(j + 1) * MX_BLOCK[1]]
         amax = np.max(np.abs(blk), axis=1).astype(np.float64)
         e = np.zeros(R)
-        nz = amax > 0
+        nz = (amax > 0) & np.isfinite(amax)          # NaN or infinity: scale 1
+        amax = np.where(nz, amax, 0.0)
         e[nz] = np.ceil(np.log2(amax[nz] / E4M3_MAX))
-        # guard the log2 rounding: the smallest power of two with amax / s <= 448
+        # guard the log2 rounding both ways: the smallest power of two with
+        # amax / s <= 448 (divisions by powers of two are exact)
         s = np.ldexp(1.0, e.astype(int))
+        higher = nz & (amax / s > E4M3_MAX)
+        s[higher] *= 2
         lower = nz & (amax / (s / 2) <= E4M3_MAX)
         s[lower] /= 2
         s[~nz] = 1.0
