@@ -20,6 +20,7 @@ import sys
 import numpy as np
 
 from mixture_experts_layer_28_b200 import workloads as wl
+from oracle import moe_zc_ref
 from oracle.moe_zc_ref import router_logits, softmax, _f64
 
 OUT = os.path.join(os.path.dirname(wl.__file__), "bias_shift.json")
@@ -27,15 +28,17 @@ TOL = 0.005
 
 
 def zero_share(p: np.ndarray, b0: np.ndarray, N: int, K: int, delta: float) -> float:
-    """Share of picks on zero experts when the zero experts' bias is shifted."""
+    """Share of all T*K picks that land on zero experts when every zero
+    expert's bias is shifted by delta.
+
+    The picks are the oracle's own: the top-K of s = p + b (bias added after
+    the softmax, equal scores to the lower index, so an FFN expert wins a tie
+    against a zero expert), counted with zero_pick_fraction.
+    """
     s = p + b0[None, :]
     s[:, N:] += delta
-    T, E = s.shape
-    if K >= E:
-        return (E - N) / E
-    kth = -np.partition(-s, K - 1, axis=1)[:, K - 1]
-    zero_picks = (s[:, N:] >= kth[:, None]).sum()
-    return float(zero_picks) / (T * K)
+    idx, _ = moe_zc_ref.select_topk(s, K)
+    return moe_zc_ref.zero_pick_fraction(idx, N)
 
 
 def calibrate(w: wl.Workload) -> float:

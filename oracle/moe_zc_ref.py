@@ -164,6 +164,11 @@ def expert_load(idx: np.ndarray, E: int) -> np.ndarray:
 
 
 def zero_pick_fraction(idx: np.ndarray, N: int) -> float:
-    """Share of all T*K picks that land on zero experts."""
+    """Share of all T*K picks that land on zero experts (indices N..E-1, R5).
+
+    Section "Zero-computation experts": a token's picks split between FFN
+    experts and zero experts, so the number of FFN experts it runs varies;
+    this is the share of the pool's picks the zero experts take.
+    """
     idx = np.asarray(idx)
     return float((idx >= N).sum()) / max(idx.size, 1)

@@ -266,6 +266,58 @@ def pin_zero_expert_is_identity(ref):
     np.testing.assert_allclose(out, want.numpy(), rtol=1e-12, atol=1e-13)
 
 
+def pin_zero_pick_fraction(ref):
+    """Share of picks on zero experts, counted by hand on small index arrays.
+
+    Experts N..E-1 are the zero experts (reading R5), so index N counts as a
+    zero pick and index N-1 does not.
+    """
+    N = 3
+    cases = [
+        ([[0, 3], [3, 4], [2, 1]], 3 / 6),    # 3 (== N) and 4 are zero experts
+        ([[2, 1, 0]], 0.0),                   # 2 (== N - 1) is the last FFN expert
+        ([[5, 4, 3]], 1.0),
+        ([[3], [2], [3], [2]], 2 / 4),
+        ([[4, 0, 1, 2], [0, 1, 2, 3]], 2 / 8),
+    ]
+    for idx, want in cases:
+        got = ref.zero_pick_fraction(np.array(idx), N)
+        assert got == want, (idx, got, want)
+    # a routing whose every pick is a zero expert, and one with no zero experts
+    L = _layer(14, T=12, d=4, N=N, Z=4, I=3)
+    r = ref.route(L["x"], L["W_r"], np.concatenate([np.zeros(N), np.full(4, 10.0)]), N, 2)
+    assert ref.zero_pick_fraction(r.idx, N) == 1.0
+    r = ref.route(L["x"], L["W_r"], np.concatenate([np.full(N, 10.0), np.zeros(4)]), N, 2)
+    assert ref.zero_pick_fraction(r.idx, N) == 0.0
+
+
+def pin_zero_share_ties(ref):
+    """The calibration's zero-expert share on score tables solved by hand.
+
+    N = 2 FFN experts, Z = 2 zero experts, scores in sixteenths (exact in
+    binary).  Row 0 scores every expert alike, row 1 is [6, 1, 5, 4]; the
+    shift delta is added to the zero experts (2 and 3).  Equal scores go to
+    the lower index (reading R6), so an FFN expert beats a zero expert it
+    ties with.  For example K = 1, delta = 1/16: row 0 picks expert 2 (zero),
+    row 1 has s = [6, 1, 6, 5] and picks expert 0 (tie, lower index): 1/2.
+    """
+    from oracle import calibrate_bias_shift as cal
+    p = np.array([[4.0, 4.0, 4.0, 4.0], [6.0, 1.0, 5.0, 4.0]]) / 16.0
+    b0 = np.zeros(4)
+    cases = [
+        (1, 0.0, 0 / 2),     # row 0: four-way tie -> expert 0; row 1 -> expert 0
+        (1, 1.0, 1 / 2),     # row 0 -> 2; row 1: tie 0 vs 2 -> 0
+        (2, 1.0, 3 / 4),     # row 0 -> {2, 3}; row 1 -> {0, 2}
+        (2, 2.0, 3 / 4),     # row 1: s = [6, 1, 7, 6] -> 2, then tie 0 vs 3 -> 0
+        (3, 2.0, 4 / 6),     # row 1 -> {2, 0, 3}; row 0 -> {2, 3, 0}
+        (2, -1.0, 1 / 4),    # row 0: s = [4, 4, 3, 3] -> {0, 1}; row 1 -> {0, 2}
+        (4, -3.0, 2 / 4),    # K = E: every expert is picked whatever the shift
+    ]
+    for K, shift16, want in cases:
+        got = cal.zero_share(p.copy(), b0, 2, K, shift16 / 16.0)
+        assert got == want, (K, shift16, got, want)
+
+
 ALL_PINS = [
     pin_worked_examples,
     pin_topk_brute_force,
@@ -278,4 +330,6 @@ ALL_PINS = [
     pin_logit_offset,
     pin_invariants,
     pin_zero_expert_is_identity,
+    pin_zero_pick_fraction,
+    pin_zero_share_ties,
 ]

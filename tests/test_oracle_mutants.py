@@ -3,18 +3,22 @@
 Every mutant below breaks one reading of the LongCat-Flash write-up's
 "Zero-computation experts" section (softmax over all experts, bias for
 selection only, unbiased gates, identity zero experts, SwiGLU experts,
-lower-index ties, histogram over all experts).  A mutant that no pin catches
+lower-index ties, histogram over all experts, zero experts at indices
+N..E-1), or of the helpers that measure and calibrate the zero-expert share
+of the picks (the workloads' "b set so ~X% of picks are zero experts").  A mutant that no pin catches
 would mean the oracle could carry that mistake unnoticed.
 """
 import numpy as np
 import pytest
 
+from oracle import calibrate_bias_shift as cal
 from oracle import moe_zc_ref as ref
 from oracle_pins import ALL_PINS
 
 _orig = {k: getattr(ref, k) for k in ("softmax", "select_topk", "route", "silu",
                                       "swiglu_expert", "forward_rows", "expert_load",
-                                      "router_logits")}
+                                      "router_logits", "zero_pick_fraction")}
+_orig_cal = {"zero_share": cal.zero_share}
 
 
 def _route_bias_before_softmax(x, W_r, b, N, K, logit_offset=None):
@@ -102,6 +106,42 @@ def _logits_offset_negated(x, W_r, logit_offset=None):
     return l
 
 
+def _zero_fraction_strict(idx, N):
+    idx = np.asarray(idx)
+    return float((idx > N).sum()) / max(idx.size, 1)
+
+
+def _zero_fraction_counts_last_ffn(idx, N):
+    idx = np.asarray(idx)
+    return float((idx >= N - 1).sum()) / max(idx.size, 1)
+
+
+def _zero_share_ties_to_zero(p, b0, N, K, delta):
+    # every zero expert scoring at least the K-th score counts, so a tie at
+    # the selection boundary goes to the zero expert (and can exceed K picks)
+    s = p + b0[None, :]
+    s[:, N:] += delta
+    T, E = s.shape
+    if K >= E:
+        return (E - N) / E
+    kth = -np.partition(-s, K - 1, axis=1)[:, K - 1]
+    return float((s[:, N:] >= kth[:, None]).sum()) / (T * K)
+
+
+def _zero_share_shifts_ffn(p, b0, N, K, delta):
+    s = p + b0[None, :]
+    s[:, :N] += delta
+    idx, _ = ref.select_topk(s, K)
+    return ref.zero_pick_fraction(idx, N)
+
+
+def _zero_share_strict_boundary(p, b0, N, K, delta):
+    s = p + b0[None, :]
+    s[:, N:] += delta
+    idx, _ = ref.select_topk(s, K)
+    return float((idx > N).sum()) / idx.size
+
+
 MUTANTS = {
     "bias_before_softmax": ("route", _route_bias_before_softmax),
     "renormalised_gates": ("route", _route_renormalised),
@@ -118,13 +158,21 @@ MUTANTS = {
     "zero_expert_wrong_gate": ("forward_rows", _forward_rows_zero_is_zero_gate),
     "load_drops_last_zero_expert": ("expert_load", _load_drops_last_expert),
     "offset_sign_flipped": ("router_logits", _logits_offset_negated),
+    "zero_fraction_misses_expert_N": ("zero_pick_fraction", _zero_fraction_strict),
+    "zero_fraction_counts_last_ffn": ("zero_pick_fraction", _zero_fraction_counts_last_ffn),
+    "zero_share_ties_to_zero_expert": ("cal.zero_share", _zero_share_ties_to_zero),
+    "zero_share_shifts_ffn_bias": ("cal.zero_share", _zero_share_shifts_ffn),
+    "zero_share_misses_expert_N": ("cal.zero_share", _zero_share_strict_boundary),
 }
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_mutant_is_caught(name, monkeypatch):
     attr, fn = MUTANTS[name]
-    monkeypatch.setattr(ref, attr, fn)
+    if attr.startswith("cal."):
+        monkeypatch.setattr(cal, attr[4:], fn)
+    else:
+        monkeypatch.setattr(ref, attr, fn)
     caught = []
     for pin in ALL_PINS:
         try:
