@@ -145,7 +145,6 @@ struct GemmParams {
                           // slice s writes its partial sums to out + s * split_stride
   long long split_stride;
   int single_a;           // MODE_ROUTER/MODE_DOWN: 1 = one 128-row A block per tile (no pair)
-  int mgroup;             // pair kernel: weight blocks per tile group (divides mblocks; 0 = all)
   int l2_stream;          // 1: weight and token tiles loaded, and outputs stored, with an
                           // L2 evict-first policy (decode: every weight byte is read once)
   int b_box_full;         // 1: a full token tile's B rows come in one GEMM_BN-row copy
@@ -184,22 +183,6 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
 cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, const CUtensorMap& xp,
                               const CUtensorMap& wd, const CUtensorMap& h, const GemmParams& pg,
                               const GemmParams& pd, int grid, cudaStream_t stream);
-
-// The FFN expert GEMMs on CTA pairs (cta_group::2, M = 256 per MMA), for
-// batches with many tokens per expert; `clusters` pairs are launched.
-//   gate/up: a0 = W_gate [N*I, d] and a1 = W_up with 64-row boxes; mblocks = I/128
-//   down:    a0 = a1 = W_down [N*d, I] with 128-row boxes; mblocks = d/256
-//   b: tokens with 32-row boxes, as for launch_gemm
-constexpr int PAIR_EPI_WARPS = 8;           // two per TMEM lane quadrant
-constexpr int PAIR_THREADS = 128 + PAIR_EPI_WARPS * 32;
-constexpr int PAIR_STAGES = 6;
-constexpr int PAIR_A_BYTES = GEMM_BM * GEMM_BK * 2;          // 128 weight rows per CTA
-constexpr int PAIR_STAGE_BYTES = PAIR_A_BYTES + 128 * GEMM_BK * 2;   // + 128 tokens per CTA
-constexpr int PAIR_XCHG_BYTES = 2 * 4096;                     // gate/up swap, reused for staging
-constexpr int PAIR_SMEM_BYTES = PAIR_STAGES * PAIR_STAGE_BYTES + 4 * PAIR_XCHG_BYTES + 1024;
-cudaError_t launch_gemm_pair(GemmMode mode, const CUtensorMap& a0, const CUtensorMap& a1,
-                             const CUtensorMap& b, const GemmParams& p, int clusters,
-                             cudaStream_t stream);
 
 // ------------------------------------------------------------------ router
 // softmax over E logits (+offset), + bias, top-K, zero-gate sums, histogram.

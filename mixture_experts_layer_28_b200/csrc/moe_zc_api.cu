@@ -23,7 +23,6 @@
 #include <cudaTypedefs.h>
 
 #include <cstdint>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -204,30 +203,6 @@ RouterPlan router_plan(int64_t T, int E, int ksteps, int sms) {
     rp.splits = s < 1 ? 1 : static_cast<int>(s);
   }
   return rp;
-}
-
-// Weight blocks per tile group of the pair kernel: the largest divisor of
-// mblocks not above MOE_ZC_PAIR_MGROUP (default: half of mblocks).
-int pair_mgroup(int mblocks) {
-  int want = mblocks / 2 > 0 ? mblocks / 2 : 1;
-  const char* env = getenv("MOE_ZC_PAIR_MGROUP");
-  if (env && atoi(env) > 0) want = atoi(env);
-  for (int g = want < mblocks ? want : mblocks; g >= 1; --g)
-    if (mblocks % g == 0) return g;
-  return 1;
-}
-
-// Expert GEMMs on CTA pairs only when MOE_ZC_GEMM_PAIR=1 (and the down
-// projection's 256-row blocks tile d).  Measured at the prefill workload the
-// single-SM engine is faster (gate/up 5.3 vs 6.6 ms, down 2.8 vs 3.3 ms): the
-// pair's MMA waits on operands ~37% of the time even with a six-deep ring and
-// grouped tile order, so the single-SM kernels are the default.
-bool use_pair_gemm(int64_t T, int K, int d) {
-  (void)T;
-  (void)K;
-  if (d % (2 * GEMM_BM) != 0) return false;
-  const char* env = getenv("MOE_ZC_GEMM_PAIR");
-  return env && env[0] == '1';
 }
 
 int reserve_impl(Ctx& c, int64_t T, int d, int N, int Z, int K, int I) {
@@ -439,45 +414,6 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
                         static_cast<__nv_bfloat16*>(c.Xp.p), st));
       rec.mark(4);
       const int64_t tiles_ub = (T * K + GEMM_BN - 1) / GEMM_BN + N;
-      if (use_pair_gemm(T, K, d)) {
-        // 5-6 on CTA pairs
-        CUtensorMap mWg, mWu, mXp, mWd, mH;
-        if (!make_map(&mWg, W_gate, static_cast<uint64_t>(N) * I, d, 64) ||
-            !make_map(&mWu, W_up, static_cast<uint64_t>(N) * I, d, 64) ||
-            !make_map(&mXp, c.Xp.p, c.rows_cap, d, GEMM_B_BOX_ROWS) ||
-            !make_map(&mWd, W_down, static_cast<uint64_t>(N) * d, I, GEMM_BM) ||
-            !make_map(&mH, c.H.p, c.rows_cap, I, GEMM_B_BOX_ROWS))
-          return MOE_ZC_ERR_CUDA;
-        GemmParams pg{};
-        pg.grp_count = cnt;
-        pg.grp_off = grp_off;
-        pg.grp_ttp = grp_ttp;
-        pg.G = N;
-        pg.ksteps = d / GEMM_BK;
-        pg.mblocks = I / GEMM_BM;
-        pg.a_rows = I;
-        pg.out = c.H.p;
-        pg.out_ld = I;
-        pg.err = err;
-        pg.wait_ns = wait_ns;
-        const int64_t pairs_max = c.sms / 2;
-        pg.mgroup = pair_mgroup(pg.mblocks);
-        const int64_t g_ub = tiles_ub * pg.mblocks;
-        CK(launch_gemm_pair(MODE_GATEUP, mWg, mWu, mXp, pg,
-                            static_cast<int>(g_ub < pairs_max ? g_ub : pairs_max), st));
-        rec.mark(5);
-        GemmParams pd = pg;
-        pd.ksteps = I / GEMM_BK;
-        pd.mblocks = d / (2 * GEMM_BM);
-        pd.a_rows = d;
-        pd.out = c.Y.p;
-        pd.out_ld = d;
-        pd.mgroup = pair_mgroup(pd.mblocks);
-        const int64_t d_ub = tiles_ub * pd.mblocks;
-        CK(launch_gemm_pair(MODE_DOWN, mWd, mWd, mH, pd,
-                            static_cast<int>(d_ub < pairs_max ? d_ub : pairs_max), st));
-        rec.mark(6);
-      } else {
       // 5  gate/up GEMM
       CUtensorMap mWg, mWu, mXp;
       if (!make_map(&mWg, W_gate, static_cast<uint64_t>(N) * I, d, GEMM_BM) ||
@@ -546,7 +482,6 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
         CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd,
                        static_cast<int>(d_ub < c.sms ? d_ub : c.sms), st));
         rec.mark(6);
-      }
       }
     } else {
       CK(launch_assign_slots(cnt, idx, T * K, N, grp_off, grp_ttp, fill, slot, st));
