@@ -19,7 +19,11 @@ steps.  With N > 1 GPUs each rank runs its own batch of T tokens against its
 own weight replica (tokens are independent: no collective in the step), so
 `value` is N*T*K / max-rank time ("weak" scaling).
 
-The JSON line also carries: `e2e` (the same metric through moe_zc_forward_host: the
+The JSON line also carries `workloads`: the decode, small and skewed40
+workloads (--workloads), each timed the same way in the same run, with its own
+ms_per_step, tokens/s, e2e, roofline, layer_roofline and clocks (each timed
+region lasts at least about a second, so the clocks are sampled inside it).
+Also: `e2e` (the same metric through moe_zc_forward_host: the
 step's input is copied from pinned host memory and its output back inside the
 timed region, in chunks whose copies overlap the kernels), `roofline` (the dominant kernel's achieved rate against the measured
 peak in MEASURED_PEAKS.json, from per-stage CUDA events recorded on the
@@ -54,25 +58,37 @@ from mixture_experts_layer_28_b200 import workloads as wl  # noqa: E402
 METRIC = "MoE-layer tokens/s; executed-FFN TFLOPS as % of B200 bf16 peak (HBM % at decode)"
 UNIT = "tokens/s"
 L2_BYTES = 126 * 2 ** 20
-KERNELS_PER_FORWARD = 7   # router_gemm, route, assign, permute, gateup, down, combine
-SMALL_BATCH = 64          # batches of at most this many tokens run gate/up and down as one kernel
 
 
-def kernels_per_forward(w):
-    if w.N == 0:
-        return 4          # router_gemm, route, assign, combine
-    return KERNELS_PER_FORWARD - 1 if w.T <= SMALL_BATCH else KERNELS_PER_FORWARD
+def kernels_per_forward(w, sms=148):
+    """Kernels one forward launches (the library's own launch plan)."""
+    from mixture_experts_layer_28_b200 import moe_zc as mz
+    return mz.plan(w.T, w.d, w.N, w.Z, w.K, w.I, sms=sms, resident_blocks=sms)["kernels"]
 
-# dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel
-# from an ncu capture of the current kernel build at the full workload (one
-# pass; mean over the captured launches; the full-size GEMM traffic summary
-# under profiles/), per workload.
-# Clear an entry when that kernel changes.
-NCU_TRAFFIC_BYTES = {
-    "prefill": 8_885_600_000 + 558_700_000,    # gate/up GEMM
-    "decode": 2_278_000_000 + 5_900_000,       # gate/up + down GEMMs in one kernel
-    "prefill_balanced": 30_013_700_000 + 565_300_000,   # gate/up GEMM, paired tiles
+
+# DRAM traffic of the dominant kernel: dram__bytes_read.sum +
+# dram__bytes_write.sum of one launch over that launch's algorithmic bytes,
+# from an ncu capture of a small case of the same kernel (the GEMM summaries
+# under profiles/ give the command), with the sha256 (first 16 hex digits) of
+# the GEMM engine's sources at the capture.  `traffic` = ratio x the
+# algorithmic bytes of this run's launch (traffic scales with the units a
+# launch processes); null when the sources have changed since the capture.
+GEMM_SOURCES = ["gemm_tcgen05.cu", "ptx.cuh", "epilogue.cuh", "kernels.cuh"]
+NCU_TRAFFIC_RATIO = {
+    # workload: (dominant kernel, DRAM bytes / algorithmic bytes, sources sha16, case)
 }
+SUSTAINED_REGION_S = 2.0   # timed regions at least this long use the sustained bf16 peak
+NOMINAL_HBM_GBS = 7700.0   # B200 HBM3e, HGX figure (context beside the measured copy peak)
+EXTRA_WORKLOADS = "decode,small,skewed40"
+
+
+def gemm_sources_sha16():
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "mixture_experts_layer_28_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def parse():
@@ -90,6 +106,9 @@ def parse():
                     help="time replays of one forward captured into a CUDA graph")
     ap.add_argument("--shape", default="",
                     help="override workload sizes, e.g. T=4096,N=32,Z=16 (for profiling runs)")
+    ap.add_argument("--workloads", default=EXTRA_WORKLOADS,
+                    help="comma-separated workloads also timed in the same run and reported "
+                         "under `workloads` ('none': only the headline)")
     return ap.parse_args()
 
 
@@ -155,7 +174,10 @@ class Dist:
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples (every 100 ms, each with its own timestamp) of SM
+    clocks and throttle reasons; summary() keeps the samples taken inside
+    the timed region [t0, t1] (host wall clock)."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -182,31 +204,48 @@ class ClockSampler:
 
     def stop(self):
         if not self.proc:
-            return None
+            return
+        time.sleep(0.3)   # the sample covering the region's end
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.thread.join(timeout=2)
-        sm, mx, reasons = [], None, set()
+
+    @staticmethod
+    def _stamp(text):
+        import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(text, fmt).timestamp()
+            except ValueError:
+                pass
+        return None
+
+    def summary(self, t0=None, t1=None):
+        sm, mx, reasons, n_all = [], None, set(), 0
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
+                continue
+            n_all += 1
+            ts = self._stamp(parts[0])
+            if t0 is not None and ts is not None and not (t0 - 0.1 <= ts <= t1 + 0.1):
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                sm.append(float(parts[2]))
+                mx = float(parts[3])
             except ValueError:
                 continue
-            for nm, v in zip(names, parts[5:9]):
+            for nm, v in zip(names, parts[6:10]):
                 if v.lower().startswith("active"):
                     reasons.add(nm)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "samples_outside_region": n_all - len(sm)}
 
 
 # ----------------------------------------------------------------- inputs
@@ -287,13 +326,83 @@ def config_of(w, extra=None):
     return c
 
 
-def run_ours(args, dist, w):
+def bf16_peak(pk, region_s):
+    """The bf16 peak a kernel timed inside a region of region_s seconds is held
+    to: the burst figure for a short region, the sustained one (seconds of
+    back-to-back GEMMs under the power cap) for a long one."""
+    if region_s >= SUSTAINED_REGION_S:
+        return pk["bf16_sus"], f"bf16 dense, sustained ({pk['src']}, MEASURED_PEAKS.json)"
+    return pk["bf16"], f"bf16 dense, burst ({pk['src']}, MEASURED_PEAKS.json)"
+
+
+def kernel_roofline(w, rf, plan, per, pk, region_s):
+    """The dominant stage's achieved rate against its bound."""
+    dom = max(per, key=per.get)
+    # (with the one-grid expert GEMMs the gate/up stage is the kernel that
+    # runs both)
+    one_grid = bool(plan["expert_gemms_one_grid"])
+    kern = {"gateup_gemm": ((rf["F_gateup"] + rf["F_down"], rf["B_gateup"] + rf["B_down"])
+                            if one_grid else (rf["F_gateup"], rf["B_gateup"])),
+            "down_gemm": (rf["F_down"], rf["B_down"])}.get(dom)
+    if not kern or per[dom] <= 0:
+        return None
+    F, B = kern
+    sec = per[dom] / 1e3
+    peak, kind = bf16_peak(pk, region_s)
+    t_tensor, t_hbm = F / (peak * 1e12), B / (pk["hbm"] * 1e9)
+    if t_tensor >= t_hbm:
+        ach = F / sec / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "peak_kind": kind,
+                "frac_of_sustained_peak": ach / pk["bf16_sus"]}
+    else:
+        ach = B / sec / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": ach / pk["hbm"],
+                "peak_kind": f"HBM copy, read + write ({pk['src']}, MEASURED_PEAKS.json)",
+                "frac_of_nominal_hbm": ach / NOMINAL_HBM_GBS}
+    roof["kernel"] = "gateup_down_gemm (one kernel)" if one_grid and dom == "gateup_gemm" else dom
+    roof["ms_per_launch"] = per[dom]
+    roof["algorithmic_bytes"] = B
+    roof["algorithmic_flops"] = F
+    tr = NCU_TRAFFIC_RATIO.get(w.name)
+    roof["traffic"] = None
+    if tr and tr[0] == roof["kernel"] and tr[2] == gemm_sources_sha16():
+        roof["traffic"] = tr[1] * B
+        roof["traffic_source"] = f"ncu DRAM bytes / algorithmic bytes = {tr[1]:.3f} on {tr[3]}"
+    return roof
+
+
+def layer_roofline(rf, pk, ms, region_s):
+    """The whole layer: the slower of executed FFN FLOPs at the bf16 peak and
+    the bytes it must touch at the HBM peak, against the measured step."""
+    peak, kind = bf16_peak(pk, region_s)
+    t_f, t_b = rf["F_layer"] / (peak * 1e12), rf["B_layer"] / (pk["hbm"] * 1e9)
+    sec = ms / 1e3
+    ffn_tflops = rf["F_layer"] / sec / 1e12
+    hbm_gbs = rf["B_layer"] / sec / 1e9
+    return {"bound": "tensor" if t_f >= t_b else "hbm", "roofline_ms": max(t_f, t_b) * 1e3,
+            "frac": max(t_f, t_b) / sec, "bf16_peak_kind": kind,
+            "frac_vs_sustained_bf16": max(rf["F_layer"] / (pk["bf16_sus"] * 1e12), t_b) / sec,
+            "executed_ffn_tflops": ffn_tflops,
+            "pct_of_bf16_peak_burst": 100.0 * ffn_tflops / pk["bf16"],
+            "pct_of_bf16_peak_sustained": 100.0 * ffn_tflops / pk["bf16_sus"],
+            "hbm_gbs": hbm_gbs, "pct_of_hbm": 100.0 * hbm_gbs / pk["hbm"],
+            "pct_of_nominal_hbm": 100.0 * hbm_gbs / NOMINAL_HBM_GBS}
+
+
+def measure(args, dist, w, steps, e2e_steps, headline):
+    """Time `steps` forwards of workload w (device-resident inputs), then the
+    same with per-stage events, then e2e through the host-buffer entry point.
+    steps <= 0: as many as fill about one second (at least 20)."""
     from mixture_experts_layer_28_b200 import moe_zc as mz
     pk = peaks()
     ri, b, ew, dev = make_inputs(w)
     out = torch.empty_like(dev["x"])
     stream = torch.cuda.current_stream()
     mz.reserve(w.T, w.d, w.N, w.Z, w.K, w.I)
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    plan = mz.plan(w.T, w.d, w.N, w.Z, w.K, w.I, sms=sms, resident_blocks=sms)
 
     def step(x=None, o=None):
         mz.forward(dev["x"] if x is None else x, dev["W_r"], dev["b"], ew.W_gate, ew.W_up,
@@ -306,11 +415,20 @@ def run_ours(args, dist, w):
     mz.synchronize()
     st = routing_stats(w, mz.expert_load(w.E))
     rf = roofline_numbers(w, st, pk)
+    if steps <= 0:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(5):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        steps = max(20, int(1.0 / max(e0.elapsed_time(e1) / 5 / 1e3, 1e-6)))
+        steps = int(dist.max(float(steps)))   # every rank the same count
 
     # --graph: the forward captured once into a CUDA graph (its launches on
     # the capture stream), each timed step one replay
     graph = None
-    if args.graph:
+    if args.graph and headline:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             mz.forward(dev["x"], dev["W_r"], dev["b"], ew.W_gate, ew.W_up, ew.W_down,
@@ -333,16 +451,22 @@ def run_ours(args, dist, w):
     dist.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
     e0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         timed_step()
     e1.record(stream)
     torch.cuda.synchronize()
+    t1 = time.time()
     dist.barrier()
-    ms = e0.elapsed_time(e1) / args.steps
-    clk = clocks.stop() if clocks else None
+    ms = e0.elapsed_time(e1) / steps
+    clk = None
+    if clocks:
+        clocks.stop()
+        clk = clocks.summary(t0, t1)
     mz.synchronize()
     ms_max = dist.max(ms)
+    region_s = ms_max * steps / 1e3
     value = dist.world * w.T / (ms_max / 1e3)
 
     # ---- a second timed region of the same length with CUDA events between
@@ -350,7 +474,8 @@ def run_ours(args, dist, w):
     mz.profile(True)
     dist.barrier()
     torch.cuda.synchronize()
-    for _ in range(args.steps):
+    n_prof = min(steps, 256)
+    for _ in range(n_prof):
         step()
     torch.cuda.synchronize()
     dist.barrier()
@@ -375,80 +500,81 @@ def run_ours(args, dist, w):
     dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(args.e2e_steps):
+    for _ in range(e2e_steps):
         step_host()
     e1.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
-    e2e_ms = dist.max(e0.elapsed_time(e1) / args.e2e_steps)
+    e2e_ms = dist.max(e0.elapsed_time(e1) / e2e_steps)
     mz.synchronize()
 
-    # ---- roofline of the dominant kernel (largest share of the step)
     per = {k: v / max(nfw, 1) for k, v in stage_ms.items()}
-    dom = max(per, key=per.get)
-    # (batches of at most SMALL_BATCH tokens: the gate/up stage is the one
-    # kernel that runs both expert GEMMs)
-    fused = w.N > 0 and w.T <= SMALL_BATCH
-    kern = {"gateup_gemm": ((rf["F_gateup"] + rf["F_down"], rf["B_gateup"] + rf["B_down"])
-                            if fused else (rf["F_gateup"], rf["B_gateup"])),
-            "down_gemm": (rf["F_down"], rf["B_down"])}.get(dom)
-    roof = None
-    if kern and per[dom] > 0:
-        F, B = kern
-        sec = per[dom] / 1e3
-        t_tensor, t_hbm = F / (pk["bf16_sus"] * 1e12), B / (pk["hbm"] * 1e9)
-        if t_tensor >= t_hbm:
-            ach = F / sec / 1e12
-            roof = {"bound": "tensor", "achieved": ach, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
-                    "frac": ach / pk["bf16_sus"],
-                    "peak_kind": f"bf16 dense, sustained ({pk['src']}, MEASURED_PEAKS.json)"}
-        else:
-            ach = B / sec / 1e9
-            roof = {"bound": "hbm", "achieved": ach, "peak": pk["hbm"], "unit": "GB/s",
-                    "frac": ach / pk["hbm"], "peak_kind": f"HBM copy ({pk['src']})"}
-        roof["kernel"] = "gateup_down_gemm (one kernel)" if fused and dom == "gateup_gemm" else dom
-        roof["ms_per_launch"] = per[dom]
-        tr = NCU_TRAFFIC_BYTES.get(w.name)
-        roof["traffic"] = tr
+    res = {
+        "value": value, "ms_per_step": ms_max, "steps": steps,
+        "e2e": {"value": dist.world * w.T / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": int(x_host.numel() * 2),
+                "d2h_bytes_per_step": int(out_host.numel() * 2), "ms_per_step": e2e_ms,
+                "steps": e2e_steps},
+        "roofline": kernel_roofline(w, rf, plan, per, pk, region_s),
+        "layer_roofline": layer_roofline(rf, pk, ms_max, region_s),
+        "gpu_launches": plan["kernels"] * steps,
+        "clocks": clk,
+        "routing": st,
+        "stage_ms": {k: round(v, 5) for k, v in per.items()},
+        "touched_bytes": st["experts_hit"] * 3.0 * w.d * w.I * 2,
+        "_keep": (ri, b, ew),
+    }
+    del graph
+    return res
 
-    # whole-layer roofline: slower of executed FFN FLOPs at tensor peak and
-    # touched bytes at HBM peak, against the measured step time
-    t_bound = max(rf["F_layer"] / (pk["bf16_sus"] * 1e12), rf["B_layer"] / (pk["hbm"] * 1e9))
-    ffn_tflops = rf["F_layer"] / (ms_max / 1e3) / 1e12
-    layer = {"bound": "tensor" if rf["F_layer"] / (pk["bf16_sus"] * 1e12) >= rf["B_layer"] / (pk["hbm"] * 1e9) else "hbm",
-             "roofline_ms": t_bound * 1e3, "frac": t_bound / (ms_max / 1e3),
-             "executed_ffn_tflops": ffn_tflops,
-             "pct_of_bf16_peak_burst": 100.0 * ffn_tflops / pk["bf16"],
-             "pct_of_bf16_peak_sustained": 100.0 * ffn_tflops / pk["bf16_sus"],
-             "hbm_gbs": rf["B_layer"] / (ms_max / 1e3) / 1e9,
-             "pct_of_hbm": 100.0 * rf["B_layer"] / (ms_max / 1e3) / 1e9 / pk["hbm"]}
 
+def run_ours(args, dist, w):
+    res = measure(args, dist, w, args.steps, args.e2e_steps, headline=True)
+    ri, b, ew = res.pop("_keep")
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, ri, b, ew)
-
-    touched = st["experts_hit"] * 3.0 * w.d * w.I * 2
+    del ri, b, ew
+    touched = res.pop("touched_bytes")
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded inputs, random-init weights of the workload's shapes",
         "config": config_of(w, {
             "global_batch": w.T * dist.world, "parallelism": f"replicas{dist.world}",
             "cuda_graph": bool(args.graph),
             "l2": f"no flush: expert weights touched per step {touched / 1e9:.2f} GB > L2 126 MB"}),
-        "e2e": {"value": dist.world * w.T / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": int(x_host.numel() * 2),
-                "d2h_bytes_per_step": int(out_host.numel() * 2), "ms_per_step": e2e_ms},
-        "roofline": roof,
-        "layer_roofline": layer,
+        "e2e": res["e2e"],
+        "roofline": res["roofline"],
+        "layer_roofline": res["layer_roofline"],
         "cpu_baseline": cpu,
-        "gpu_launches": kernels_per_forward(w) * args.steps,
-        "clocks": clk,
-        "routing": st,
-        "stage_ms": {k: round(v, 5) for k, v in per.items()},
+        "gpu_launches": res["gpu_launches"],
+        "clocks": res["clocks"],
+        "routing": res["routing"],
+        "stage_ms": res["stage_ms"],
     }
+    extra = [n for n in args.workloads.split(",") if n and n != "none" and n != w.name]
+    if extra:
+        line["workloads"] = {}
+    for name in extra:
+        gc_collect()
+        wx = wl.get(name)
+        r = measure(args, dist, wx, 0, max(args.e2e_steps, 20), headline=False)
+        r.pop("_keep")
+        touched = r.pop("touched_bytes")
+        r["config"] = config_of(wx, {
+            "global_batch": wx.T * dist.world,
+            "l2": (f"no flush: expert weights touched per step {touched / 1e9:.2f} GB"
+                   f"{' > ' if touched > L2_BYTES else ' <= '}L2 126 MB")})
+        line["workloads"][name] = r
     return line
+
+
+def gc_collect():
+    import gc
+    gc.collect()
+    torch.cuda.empty_cache()
 
 
 def run_reference(args, dist, w):

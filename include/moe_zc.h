@@ -53,7 +53,7 @@ extern "C" {
 typedef enum moe_zc_status {
   MOE_ZC_OK = 0,
   MOE_ZC_ERR_INVALID_ARG = -1,  /* null pointer, K < 1, K > E, T < 0, N < 0, Z < 0, E < 1 */
-  MOE_ZC_ERR_UNSUPPORTED = -2,  /* d % 128, I % 128, K > 32, E > 1024, misaligned pointer */
+  MOE_ZC_ERR_UNSUPPORTED = -2,  /* d % 64, I % 128, K > 32, E > 1024, misaligned pointer */
   MOE_ZC_ERR_CUDA = -3,         /* a CUDA runtime or driver call failed */
   MOE_ZC_ERR_OOM = -4,          /* workspace allocation failed */
   MOE_ZC_ERR_TIMEOUT = -5,      /* a bounded device-side wait ran out */
@@ -68,7 +68,7 @@ typedef enum moe_zc_status {
  * Forward pass of the layer defined above ("Zero-computation experts").
  * T may be 0 (no work, returns MOE_ZC_OK; x and out may then be NULL, and
  * the expert-load histogram of the call is all zero).  N may be 0 (every pick is a zero
- * expert) and Z may be 0 (plain softmax top-K MoE).  Requires d % 128 == 0,
+ * expert) and Z may be 0 (plain softmax top-K MoE).  Requires d % 64 == 0,
  * I % 128 == 0, 1 <= K <= min(E, 32), E <= 1024, 16-byte aligned pointers.
  * W_gate/W_up/W_down may be NULL only when N == 0.
  * Asynchronous on `stream`; the expert-load histogram and routing of this
@@ -83,9 +83,11 @@ typedef enum moe_zc_status {
  * only: every launch gives the same bits.  Batches of at most 64 tokens run
  * both expert GEMMs in one grid of at most one block per multiprocessor,
  * whose down-projection tiles wait (bounded, like every device wait) for
- * other blocks' gate/up results: should other work hold multiprocessors
- * for longer than the wait bound (2 s), the call reports
- * MOE_ZC_ERR_TIMEOUT instead of hanging.
+ * other blocks' gate/up results; that grid is launched as a cooperative
+ * launch, so the driver either makes all its blocks resident at once or
+ * refuses it, and a refused launch (e.g. too few multiprocessors free to
+ * this process) falls back to two launches with the same bits
+ * (moe_zc_plan shows the choice).
  */
 int moe_zc_forward(const void* x, const void* W_r, const float* b,
                    const void* W_gate, const void* W_up, const void* W_down,
@@ -209,6 +211,34 @@ enum { MOE_ZC_FP8_BLOCK128 = 0, MOE_ZC_FP8_MX32 = 1 };
 int moe_zc_fp8_quantize(const void* W, int64_t rows, int64_t cols, int32_t mode,
                         uint8_t* codes, float* scales);
 
+/*
+ * How moe_zc_forward would launch a batch of these sizes on a device with
+ * `sms` multiprocessors, of which the one-grid expert GEMMs could hold
+ * `resident_blocks` blocks at once (the forward passes its device's
+ * occupancy).  Plain host code (no CUDA call); the forward takes its
+ * decisions from the same function.
+ *   kernels                 kernels one forward launches (0 for T = 0)
+ *   router_grid             blocks of the router GEMM
+ *   router_token_tile       tokens per router tile
+ *   router_k_slices         contraction slices of the router GEMM (1: none)
+ *   expert_gemms_one_grid   1: gate/up and down GEMMs in one persistent grid
+ *                           (batches of at most 64 tokens whose grid can be
+ *                           resident at once), 0: two launches
+ *   expert_grid             blocks of that one grid, or of the gate/up GEMM
+ * Returns the forward's argument-check status (nothing is written unless
+ * MOE_ZC_OK), or MOE_ZC_ERR_INVALID_ARG for a NULL plan or sms < 1.
+ */
+typedef struct moe_zc_launch_plan {
+  int32_t kernels;
+  int32_t router_grid;
+  int32_t router_token_tile;
+  int32_t router_k_slices;
+  int32_t expert_gemms_one_grid;
+  int32_t expert_grid;
+} moe_zc_launch_plan;
+int moe_zc_plan(int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I,
+                int32_t sms, int32_t resident_blocks, moe_zc_launch_plan* plan);
+
 /* Wait for the last forward; report (and clear) a device-side timeout. */
 int moe_zc_synchronize(void);
 
@@ -252,14 +282,16 @@ const char* moe_zc_stage_name(int32_t i);
  * idx (device int32 [T*K], picks in descending biased score), gate (device
  * float [T*K], unbiased softmax probabilities) and counts (device int32 [E],
  * expert-load histogram, cleared by the call).  x, W_r, b, logit_offset
- * (may be NULL) as for moe_zc_forward_ex.  dev_status: device int32 that the
- * call clears and the kernels set non-zero if a bounded wait runs out; NULL
- * uses a word of the library's own array.  Asynchronous on `stream`.
+ * (may be NULL) as for moe_zc_forward_ex.  dev_status (required, device
+ * int32): the call clears it and the kernels set it non-zero if a bounded
+ * wait (2 s) runs out; that is the only place such a timeout is reported,
+ * so read it once the stream's work is done (NULL: MOE_ZC_ERR_INVALID_ARG).
+ * Asynchronous on `stream`.
  *
  * Its scratch (fp32 logits and zero-gate sums) is one fixed array of
  * MOE_ZC_NOALLOC_SCRATCH_BYTES in the library image, held by every GPU that
  * loads the library until the process exits; sizes need
- * 256*ceil(T*E*4/256) + 256*ceil(T*4/256) + 256 <= that, else the call
+ * 256*ceil(T*E*4/256) + 256*ceil(T*4/256) <= that, else the call
  * returns MOE_ZC_ERR_UNSUPPORTED and launches nothing (e.g. E = 768 allows
  * T <= 1363).  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress, with that device current); make that first
@@ -280,6 +312,13 @@ int moe_zc_route_noalloc(const void* x, const void* W_r, const float* b,
  * timeout path runs without a fault.  Not for production use.
  */
 void moe_zc_test_inject(int32_t fail_allocs, int64_t wait_limit);
+
+/*
+ * Test hook: with one_grid_off != 0, forwards never run the two expert GEMMs
+ * of small batches in one grid (the fallback path, same bits); 0 restores
+ * the default.  Not for production use.
+ */
+void moe_zc_test_one_grid(int32_t one_grid_off);
 
 #ifdef __cplusplus
 }

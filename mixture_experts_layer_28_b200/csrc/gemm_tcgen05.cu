@@ -613,16 +613,20 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         __nv_bfloat16* out =
             static_cast<__nv_bfloat16*>(MODE == MODE_FUSED ? p2.out : p.out) + row_blk;
         const int64_t out_ld = MODE == MODE_FUSED ? p2.out_ld : p.out_ld;
+        // d % 128 == 64: the last weight block's upper 64 rows lie past d
+        // (their accumulator lanes hold no output feature and are not stored)
+        const int a_rows = MODE == MODE_FUSED ? p2.a_rows : p.a_rows;
         uint32_t hp[3][16];
         epi_read_bf16<MODE_DOWN>(tacc, group, tl.nmma, hp);
         tc_fence_before();
         mbar_arrive(&acc_empty_bar[buf]);
-        epi_store_bf16(stg, lane, group, tl, hp, out, out_ld, pol_out);
+        if (row_blk < a_rows) epi_store_bf16(stg, lane, group, tl, hp, out, out_ld, pol_out);
         if (nbuf == 1) {
           if (tl.has_a1) epi_read_bf16<MODE_DOWN>(tacc + 256, group, tl.nmma, hp);
           tc_fence_before();
           mbar_arrive(&acc_empty_bar[1]);
-          if (tl.has_a1) epi_store_bf16(stg, lane, group, tl, hp, out + GEMM_BM, out_ld, pol_out);
+          if (tl.has_a1 && row_blk + GEMM_BM < a_rows)
+            epi_store_bf16(stg, lane, group, tl, hp, out + GEMM_BM, out_ld, pol_out);
         }
       }
     }
@@ -654,6 +658,11 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
     }
     p.pair_tiles = 0;
   }
+  // a down tile of the one grid may wait for any other block's gate/up
+  // tiles: every block must be resident at once
+  if (MODE == MODE_FUSED)
+    return launch_pdl_coop(gemm_kernel<MODE, NST, SB>, dim3(grid), dim3(GEMM_THREADS), smem,
+                           stream, a0, a1, b, b_full, a2, b2, p, p2);
   return launch_pdl(gemm_kernel<MODE, NST, SB>, dim3(grid), dim3(GEMM_THREADS), smem, stream,
                     a0, a1, b, b_full, a2, b2, p, p2);
 }
@@ -701,15 +710,26 @@ cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, cons
                               const CUtensorMap& wd, const CUtensorMap& h, const GemmParams& pg,
                               const GemmParams& pd, int grid, cudaStream_t stream) {
   if (grid <= 0) return cudaSuccess;
-  // every CTA resident at once (one per SM): a down tile may wait for
-  // gate/up tiles of any other CTA
   if (grid > device_sms() || !pg.small_b || pg.pair_tiles || pg.b_box_full || pd.single_a ||
       pg.done == nullptr)
     return cudaErrorInvalidValue;
-  const cudaError_t e = launch_mode<MODE_FUSED, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>(
+  // (a refused cooperative launch leaves nothing queued: launch_mode's error
+  // is returned as is, without cudaGetLastError, for the caller to clear)
+  return launch_mode<MODE_FUSED, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>(
       wg, wu, xp, xp, wd, h, pg, pd, grid, stream);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+}
+
+int fused_resident_blocks() {
+  constexpr int smem = GEMM_SMALL_STAGES * GEMM_SMALL_STAGE_BYTES +
+                       GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024;
+  if (smem_limit<gemm_kernel<MODE_FUSED, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>>(smem) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return blocks_per_sm<gemm_kernel<MODE_FUSED, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>>(
+             GEMM_THREADS, smem) *
+         device_sms();
 }
 
 }  // namespace moezc

@@ -29,6 +29,26 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// launch_pdl as a cooperative launch: the driver makes every block of the
+// grid resident at once, or refuses the launch (cudaErrorCooperativeLaunchTooLarge).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_coop(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                   cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Raises a kernel's dynamic shared-memory limit to `bytes` on the current
 // device, once: later calls only read a per-device cache, so a forward makes
 // no attribute calls after its first (e.g. while a caller captures it into a
@@ -99,6 +119,10 @@ inline int device_sms() {
   }
   return cached[dev];
 }
+
+// The wait bound that moe_zc_test_inject set for the next call (0: none), and
+// clear it; the forward and the no-allocation routing call take it.
+long long take_injected_wait_ns();
 
 // ------------------------------------------------------------------ GEMM
 // One tcgen05 engine serves the three contractions of the layer.  Weights are
@@ -179,10 +203,15 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
 // Gate/up then down in one persistent grid of `grid` CTAs (batches of at most
 // GEMM_SMALL_B tokens): wg, wu, xp as for the gate/up launch (parameters pg,
 // with pg.done and pg.down_lead set), wd and h as for the down launch
-// (parameters pd).
+// (parameters pd).  A cooperative launch: an error return (the grid cannot be
+// resident at once) launches nothing, and the caller runs the two GEMMs as
+// separate launches instead.
 cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, const CUtensorMap& xp,
                               const CUtensorMap& wd, const CUtensorMap& h, const GemmParams& pg,
                               const GemmParams& pd, int grid, cudaStream_t stream);
+// Blocks of the one-grid expert GEMM kernel the current device holds at once
+// (its occupancy times the multiprocessors).
+int fused_resident_blocks();
 
 // ------------------------------------------------------------------ router
 // softmax over E logits (+offset), + bias, top-K, zero-gate sums, histogram.

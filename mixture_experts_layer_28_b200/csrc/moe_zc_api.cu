@@ -68,6 +68,7 @@ struct Ctx {
   int hist_N = 0;
   bool pair_hint = false;            // most FFN pairs sit in experts with two token tiles
   bool spread_hint = false;          // at least half of the N FFN experts were hit
+  bool one_grid_refused = false;     // the one-grid expert GEMMs' cooperative launch was refused
 };
 
 Ctx g_ctx[kMaxDevices];
@@ -205,6 +206,41 @@ RouterPlan router_plan(int64_t T, int E, int ksteps, int sms) {
   return rp;
 }
 
+// The launch plan of a forward (moe_zc_plan; forward_impl takes its decisions
+// from it).  The expert GEMMs' grids are sized from an upper bound of their
+// tiles (every expert's last token tile may be partial), since the routing is
+// not known on the host.
+struct Plan {
+  RouterPlan rp;
+  int64_t router_grid = 0;
+  bool one_grid = false;        // gate/up and down GEMMs in one persistent grid
+  int64_t gateup_grid = 0, down_grid = 0, fused_grid = 0;
+  int kernels = 0;
+};
+bool g_one_grid_off = false;    // test hook: never use the one grid
+
+Plan make_plan(int64_t T, int d, int N, int Z, int K, int I, int sms, int64_t resident) {
+  Plan pl;
+  const int E = N + Z;
+  pl.rp = router_plan(T, E, d / GEMM_BK, sms);
+  const int64_t rg = pl.rp.tiles * pl.rp.splits;
+  pl.router_grid = rg < sms ? rg : sms;
+  if (T == 0) return pl;                         // a memset of the histogram only
+  if (N == 0) {
+    pl.kernels = 4;                              // router GEMM, route, assign, combine
+    return pl;
+  }
+  const int64_t tiles_ub = (T * K + GEMM_BN - 1) / GEMM_BN + N;
+  const int64_t g_ub = tiles_ub * (I / GEMM_BM);
+  const int64_t d_ub = tiles_ub * ((d + 2 * GEMM_BM - 1) / (2 * GEMM_BM));
+  pl.gateup_grid = g_ub < sms ? g_ub : sms;
+  pl.down_grid = d_ub < sms ? d_ub : sms;
+  pl.fused_grid = g_ub + d_ub < sms ? g_ub + d_ub : sms;
+  pl.one_grid = T <= GEMM_SMALL_B && !g_one_grid_off && pl.fused_grid <= resident;
+  pl.kernels = pl.one_grid ? 6 : 7;
+  return pl;
+}
+
 int reserve_impl(Ctx& c, int64_t T, int d, int N, int Z, int K, int I) {
   const int64_t E = static_cast<int64_t>(N) + Z;
   const int64_t pairs = T * K;
@@ -249,7 +285,7 @@ int check_args(const void* x, const void* W_r, const float* b, const void* W_gat
   if (E < 1 || K < 1 || K > E) return MOE_ZC_ERR_INVALID_ARG;
   if (N > 0 && (!W_gate || !W_up || !W_down || I <= 0)) return MOE_ZC_ERR_INVALID_ARG;
   if (K > MOE_ZC_MAX_K || E > MOE_ZC_MAX_E) return MOE_ZC_ERR_UNSUPPORTED;
-  if (d % 128 != 0) return MOE_ZC_ERR_UNSUPPORTED;
+  if (d % GEMM_BK != 0) return MOE_ZC_ERR_UNSUPPORTED;   // whole 64-wide K steps
   if (N > 0 && I % 128 != 0) return MOE_ZC_ERR_UNSUPPORTED;
   if (T * K + 16LL * N + 16 > (1LL << 31) - 1) return MOE_ZC_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(N) * (d > I ? d : I) > (1LL << 31) - 1) return MOE_ZC_ERR_UNSUPPORTED;
@@ -364,10 +400,14 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   // concentrated).  The choice follows the histogram of an earlier forward.
   if (!captured && (s = read_load_hints(c, N)) != MOE_ZC_OK) return s;
   const bool pace_tiles = N > 0 && T >= 1024 && c.pair_hint;
+  const Plan plan = make_plan(T, d, N, Z, K, I, c.sms,
+                              T > 0 && T <= GEMM_SMALL_B && N > 0 && !c.one_grid_refused
+                                  ? fused_resident_blocks()
+                                  : 0);
   if (T > 0) {
     // 1  router GEMM
     CUtensorMap mWr, mX;
-    const RouterPlan rp = router_plan(T, E, d / GEMM_BK, c.sms);
+    const RouterPlan rp = plan.rp;
     // x in boxes of 32 tokens, and of one full token tile (rp.tok_tile)
     CUtensorMap mXf;
     const bool full_ok = T >= rp.tok_tile;
@@ -392,15 +432,13 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     const int splits = rp.splits;
     pr.ksplit = splits;
     pr.split_stride = T * E;
-    const int64_t rgrid = rp.tiles * splits;
     pr.b_box_full = full_ok ? 1 : 0;
     pr.small_b = T <= GEMM_SMALL_B ? 1 : 0;
     pr.zero0 = cnt;
     pr.nzero0 = E;
     pr.zero1 = fill;
     pr.nzero1 = 2 * N + 2;
-    CK(launch_gemm(MODE_ROUTER, mWr, mWr, mX, mXf, pr,
-                   static_cast<int>(rgrid < c.sms ? rgrid : c.sms), st));
+    CK(launch_gemm(MODE_ROUTER, mWr, mWr, mX, mXf, pr, static_cast<int>(plan.router_grid), st));
     rec.mark(1);
     // 2  route
     CK(launch_route(static_cast<const float*>(c.logits.p), b, off, T, E, N, K, idx, gate, zsum,
@@ -413,7 +451,6 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       CK(launch_permute(static_cast<const __nv_bfloat16*>(x), slot, T, d, K,
                         static_cast<__nv_bfloat16*>(c.Xp.p), st));
       rec.mark(4);
-      const int64_t tiles_ub = (T * K + GEMM_BN - 1) / GEMM_BN + N;
       // 5  gate/up GEMM
       CUtensorMap mWg, mWu, mXp;
       if (!make_map(&mWg, W_gate, static_cast<uint64_t>(N) * I, d, GEMM_BM) ||
@@ -457,30 +494,38 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       pd.a_rows = d;
       pd.out = c.Y.p;
       pd.out_ld = d;
-      const int64_t g_ub = tiles_ub * pg.mblocks;
-      const int64_t d_ub = tiles_ub * pd.mblocks;
-      if (pg.small_b) {
+      bool one_grid = plan.one_grid;
+      if (one_grid) {
         // 5-6  at most 64 tokens: both expert GEMMs in one persistent grid,
         // the down tiles of an expert starting as soon as its H rows are
         // stored (the SMs that the last round of gate/up tiles leaves idle
         // stream down weights meanwhile); a gate/up tile costs about d / I
         // down tiles
-        pg.b_box_full = 0;
-        pg.done = fill + N + 1;
-        pg.down_lead = (d + I / 2) / I;
-        const int64_t f_ub = g_ub + d_ub;
-        CK(launch_gemm_fused(mWg, mWu, mXp, mWd, mH, pg, pd,
-                             static_cast<int>(f_ub < c.sms ? f_ub : c.sms), st));
-        rec.mark(5);
-        rec.mark(6);
-      } else {
+        GemmParams pf = pg;
+        pf.b_box_full = 0;
+        pf.done = fill + N + 1;
+        pf.down_lead = (d + I / 2) / I;
+        const cudaError_t e = launch_gemm_fused(mWg, mWu, mXp, mWd, mH, pf, pd,
+                                                static_cast<int>(plan.fused_grid), st);
+        if (e != cudaSuccess) {
+          // refused as a cooperative launch (its blocks cannot all be
+          // resident): nothing was queued; run the two launches from now on
+          cudaGetLastError();
+          if (captured) return MOE_ZC_ERR_CUDA;   // (the capture is invalidated)
+          c.one_grid_refused = true;
+          one_grid = false;
+        } else {
+          rec.mark(5);
+          rec.mark(6);
+        }
+      }
+      if (!one_grid) {
         // 5  gate/up GEMM
-        CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg,
-                       static_cast<int>(g_ub < c.sms ? g_ub : c.sms), st));
+        CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg, static_cast<int>(plan.gateup_grid),
+                       st));
         rec.mark(5);
         // 6  down GEMM
-        CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd,
-                       static_cast<int>(d_ub < c.sms ? d_ub : c.sms), st));
+        CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd, static_cast<int>(plan.down_grid), st));
         rec.mark(6);
       }
     } else {
@@ -642,6 +687,13 @@ int sync_impl(Ctx& c) {
 }
 
 }  // namespace
+
+long long moezc::take_injected_wait_ns() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const long long v = g_wait_ns_next;
+  g_wait_ns_next = 0;
+  return v;
+}
 
 extern "C" {
 
@@ -831,6 +883,32 @@ int moe_zc_profile_read(float* stage_ms, int32_t max_stages, int32_t* n_forwards
 
 const char* moe_zc_stage_name(int32_t i) {
   return (i >= 0 && i < kStages) ? kStageNames[i] : nullptr;
+}
+
+int moe_zc_plan(int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I, int32_t sms,
+                int32_t resident_blocks, moe_zc_launch_plan* plan) {
+  if (!plan || sms < 1) return MOE_ZC_ERR_INVALID_ARG;
+  const void* f = reinterpret_cast<const void*>(16);   // stand-ins for the device pointers
+  const int s = check_args(f, f, static_cast<const float*>(f), f, f, f, T, d, N, Z, K, I,
+                           nullptr, f);
+  if (s != MOE_ZC_OK) return s;
+  Plan pl;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    pl = make_plan(T, d, N, Z, K, N > 0 ? I : 128, sms, resident_blocks);
+  }
+  plan->kernels = pl.kernels;
+  plan->router_grid = static_cast<int32_t>(pl.router_grid);
+  plan->router_token_tile = pl.rp.tok_tile;
+  plan->router_k_slices = pl.rp.splits;
+  plan->expert_gemms_one_grid = pl.one_grid ? 1 : 0;
+  plan->expert_grid = static_cast<int32_t>(pl.one_grid ? pl.fused_grid : pl.gateup_grid);
+  return MOE_ZC_OK;
+}
+
+void moe_zc_test_one_grid(int32_t one_grid_off) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_one_grid_off = one_grid_off != 0;
 }
 
 void moe_zc_test_inject(int32_t fail_allocs, int64_t wait_limit) {

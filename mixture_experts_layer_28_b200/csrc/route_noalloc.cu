@@ -22,8 +22,10 @@
 // cudaGetSymbolAddress and keeps it; make that first call before any stream
 // capture.  All calls share the array and it keeps the last call's contents:
 // the entry point clears what must start at zero (the caller's counts and
-// status), and calls whose work overlaps on the GPU (two streams, or two
-// threads) race on the array -- serialise them.
+// status word), and calls whose work overlaps on the GPU (two streams, or two
+// threads) race on the array -- serialise them.  The status word is the
+// caller's (required): a bounded device wait that runs out is reported there
+// and nowhere else.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -40,7 +42,7 @@ using namespace moezc;
 
 constexpr size_t kStaticScratchBytes = MOE_ZC_NOALLOC_SCRATCH_BYTES;
 constexpr int kMaxDev = 16;
-constexpr long long kNoallocWaitNs = 2000000000LL;
+constexpr long long kNoallocWaitNs = 2000000000LL;   // bound of every device wait
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kStaticScratchBytes];
 
@@ -105,18 +107,18 @@ extern "C" int moe_zc_route_noalloc(const void* x, const void* W_r, const float*
                                     const float* logit_offset, int64_t T, int32_t d, int32_t N,
                                     int32_t Z, int32_t K, int32_t* idx, float* gate,
                                     int32_t* counts, int32_t* dev_status, void* stream) {
-  if (!W_r || !b || !counts) return MOE_ZC_ERR_INVALID_ARG;
+  if (!W_r || !b || !counts || !dev_status) return MOE_ZC_ERR_INVALID_ARG;
   if (T < 0 || N < 0 || Z < 0 || d <= 0) return MOE_ZC_ERR_INVALID_ARG;
   const int64_t E = static_cast<int64_t>(N) + Z;
   if (E < 1 || K < 1 || K > E) return MOE_ZC_ERR_INVALID_ARG;
   if (T > 0 && (!x || !idx || !gate)) return MOE_ZC_ERR_INVALID_ARG;
-  if (K > MOE_ZC_MAX_K || E > MOE_ZC_MAX_E || d % 128 != 0) return MOE_ZC_ERR_UNSUPPORTED;
+  if (K > MOE_ZC_MAX_K || E > MOE_ZC_MAX_E || d % GEMM_BK != 0) return MOE_ZC_ERR_UNSUPPORTED;
   auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!al(x) || !al(W_r) || !al(b) || !al(logit_offset)) return MOE_ZC_ERR_UNSUPPORTED;
-  // scratch: logits [T, E] fp32, zero-gate sums [T] fp32, status word
+  // scratch: logits [T, E] fp32, then zero-gate sums [T] fp32
   const size_t logits_bytes = round256(static_cast<size_t>(T) * E * sizeof(float));
   const size_t zsum_bytes = round256(static_cast<size_t>(T) * sizeof(float));
-  if (logits_bytes + zsum_bytes + 256 > kStaticScratchBytes) return MOE_ZC_ERR_UNSUPPORTED;
+  if (logits_bytes + zsum_bytes > kStaticScratchBytes) return MOE_ZC_ERR_UNSUPPORTED;
 
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
   NoallocDevice* s = nullptr;
@@ -125,13 +127,14 @@ extern "C" int moe_zc_route_noalloc(const void* x, const void* W_r, const float*
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   float* logits = reinterpret_cast<float*>(s->scratch);
   float* zsum = reinterpret_cast<float*>(s->scratch + logits_bytes);
-  int* err = dev_status ? dev_status
-                        : reinterpret_cast<int*>(s->scratch + logits_bytes + zsum_bytes);
+  int* err = dev_status;
   if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, cs) != cudaSuccess ||
       cudaMemsetAsync(err, 0, sizeof(int32_t), cs) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ZC_ERR_CUDA;
   }
+  // (the error-path test hook may shorten the waits of this call)
+  const long long injected = take_injected_wait_ns();
   if (T == 0) return MOE_ZC_OK;
 
   CUtensorMap mWr, mX;
@@ -146,7 +149,7 @@ extern "C" int moe_zc_route_noalloc(const void* x, const void* W_r, const float*
   pr.out = logits;
   pr.out_ld = static_cast<int>(E);
   pr.err = err;
-  pr.wait_ns = kNoallocWaitNs;
+  pr.wait_ns = injected > 0 ? injected : kNoallocWaitNs;
   const int64_t tiles = ((T + GEMM_BN - 1) / GEMM_BN) * pr.mblocks;
   if (launch_gemm(MODE_ROUTER, mWr, mWr, mX, mX, pr, static_cast<int>(tiles < s->sms ? tiles : s->sms),
                   cs) != cudaSuccess ||

@@ -42,6 +42,13 @@ class Pid(ctypes.Structure):
                 ("ki", ctypes.c_float), ("kd", ctypes.c_float), ("max_shift", ctypes.c_float)]
 
 
+class LaunchPlan(ctypes.Structure):
+    """moe_zc_launch_plan (include/moe_zc.h)."""
+    _fields_ = [("kernels", ctypes.c_int32), ("router_grid", ctypes.c_int32),
+                ("router_token_tile", ctypes.c_int32), ("router_k_slices", ctypes.c_int32),
+                ("expert_gemms_one_grid", ctypes.c_int32), ("expert_grid", ctypes.c_int32)]
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 
@@ -93,6 +100,11 @@ def lib() -> ctypes.CDLL:
         L.moe_zc_test_inject.restype = None
         L.moe_zc_fp8_quantize.argtypes = [vp, i64, i64, i32, vp, vp]
         L.moe_zc_fp8_quantize.restype = ctypes.c_int
+        L.moe_zc_plan.argtypes = [i64, i32, i32, i32, i32, i32, i32, i32,
+                                  ctypes.POINTER(LaunchPlan)]
+        L.moe_zc_plan.restype = ctypes.c_int
+        L.moe_zc_test_one_grid.argtypes = [i32]
+        L.moe_zc_test_one_grid.restype = None
         _lib = L
     return _lib
 
@@ -219,11 +231,12 @@ NOALLOC_SCRATCH_BYTES = 4 << 20
 
 def route_noalloc(x: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor, N: int, Z: int, K: int,
                   idx: torch.Tensor, gate: torch.Tensor, counts: torch.Tensor,
-                  logit_offset: Optional[torch.Tensor] = None,
-                  status: Optional[torch.Tensor] = None, stream=None) -> None:
+                  status: torch.Tensor, logit_offset: Optional[torch.Tensor] = None,
+                  stream=None) -> None:
     """moe_zc_route_noalloc: routing into caller-owned device tensors
-    (idx int32 [T, K], gate fp32 [T, K], counts int32 [E], status int32 [1]),
-    with no device allocation by the library."""
+    (idx int32 [T, K], gate fp32 [T, K], counts int32 [E]) with no device
+    allocation by the library; status (int32 [1], device) is cleared by the
+    call and set non-zero on the device if a bounded wait runs out."""
     T, d = x.shape
     st = lib().moe_zc_route_noalloc(
         _dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(W_r, torch.bfloat16, "W_r"),
@@ -310,6 +323,20 @@ def allreduce_expert_load(counts: np.ndarray, group=None) -> np.ndarray:
 
 def test_inject(fail_allocs: int = 0, wait_limit_ns: int = 0) -> None:
     lib().moe_zc_test_inject(fail_allocs, wait_limit_ns)
+
+
+def plan(T: int, d: int, N: int, Z: int, K: int, I: int, sms: int = 148,
+         resident_blocks: int = 148) -> dict:
+    """moe_zc_plan: how a forward of these sizes is launched (host only)."""
+    p = LaunchPlan()
+    _check(lib().moe_zc_plan(T, d, N, Z, K, I, sms, resident_blocks, ctypes.byref(p)),
+           "moe_zc_plan")
+    return {name: getattr(p, name) for name, _ in LaunchPlan._fields_}
+
+
+def test_one_grid(off: bool) -> None:
+    """Test hook: keep small batches off the one-grid expert GEMMs."""
+    lib().moe_zc_test_one_grid(1 if off else 0)
 
 
 def declared_symbols() -> list[str]:

@@ -4,6 +4,7 @@ invalid arguments are rejected before any CUDA call)."""
 import ctypes
 
 import pytest
+import torch
 
 from mixture_experts_layer_28_b200 import build as mb
 from mixture_experts_layer_28_b200 import moe_zc as mz
@@ -56,7 +57,8 @@ def _fwd(L, x=FAKE, W_r=FAKE, b=FAKE, Wg=FAKE, Wu=FAKE, Wd=FAKE, T=16, d=128, N=
     (dict(N=0, Z=0, K=1), mz.ERR_INVALID_ARG),    # empty expert pool
     (dict(Wg=None), mz.ERR_INVALID_ARG),          # FFN experts need weights
     (dict(I=0), mz.ERR_INVALID_ARG),
-    (dict(d=192), mz.ERR_UNSUPPORTED),            # d % 128
+    (dict(d=96), mz.ERR_UNSUPPORTED),             # d % 64
+    (dict(d=200), mz.ERR_UNSUPPORTED),
     (dict(I=64), mz.ERR_UNSUPPORTED),             # I % 128
     (dict(N=40, Z=0, K=33), mz.ERR_UNSUPPORTED),  # K > 32
     (dict(N=1000, Z=100, K=2), mz.ERR_UNSUPPORTED),  # E > 1024
@@ -68,10 +70,40 @@ def test_argument_checks(L, kw, status):
     assert _fwd(L, **kw) == status
 
 
+# The next checks pass the argument checks with fake pointers, so the call
+# goes on to the device: run them only where there is none.
+_no_device = pytest.mark.skipif(torch.cuda.is_available(),
+                                reason="fake pointers must not reach a GPU")
+
+
+@_no_device
 def test_zero_ffn_experts_need_no_weights(L):
     # N = 0: weights may be NULL and I is ignored; only the device call can fail here
     st = _fwd(L, Wg=None, Wu=None, Wd=None, N=0, Z=4, K=2, I=0)
     assert st in (mz.OK, mz.ERR_CUDA, mz.ERR_UNSUPPORTED)
+
+
+@_no_device
+@pytest.mark.parametrize("d", [64, 192, 320])
+def test_widths_of_whole_k_steps_are_accepted(L, d):
+    """d needs only whole 64-wide contraction steps (d % 64 == 0); the
+    down projection's last 128-row weight block may be half past d."""
+    assert _fwd(L, d=d) == mz.ERR_CUDA   # past the checks; no device here
+
+
+def _noalloc(L, status=FAKE, d=128, **kw):
+    a = dict(x=FAKE, W_r=FAKE, b=FAKE, off=None, T=16, N=4, Z=2, K=2, idx=FAKE, gate=FAKE,
+             counts=FAKE)
+    a.update(kw)
+    return L.moe_zc_route_noalloc(a["x"], a["W_r"], a["b"], a["off"], a["T"], d, a["N"], a["Z"],
+                                  a["K"], a["idx"], a["gate"], a["counts"], status, None)
+
+
+def test_noalloc_argument_checks(L):
+    assert _noalloc(L, status=None) == mz.ERR_INVALID_ARG   # the status word is required
+    assert _noalloc(L, counts=None) == mz.ERR_INVALID_ARG
+    assert _noalloc(L, d=96) == mz.ERR_UNSUPPORTED
+    assert _noalloc(L, T=1364, N=512, Z=256, K=12) == mz.ERR_UNSUPPORTED   # past the array
 
 
 def test_reserve_argument_checks(L):

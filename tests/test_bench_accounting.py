@@ -58,3 +58,57 @@ def test_prefill_executed_ffn_flops():
     rf = bench.roofline_numbers(w, dict(ffn_pairs=137695, experts_hit=57), None)
     assert rf["F_layer"] == 6.0 * 6144 * 2048 * 137695
     assert abs(rf["F_layer"] / 9.06e-3 / 1e12 / 1662.4 - 0.69) < 0.005
+
+
+def _pk():
+    return dict(hbm=6457.4, bf16=1662.4, bf16_sus=1374.8, src="measured")
+
+
+def test_short_regions_use_the_burst_peak():
+    """A timed region of 20 prefill steps (~0.2 s) holds kernels to the burst
+    bf16 peak; only regions of seconds use the sustained one."""
+    assert bench.bf16_peak(_pk(), 0.18)[0] == 1662.4
+    assert bench.bf16_peak(_pk(), 5.0)[0] == 1374.8
+
+
+def test_prefill_gateup_roofline_against_burst_peak():
+    """The gate/up GEMM of the prefill layer: 4 d I FLOPs per pair over
+    137,695 pairs in 5.2495 ms is 1320 TFLOP/s, 0.794 of the 1662.4 burst
+    peak (0.960 of the sustained one)."""
+    w = wl.get("prefill")
+    rf = bench.roofline_numbers(w, dict(ffn_pairs=137695, experts_hit=57), None)
+    plan = dict(expert_gemms_one_grid=0)
+    per = {"router_gemm": 0.15, "gateup_gemm": 5.2495, "down_gemm": 2.83}
+    roof = bench.kernel_roofline(w, rf, plan, per, _pk(), region_s=0.18)
+    assert roof["bound"] == "tensor" and roof["kernel"] == "gateup_gemm"
+    assert abs(roof["achieved"] - 1320.2) < 0.5
+    assert abs(roof["frac"] - 0.794) < 0.001
+    assert abs(roof["frac_of_sustained_peak"] - 0.960) < 0.001
+
+
+def test_decode_one_grid_roofline_is_hbm_bound():
+    """Decode: the one kernel running both expert GEMMs moves 2.279 GB; at
+    0.35 ms that is 6.51 TB/s, against the 6457.4 GB/s measured copy peak and
+    the 7.7 TB/s nominal figure."""
+    w = wl.get("decode")
+    rf = bench.roofline_numbers(w, dict(ffn_pairs=460, experts_hit=30), None)
+    roof = bench.kernel_roofline(w, rf, dict(expert_gemms_one_grid=1),
+                                 {"gateup_gemm": 0.35, "route": 0.02}, _pk(), region_s=1.0)
+    assert roof["bound"] == "hbm" and roof["kernel"].startswith("gateup_down_gemm")
+    assert abs(roof["achieved"] - 2.279e9 / 0.35e-3 / 1e9) < 5
+    assert abs(roof["frac_of_nominal_hbm"] - roof["achieved"] / 7700.0) < 1e-12
+
+
+def test_clock_samples_outside_the_region_are_dropped():
+    c = bench.ClockSampler(0)
+    c.lines = [
+        "2026/12/02 10:00:00.000, 0, 600, 1965, 200, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/02 10:00:01.000, 0, 1965, 1965, 900, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/02 10:00:01.100, 0, 1900, 1965, 950, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/02 10:00:03.000, 0, 700, 1965, 250, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    t0 = bench.ClockSampler._stamp("2026/12/02 10:00:00.900")
+    t1 = bench.ClockSampler._stamp("2026/12/02 10:00:01.200")
+    s = c.summary(t0, t1)
+    assert s["samples"] == 2 and s["sm_mhz"] == (1965 + 1900) / 2
+    assert s["reasons"] == ["sw_power_cap"] and s["samples_outside_region"] == 2
