@@ -16,7 +16,11 @@
 //   law         b_i = base_i + clip(kp e_i + ki sum_s e_i(s) + kd (e_i - e_i,prev))
 //
 // with base_i the bias when the controller was (re)started.  An expert that
-// gets too few picks has e_i > 0 and its bias rises.  Arithmetic in double.
+// gets too few picks has e_i > 0 and its bias rises.  With a clip, a step
+// whose unclipped output lies beyond it on the side its error pushes towards
+// leaves the integral as it was (conditional integration against integral
+// windup): after a long saturated stretch the bias leaves the clip as soon as
+// the error turns.  Arithmetic in double.
 #include <cmath>
 #include <cstdint>
 
@@ -48,10 +52,16 @@ extern "C" int moe_zc_bias_controller_step(const int32_t* counts, int32_t N, int
   for (int32_t i = 0; i < E; ++i) {
     const double target = i < N ? (1.0 - rho) * picks / N : rho * picks / Z;
     const double e = (target - counts[i]) / mean;
-    const double integral = static_cast<double>(state[E + i]) + e;
+    double integral = static_cast<double>(state[E + i]) + e;
     const double deriv = e - static_cast<double>(state[2 * E + i]);
     double shift = pid->kp * e + pid->ki * integral + pid->kd * deriv;
-    if (clip > 0.0) shift = std::fmax(-clip, std::fmin(clip, shift));
+    if (clip > 0.0) {
+      if (std::fabs(shift) > clip && (shift > 0.0) == (e > 0.0) && e != 0.0) {
+        integral = static_cast<double>(state[E + i]);   // saturated: do not wind up
+        shift = pid->kp * e + pid->ki * integral + pid->kd * deriv;
+      }
+      shift = std::fmax(-clip, std::fmin(clip, shift));
+    }
     b[i] = static_cast<float>(static_cast<double>(state[i]) + shift);
     state[E + i] = static_cast<float>(integral);
     state[2 * E + i] = static_cast<float>(e);

@@ -8,6 +8,11 @@ reading taken (the same as the library's controller states):
   set-point  L*_i = (1 - rho) T K / N for FFN experts, rho T K / Z for zero experts
   error      e_i = (L*_i - L_i) / (T K / E)
   law        b_i = base_i + clip(kp e_i + ki sum_s e_i(s) + kd (e_i - e_i,prev))
+
+with conditional integration (the textbook remedy for integral windup of a
+clipped PID): a step whose unclipped output would lie beyond the clip on the
+side its error pushes towards leaves the integral as it was, so that after a
+long saturated stretch the bias leaves the clip as soon as the error turns.
 """
 from __future__ import annotations
 
@@ -47,9 +52,14 @@ def step(state: PidState, counts, N: int, Z: int, tokens: int, K: int, rho: floa
     counts = np.asarray(counts, dtype=np.float64)
     E = N + Z
     e = (target_load(N, Z, tokens, K, rho) - counts) / (float(tokens) * K / E)
-    state.integral = state.integral + e
-    shift = kp * e + ki * state.integral + kd * (e - state.prev)
+    integral = state.integral + e
+    shift = kp * e + ki * integral + kd * (e - state.prev)
     if max_shift > 0:
+        # saturated, and the error pushes further out: do not integrate
+        wind = (np.abs(shift) > max_shift) & (np.sign(shift) == np.sign(e))
+        integral = np.where(wind, state.integral, integral)
+        shift = kp * e + ki * integral + kd * (e - state.prev)
         shift = np.clip(shift, -max_shift, max_shift)
+    state.integral = integral
     state.prev = e
     return state.base + shift

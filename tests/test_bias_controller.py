@@ -57,6 +57,44 @@ def test_oracle_closed_form_step_responses():
     np.testing.assert_allclose(b, base + np.clip(10 * e, -0.3, 0.3), atol=1e-15)
 
 
+def test_oracle_integral_does_not_wind_up_while_clipped():
+    """Integral term alone (ki = 0.07), error +-0.5, clip 0.3.  Step n gives
+    0.035 n until 0.035 n would pass the clip (n = 9): from then on the
+    integral stays at 8 e and the output at 0.28.  After 20 such steps the
+    load turns (error -+0.5): the integral drops to 7 e at once and the
+    output to 0.245 -- without the remedy the integral would be 20 e and the
+    output would stay clipped at 0.3 for another dozen steps."""
+    N, Z, T, K = 3, 1, 40, 2
+    base = np.array([0.1, -0.2, 0.3, 0.0])
+    rho = 0.25
+    st = pc.PidState(base)
+    for n in range(1, 21):
+        b = pc.step(st, [10, 30, 20, 20], N, Z, T, K, rho, kp=0.0, ki=0.07, kd=0.0,
+                    max_shift=0.3)
+        want = 0.07 * 0.5 * min(n, 8)
+        np.testing.assert_allclose(b[:2], base[:2] + np.array([want, -want]), atol=1e-12)
+    np.testing.assert_allclose(st.integral[:2], [4.0, -4.0], atol=1e-12)
+    b = pc.step(st, [30, 10, 20, 20], N, Z, T, K, rho, kp=0.0, ki=0.07, kd=0.0, max_shift=0.3)
+    np.testing.assert_allclose(b[:2], base[:2] + np.array([0.245, -0.245]), atol=1e-12)
+
+
+def test_library_matches_oracle_through_saturation():
+    """The C controller against the oracle over a saturating stretch and a
+    turn of the load, with P, I and D all on."""
+    N, Z, T, K = 3, 1, 40, 2
+    base = np.array([0.1, -0.2, 0.3, 0.0], dtype=np.float32)
+    pid = dict(rho=0.25, kp=0.05, ki=0.07, kd=0.02, max_shift=0.3)
+    ctl = mz.BiasController(base, N, Z, K, target_zero_frac=pid["rho"], kp=pid["kp"],
+                            ki=pid["ki"], kd=pid["kd"], max_shift=pid["max_shift"])
+    st = pc.PidState(base.astype(np.float64))
+    for n in range(30):
+        counts = [10, 30, 20, 20] if n < 20 else [30, 10, 20, 20]
+        got = ctl.step(np.array(counts, dtype=np.int32), T)
+        want = pc.step(st, counts, N, Z, T, K, pid["rho"], pid["kp"], pid["ki"], pid["kd"],
+                       pid["max_shift"])
+        np.testing.assert_allclose(got, want, rtol=1e-5, atol=1e-6)
+
+
 # ---------------------------------------------------------------- C vs oracle
 def test_library_controller_matches_oracle():
     rng = np.random.default_rng(0)
