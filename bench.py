@@ -20,9 +20,11 @@ own weight replica (tokens are independent: no collective in the step), so
 `value` is N*T*K / max-rank time ("weak" scaling).
 
 The JSON line also carries `workloads`: the decode, small and skewed40
-workloads (--workloads), each timed the same way in the same run, with its own
-ms_per_step, tokens/s, e2e, roofline, layer_roofline and clocks (each timed
-region lasts at least about a second, so the clocks are sampled inside it).
+workloads and the decode and prefill layers with FP8 gate/up projections
+(moe_zc_forward_fp8, `dtype` says so) (--workloads), each timed the same way
+in the same run, with its own ms_per_step, tokens/s, e2e (bf16 only),
+roofline, layer_roofline and clocks (each timed region lasts at least about
+a second, so the clocks are sampled inside it).
 Also: `e2e` (the same metric through moe_zc_forward_host: the
 step's input is copied from pinned host memory and its output back inside the
 timed region, in chunks whose copies overlap the kernels), `roofline` (the dominant kernel's achieved rate against the measured
@@ -79,7 +81,7 @@ NCU_TRAFFIC_RATIO = {
 }
 SUSTAINED_REGION_S = 2.0   # timed regions at least this long use the sustained bf16 peak
 NOMINAL_HBM_GBS = 7700.0   # B200 HBM3e, HGX figure (context beside the measured copy peak)
-EXTRA_WORKLOADS = "decode,small,skewed40"
+EXTRA_WORKLOADS = "decode,small,skewed40,decode_fp8,prefill_fp8"
 
 
 def gemm_sources_sha16():
@@ -266,18 +268,21 @@ def routing_stats(w, cnt):
                 max_load=int(ffn.max()) if w.N else 0)
 
 
-def roofline_numbers(w, st, pk):
-    """Algorithmic FLOPs and bytes of the layer and of its kernels."""
+def roofline_numbers(w, st, pk, fp8=False):
+    """Algorithmic FLOPs and bytes of the layer and of its kernels.  fp8: the
+    gate/up weights and permuted tokens are E4M3 bytes plus one scale byte
+    per 32 elements; the down projection stays bf16."""
     P, hit = st["ffn_pairs"], st["experts_hit"]
     d, I, T, E = w.d, w.I, w.T, w.E
+    gu = (1.0 + 1.0 / 32) if fp8 else 2.0      # bytes per gate/up weight or token element
     F_gateup = 4.0 * d * I * P
     F_down = 2.0 * d * I * P
-    B_gateup = hit * 2.0 * I * d * 2 + P * d * 2 + P * I * 2      # weights + Xp in + H out
+    B_gateup = hit * 2.0 * I * d * gu + P * d * gu + P * I * 2    # weights + Xp in + H out
     B_down = hit * 1.0 * I * d * 2 + P * I * 2 + P * d * 2        # weights + H in + Y out
     F_layer = F_gateup + F_down
-    B_layer = hit * 3.0 * d * I * 2 + E * d * 2 + E * 4 + 2.0 * T * d * 2
+    B_layer = hit * (2.0 * d * I * gu + d * I * 2) + E * d * 2 + E * 4 + 2.0 * T * d * 2
     return dict(F_gateup=F_gateup, F_down=F_down, B_gateup=B_gateup, B_down=B_down,
-                F_layer=F_layer, B_layer=B_layer)
+                F_layer=F_layer, B_layer=B_layer, fp8=fp8)
 
 
 # ----------------------------------------------------------------- oracle timing
@@ -326,16 +331,27 @@ def config_of(w, extra=None):
     return c
 
 
-def bf16_peak(pk, region_s):
+def bf16_peak(pk, region_s, clk=None):
     """The bf16 peak a kernel timed inside a region of region_s seconds is held
-    to: the burst figure for a short region, the sustained one (seconds of
-    back-to-back GEMMs under the power cap) for a long one."""
-    if region_s >= SUSTAINED_REGION_S:
+    to: the burst figure for a short region at full clocks, the sustained one
+    (seconds of back-to-back GEMMs under the power cap) for a long region or
+    one whose sampled SM clock sat below 90% of its maximum."""
+    capped = bool(clk and clk.get("sm_max_mhz") and clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"])
+    if region_s >= SUSTAINED_REGION_S or capped:
         return pk["bf16_sus"], f"bf16 dense, sustained ({pk['src']}, MEASURED_PEAKS.json)"
     return pk["bf16"], f"bf16 dense, burst ({pk['src']}, MEASURED_PEAKS.json)"
 
 
-def kernel_roofline(w, rf, plan, per, pk, region_s):
+def tensor_peak(pk, region_s, clk=None, fp8=False):
+    """bf16_peak, or for FP8 contractions that figure times 2 (the nominal
+    dense FP8 / bf16 ratio of B200: 4.5 / 2.25 PFLOP/s)."""
+    peak, kind = bf16_peak(pk, region_s, clk)
+    if fp8:
+        return 2.0 * peak, "FP8 dense = 2 x " + kind
+    return peak, kind
+
+
+def kernel_roofline(w, rf, plan, per, pk, region_s, clk=None):
     """The dominant stage's achieved rate against its bound."""
     dom = max(per, key=per.get)
     # (with the one-grid expert GEMMs the gate/up stage is the kernel that
@@ -348,7 +364,9 @@ def kernel_roofline(w, rf, plan, per, pk, region_s):
         return None
     F, B = kern
     sec = per[dom] / 1e3
-    peak, kind = bf16_peak(pk, region_s)
+    # the FP8 forward's gate/up GEMM runs FP8 MMAs (its one-grid kernel also
+    # the bf16 down tiles: held to the FP8 peak, the optimistic bound)
+    peak, kind = tensor_peak(pk, region_s, clk, rf.get("fp8") and dom == "gateup_gemm")
     t_tensor, t_hbm = F / (peak * 1e12), B / (pk["hbm"] * 1e9)
     if t_tensor >= t_hbm:
         ach = F / sec / 1e12
@@ -373,17 +391,23 @@ def kernel_roofline(w, rf, plan, per, pk, region_s):
     return roof
 
 
-def layer_roofline(rf, pk, ms, region_s):
-    """The whole layer: the slower of executed FFN FLOPs at the bf16 peak and
-    the bytes it must touch at the HBM peak, against the measured step."""
-    peak, kind = bf16_peak(pk, region_s)
-    t_f, t_b = rf["F_layer"] / (peak * 1e12), rf["B_layer"] / (pk["hbm"] * 1e9)
+def layer_roofline(rf, pk, ms, region_s, clk=None):
+    """The whole layer: the slower of executed FFN FLOPs at the tensor peak
+    (FP8: the gate/up FLOPs at the FP8 peak, the down FLOPs at bf16) and the
+    bytes it must touch at the HBM peak, against the measured step."""
+    peak, kind = bf16_peak(pk, region_s, clk)
+    if rf.get("fp8"):
+        t_f = (rf["F_gateup"] / 2.0 + rf["F_down"]) / (peak * 1e12)
+        kind = "gate/up at 2 x, down at 1 x " + kind
+    else:
+        t_f = rf["F_layer"] / (peak * 1e12)
+    t_b = rf["B_layer"] / (pk["hbm"] * 1e9)
     sec = ms / 1e3
     ffn_tflops = rf["F_layer"] / sec / 1e12
     hbm_gbs = rf["B_layer"] / sec / 1e9
     return {"bound": "tensor" if t_f >= t_b else "hbm", "roofline_ms": max(t_f, t_b) * 1e3,
             "frac": max(t_f, t_b) / sec, "bf16_peak_kind": kind,
-            "frac_vs_sustained_bf16": max(rf["F_layer"] / (pk["bf16_sus"] * 1e12), t_b) / sec,
+            "frac_vs_sustained_bf16": max(t_f * peak / pk["bf16_sus"], t_b) / sec,
             "executed_ffn_tflops": ffn_tflops,
             "pct_of_bf16_peak_burst": 100.0 * ffn_tflops / pk["bf16"],
             "pct_of_bf16_peak_sustained": 100.0 * ffn_tflops / pk["bf16_sus"],
@@ -391,10 +415,12 @@ def layer_roofline(rf, pk, ms, region_s):
             "pct_of_nominal_hbm": 100.0 * hbm_gbs / NOMINAL_HBM_GBS}
 
 
-def measure(args, dist, w, steps, e2e_steps, headline):
+def measure(args, dist, w, steps, e2e_steps, headline, fp8=False):
     """Time `steps` forwards of workload w (device-resident inputs), then the
     same with per-stage events, then e2e through the host-buffer entry point.
-    steps <= 0: as many as fill about one second (at least 20)."""
+    steps <= 0: as many as fill about one second (at least 20).  fp8: the
+    forward with FP8 gate/up (moe_zc_forward_fp8; weights quantised on the
+    device before timing; no host-buffer entry point, so no e2e)."""
     from mixture_experts_layer_28_b200 import moe_zc as mz
     pk = peaks()
     ri, b, ew, dev = make_inputs(w)
@@ -403,8 +429,16 @@ def measure(args, dist, w, steps, e2e_steps, headline):
     mz.reserve(w.T, w.d, w.N, w.Z, w.K, w.I)
     sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     plan = mz.plan(w.T, w.d, w.N, w.Z, w.K, w.I, sms=sms, resident_blocks=sms)
+    if fp8:
+        q_gate, q_up = mz.fp8_quantize_weights(ew.W_gate), mz.fp8_quantize_weights(ew.W_up)
+        torch.cuda.synchronize()
 
     def step(x=None, o=None):
+        if fp8:
+            mz.forward_fp8(dev["x"] if x is None else x, dev["W_r"], dev["b"], q_gate, q_up,
+                           ew.W_down, w.N, w.Z, w.K, out=out if o is None else o,
+                           logit_offset=dev["off"], stream=stream)
+            return
         mz.forward(dev["x"] if x is None else x, dev["W_r"], dev["b"], ew.W_gate, ew.W_up,
                    ew.W_down, w.N, w.Z, w.K, out=out if o is None else o,
                    logit_offset=dev["off"], stream=stream)
@@ -414,7 +448,7 @@ def measure(args, dist, w, steps, e2e_steps, headline):
     torch.cuda.synchronize()
     mz.synchronize()
     st = routing_stats(w, mz.expert_load(w.E))
-    rf = roofline_numbers(w, st, pk)
+    rf = roofline_numbers(w, st, pk, fp8=fp8)
     if steps <= 0:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -486,6 +520,8 @@ def measure(args, dist, w, steps, e2e_steps, headline):
     # ---- end to end through the host-buffer entry point: the step's input
     # goes from pinned host memory to the device and its output comes back,
     # in chunks whose copies overlap the kernels (moe_zc_forward_host)
+    if fp8:
+        e2e_steps = 0
     x_host = ri.x.pin_memory()
     out_host = torch.empty_like(x_host).pin_memory()
 
@@ -494,29 +530,32 @@ def measure(args, dist, w, steps, e2e_steps, headline):
                         w.N, w.Z, w.K, out_host=out_host, logit_offset=dev["off"],
                         chunk_tokens=args.chunk_tokens, stream=stream)
 
-    for _ in range(2):
-        step_host()
-    torch.cuda.synchronize()
-    dist.barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        step_host()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    dist.barrier()
-    e2e_ms = dist.max(e0.elapsed_time(e1) / e2e_steps)
-    mz.synchronize()
+    e2e_ms = None
+    if e2e_steps > 0:
+        for _ in range(2):
+            step_host()
+        torch.cuda.synchronize()
+        dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            step_host()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e2e_ms = dist.max(e0.elapsed_time(e1) / e2e_steps)
+        mz.synchronize()
 
     per = {k: v / max(nfw, 1) for k, v in stage_ms.items()}
     res = {
         "value": value, "ms_per_step": ms_max, "steps": steps,
-        "e2e": {"value": dist.world * w.T / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": int(x_host.numel() * 2),
-                "d2h_bytes_per_step": int(out_host.numel() * 2), "ms_per_step": e2e_ms,
-                "steps": e2e_steps},
-        "roofline": kernel_roofline(w, rf, plan, per, pk, region_s),
-        "layer_roofline": layer_roofline(rf, pk, ms_max, region_s),
+        "e2e": None if e2e_ms is None else {
+            "value": dist.world * w.T / (e2e_ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(x_host.numel() * 2),
+            "d2h_bytes_per_step": int(out_host.numel() * 2), "ms_per_step": e2e_ms,
+            "steps": e2e_steps},
+        "roofline": kernel_roofline(w, rf, plan, per, pk, region_s, clk),
+        "layer_roofline": layer_roofline(rf, pk, ms_max, region_s, clk),
         "gpu_launches": plan["kernels"] * steps,
         "clocks": clk,
         "routing": st,
@@ -559,10 +598,12 @@ def run_ours(args, dist, w):
         line["workloads"] = {}
     for name in extra:
         gc_collect()
-        wx = wl.get(name)
-        r = measure(args, dist, wx, 0, max(args.e2e_steps, 20), headline=False)
+        fp8 = name.endswith("_fp8")
+        wx = wl.get(name[:-4] if fp8 else name)
+        r = measure(args, dist, wx, 0, max(args.e2e_steps, 20), headline=False, fp8=fp8)
         r.pop("_keep")
         touched = r.pop("touched_bytes")
+        r["dtype"] = "fp8 gate/up (E4M3, 1x32 UE8M0 blocks), bf16 down" if fp8 else "bf16"
         r["config"] = config_of(wx, {
             "global_batch": wx.T * dist.world,
             "l2": (f"no flush: expert weights touched per step {touched / 1e9:.2f} GB"

@@ -191,8 +191,8 @@ int moe_zc_bias_controller_step(const int32_t* counts, int32_t N, int32_t Z, int
 /*
  * FP8 (E4M3) block quantisation of one weight matrix, on the host (write-up,
  * section "System-level optimisation": fine-grained block quantisation as in
- * DeepSeek-V3).  For an FP8 expert path: moe_zc_forward itself still takes
- * bf16 weights.
+ * DeepSeek-V3).  Host reference of the FP8 formats; moe_zc_forward_fp8 takes
+ * weights quantised on the device by moe_zc_fp8_quantize_weights.
  *   W       host bf16 [rows, cols], row-major (e.g. W_gate[e], [I, d])
  *   mode    MOE_ZC_FP8_BLOCK128: 128 x 128 blocks, scale = amax / 448 in fp32;
  *           MOE_ZC_FP8_MX32: 1 x 32 blocks along a row, scale = the smallest
@@ -238,6 +238,52 @@ typedef struct moe_zc_launch_plan {
 } moe_zc_launch_plan;
 int moe_zc_plan(int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I,
                 int32_t sms, int32_t resident_blocks, moe_zc_launch_plan* plan);
+
+/*
+ * FP8 (E4M3) quantisation of one weight matrix ON THE DEVICE, in the
+ * block-scaled form moe_zc_forward_fp8 takes (write-up, section
+ * "System-level optimisation": fine-grained block quantisation; the form is
+ * MOE_ZC_FP8_MX32's: 1 x 32 blocks along a row, scale = the smallest power of
+ * two with amax / scale <= 448, codes of W / scale rounded to nearest, ties to
+ * even; an all-zero or non-finite block gets scale 1).
+ *   W       device bf16 [rows, cols], row-major (e.g. all of W_gate as
+ *           [N * I, d]); rows % 128 == 0, cols % 128 == 0
+ *   codes   device uint8 [rows, cols]: the E4M3 codes
+ *   scales  device uint8 [rows * cols / 32]: each block's scale as a UE8M0
+ *           byte (2^(byte - 127); blocks with amax < 448 * 2^-127 take
+ *           byte 0), laid out in 512-byte atoms of 128 rows x 128 columns:
+ *           the byte of row r and 32-column block k sits at
+ *           ((r / 128) * (cols / 128) + k / 4) * 512 + (r % 32) * 16
+ *             + ((r % 128) / 32) * 4 + k % 4
+ *           (the order in which the tensor cores take scale factors)
+ * Asynchronous on `stream`; allocates nothing.  Codes and scales equal
+ * moe_zc_fp8_quantize(..., MOE_ZC_FP8_MX32, ...) of the same matrix (scales
+ * there as floats in row-major order).  Returns MOE_ZC_ERR_INVALID_ARG for
+ * null pointers or sizes < 1, MOE_ZC_ERR_UNSUPPORTED for sizes that are not
+ * multiples of 128 or pointers not 16-byte aligned.
+ */
+int moe_zc_fp8_quantize_weights(const void* W, int64_t rows, int32_t cols, void* codes,
+                                void* scales, void* stream);
+
+/*
+ * moe_zc_forward_ex with the gate and up projections in block-scaled FP8
+ * (write-up, section "System-level optimisation", quantisation paragraph:
+ * fine-grained block FP8, with the down projection -- whose input
+ * activations reach extreme magnitudes -- kept in higher precision).
+ * W_gate8 / W_up8 (device uint8 [N, I, d]) and W_gate_sf / W_up_sf are
+ * moe_zc_fp8_quantize_weights of W_gate / W_up taken as [N * I, d]; W_down
+ * stays bf16.  Each token's row is quantised the same way (1 x 32 blocks
+ * along d) by the forward itself; the gate/up GEMM runs the tensor cores'
+ * block-scaled FP8 MMA with fp32 accumulation; H, the down GEMM, the
+ * router and the combine are those of moe_zc_forward.  Requires d % 128 == 0
+ * besides moe_zc_forward's conditions.  The first FP8 forward on a device
+ * grows the workspace by the quantised tokens (their count, rounded as for
+ * the bf16 buffers, times d bytes) and their scales.
+ */
+int moe_zc_forward_fp8(const void* x, const void* W_r, const float* b, const void* W_gate8,
+                       const void* W_gate_sf, const void* W_up8, const void* W_up_sf,
+                       const void* W_down, int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K,
+                       int32_t I, const float* logit_offset, void* out, void* stream);
 
 /* Wait for the last forward; report (and clear) a device-side timeout. */
 int moe_zc_synchronize(void);

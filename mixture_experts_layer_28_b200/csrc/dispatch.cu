@@ -7,9 +7,10 @@
 //
 //   assign    first every CTA takes, from the expert-load histogram, each
 //             FFN expert's rows (count rounded up to 16) and token tiles
-//             (ceil(count / 256)); exclusive prefix sums give the expert's
-//             first row in the permuted buffers (grp_off) and its first GEMM
-//             token tile (grp_ttp), which CTA 0 also stores for the GEMMs
+//             (ceil(count / 256), and for the FP8 gate/up GEMM ceil(count /
+//             240)); exclusive prefix sums give the expert's first row in the
+//             permuted buffers (grp_off) and its first GEMM token tile
+//             (grp_ttp, grp_ttp8), which CTA 0 also stores for the GEMMs
 //             (the GEMM grid walks grp_ttp).  Then one thread per (token,
 //             pick): lanes of a warp that picked the same expert are grouped
 //             with __match_any_sync and take their slots with one atomicAdd
@@ -59,16 +60,16 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total
 __global__ void __launch_bounds__(ASSIGN_THREADS)
 assign_slots_kernel(const int* __restrict__ cnt, const int* __restrict__ idx, int64_t pairs,
                     int N, int* __restrict__ grp_off, int* __restrict__ grp_ttp,
-                    int* __restrict__ fill, int* __restrict__ slot) {
+                    int* __restrict__ fill, int* __restrict__ slot, int* __restrict__ grp_ttp8) {
   __shared__ int off_s[MOE_MAX_E_INTERNAL];
   __shared__ int warp_sums[32];
   griddep_wait();
   // experts' first rows (and, in CTA 0, first token tiles) from the histogram
-  int carry_rows = 0, carry_tiles = 0;
+  int carry_rows = 0, carry_tiles = 0, carry_tiles8 = 0;
   for (int base = 0; base < N; base += ASSIGN_THREADS) {
     const int g = base + threadIdx.x;
     const int c = g < N ? cnt[g] : 0;
-    int tot_rows, tot_tiles = 0;
+    int tot_rows, tot_tiles = 0, tot_tiles8 = 0;
     const int off = block_excl_scan((c + 15) & ~15, warp_sums, &tot_rows);
     if (g < N) off_s[g] = carry_rows + off;
     if (blockIdx.x == 0) {
@@ -77,13 +78,19 @@ assign_slots_kernel(const int* __restrict__ cnt, const int* __restrict__ idx, in
         grp_off[g] = carry_rows + off;
         grp_ttp[g] = carry_tiles + ttp;
       }
+      if (grp_ttp8) {   // (uniform over the CTA)
+        const int t8 = block_excl_scan((c + FP8_BN - 1) / FP8_BN, warp_sums, &tot_tiles8);
+        if (g < N) grp_ttp8[g] = carry_tiles8 + t8;
+      }
     }
     carry_rows += tot_rows;
     carry_tiles += tot_tiles;
+    carry_tiles8 += tot_tiles8;
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     grp_off[N] = carry_rows;
     grp_ttp[N] = carry_tiles;
+    if (grp_ttp8) grp_ttp8[N] = carry_tiles8;
   }
   __syncthreads();
 
@@ -146,10 +153,10 @@ cudaError_t launch_add_counts(const int* cnt, int E, int* total, cudaStream_t st
 
 cudaError_t launch_assign_slots(const int* cnt, const int* idx, int64_t pairs, int N,
                                 int* grp_off, int* grp_ttp, int* fill, int* slot,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, int* grp_ttp8) {
   const int64_t blocks = pairs > 0 ? (pairs + ASSIGN_THREADS - 1) / ASSIGN_THREADS : 1;
   return launch_pdl(assign_slots_kernel, dim3(static_cast<unsigned>(blocks)), dim3(ASSIGN_THREADS),
-                    0, stream, cnt, idx, pairs, N, grp_off, grp_ttp, fill, slot);
+                    0, stream, cnt, idx, pairs, N, grp_off, grp_ttp, fill, slot, grp_ttp8);
 }
 
 cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, int d, int K,

@@ -68,6 +68,7 @@ struct Tile {
   int ntt;      // token tiles of the group
   bool has_a1;  // second A block present
   int a0_row, a1_row;
+  int ttile;    // expert GEMMs: the tile's index among all token tiles (FP8 scale atoms)
 };
 
 __device__ __forceinline__ int router_tok_tile(const GemmParams& p) {
@@ -139,17 +140,16 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
     tl.count = __ldg(p.grp_count + lo);
     tl.brow0 = __ldg(p.grp_off + lo);
   }
-  // An expert's ntt = ceil(count / 256) token tiles share its tokens evenly
+  // An expert's ntt = ceil(count / tile) token tiles share its tokens evenly
   // (sizes a multiple of 16): two tiles of similar size run side by side in
   // one round of the persistent grid and read the same weight blocks at the
-  // same pace, so the second read of a block is an L2 hit.
-  int tsz = MODE == MODE_ROUTER ? router_tok_tile(p) : GEMM_BN;
+  // same pace, so the second read of a block is an L2 hit.  (tile: GEMM_BN,
+  // or FP8_BN for the FP8 gate/up GEMM, whose p.tok_tile says so.)
+  int tsz = router_tok_tile(p);
+  tl.ttile = 0;
   if (MODE != MODE_ROUTER) {
-    const int ntt = __ldg(p.grp_ttp + tl.g + 1) - __ldg(p.grp_ttp + tl.g);
-    if (ntt > 1) {
-      const int even = (((tl.count + ntt - 1) / ntt) + 15) & ~15;
-      if (static_cast<long long>(ntt - 1) * even < tl.count) tsz = even;   // last tile non-empty
-    }
+    tsz = even_tile_size(tl.count, tl.ntt, tsz);
+    tl.ttile = __ldg(p.grp_ttp + tl.g) + j;
   }
   tl.tok0 = j * tsz;
   tl.ntok = min(tsz, tl.count - tl.tok0);
@@ -220,16 +220,46 @@ __device__ __forceinline__ void mma_kstep(uint32_t d, uint32_t a_smem, uint32_t 
     umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (first && kk == 0) ? 0u : 1u);
 }
 
+// FP8 (block-scaled) gate/up tiles keep their scale factors in TMEM columns
+// SF_TMEM_COL.. (behind the two FP8_BN-column accumulators): W_gate's atom
+// at +0, W_up's at +4, the token tile's at +8 (tokens 0..127) and +12
+// (128..239).  One set serves the stage whose MMAs come next: a
+// tcgen05.cp and the tcgen05.mma issued after it by the same thread run in
+// issue order, so each stage's copies simply precede its MMAs.
+constexpr uint32_t SF_TMEM_COL = 2 * FP8_BN;
+static_assert(SF_TMEM_COL + 16 <= 512, "scale-factor columns exceed TMEM");
+
+__device__ __forceinline__ void sf_to_tmem(uint32_t sf_t, uint32_t sf_smem, bool two_tok) {
+  tmem_cp_atom(sf_t, smem_desc_atom(sf_smem));
+  tmem_cp_atom(sf_t + 4, smem_desc_atom(sf_smem + SF_ATOM_BYTES));
+  tmem_cp_atom(sf_t + 8, smem_desc_atom(sf_smem + 2 * SF_ATOM_BYTES));
+  if (two_tok) tmem_cp_atom(sf_t + 12, smem_desc_atom(sf_smem + 3 * SF_ATOM_BYTES));
+}
+
+// One FP8 stage (128 contraction elements) of one A block: four K = 32
+// block-scaled MMAs into accumulator d, the k-th taking byte k of the scale
+// words at sfa_t (the A block's rows) and sfb_t (the tokens).
+__device__ __forceinline__ void mma_kstep_fp8(uint32_t d, uint32_t a_smem, uint32_t b_smem,
+                                              uint32_t nmma, uint32_t sfa_t, uint32_t sfb_t,
+                                              bool first) {
+  const uint64_t ad = smem_desc_sw128(a_smem);
+  const uint64_t bd = smem_desc_sw128(b_smem);
+#pragma unroll
+  for (uint32_t kb = 0; kb < FP8_BK / 32; ++kb)
+    umma_mxf8(d, ad + 2 * kb, bd + 2 * kb, idesc_mxf8(GEMM_BM, nmma, kb, kb), sfa_t, sfb_t,
+              (first && kb == 0) ? 0u : 1u);
+}
+
 // The epilogue chunks of warp group `group` (0..2) in its lane quadrant:
 // columns group * 32 + j * 96 (j = 0..2) below nmma, 32 wide (16 for a
 // ragged last chunk).
 //
 // Reads this warp's chunks of the accumulator at tacc (for gate/up also the
-// up accumulator 256 columns on), applies the epilogue math and rounds to
+// up accumulator acc1 columns on), applies the epilogue math and rounds to
 // bf16: hp[j][i] holds tokens 2i and 2i+1 of chunk j.
 template <int MODE>
 __device__ __forceinline__ void epi_read_bf16(uint32_t tacc, int group, int nmma,
-                                              uint32_t (&hp)[3][16]) {
+                                              uint32_t (&hp)[3][16], uint32_t acc1 = 256) {
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
     const int c0 = group * 32 + j * 32 * GEMM_EPI_GROUPS;
@@ -239,7 +269,7 @@ __device__ __forceinline__ void epi_read_bf16(uint32_t tacc, int group, int nmma
       if (cc < nmma) {
         uint32_t r0[16], r1[16];
         tmem_ld16(tacc + cc, r0);
-        if (MODE == MODE_GATEUP) tmem_ld16(tacc + 256 + cc, r1);
+        if (MODE == MODE_GATEUP) tmem_ld16(tacc + acc1 + cc, r1);
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -314,7 +344,7 @@ __device__ __forceinline__ void epi_router_f32(uint32_t tacc, uint8_t* stg, int 
 // holds all its gate/up tiles before its down tiles, gate/up tiles wait on
 // nothing outside their CTA, and the grid (one CTA per SM, at most one per
 // SM of the device) is resident as a whole.
-template <int MODE, int NST, int SB>
+template <int MODE, int NST, int SB, bool FP8>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
             const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBf,
@@ -419,7 +449,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         // group tl.g's H rows are all stored once every epilogue warp of its
         // gate/up tiles has counted itself; the acquire and the proxy fence
         // order this CTA's bulk copies of them after those stores
-        const int need = GEMM_EPI_WARPS * p.mblocks * tl.ntt;
+        const int need =
+            GEMM_EPI_WARPS * p.mblocks * (__ldg(p.grp_ttp + tl.g + 1) - __ldg(p.grp_ttp + tl.g));
         if (!wait_count_geq(p.done + tl.g, need, p.wait_ns, p.err)) {
           abort_sh = 1;
           break;
@@ -437,13 +468,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         st_cluster_u32(peer_word, begun);
         pace_until_shared(&peer_tile_sh, begun, PACE_NS);
       }
+      // FP8 kernels run their gate/up tiles in FP8 (MODE_FUSED's down tiles
+      // stay bf16): 128 contraction elements per stage instead of 64, in the
+      // same 128-byte rows, plus the stage's scale atoms
+      const bool f8 = FP8 && !down_ph;
       const int nbox = (tl.nmma + GEMM_B_BOX_ROWS - 1) / GEMM_B_BOX_ROWS;
-      // a full token tile (256 tokens; the router's tile size) in one copy
-      // of the b_full map, whose box has exactly that many rows
-      const int full_rows = MODE == MODE_ROUTER ? router_tok_tile(p) : GEMM_BN;
+      // a full token tile (the tile size: 256 tokens, 240 for FP8, the
+      // router's own) in one copy of the b_full map, whose box has exactly
+      // that many rows
+      const int full_rows = router_tok_tile(p);
       const bool full_box = MODE != MODE_FUSED && p.b_box_full && tl.nmma == full_rows;
+      const int sfb_atoms = tl.nmma > 128 ? 2 : 1;
       const uint32_t bytes = GEMM_A_BYTES * (tl.has_a1 ? 2 : 1) +
-                             (full_box ? tl.nmma : nbox * GEMM_B_BOX_ROWS) * GEMM_BK * 2;
+                             (full_box ? tl.nmma : nbox * GEMM_B_BOX_ROWS) * 128 +
+                             (f8 ? (2 + sfb_atoms) * SF_ATOM_BYTES : 0);
+      const int kstep = f8 ? FP8_BK : GEMM_BK;
       for (int ks = tl.k0; ks < tl.k1; ++ks) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1, p.wait_ns, p.err)) {
           abort_sh = 1;
@@ -453,7 +492,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         mbar_arrive_expect_tx(&full_bar[stage], bytes);
         armed |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (phase << stage);
-        const int kc = ks * GEMM_BK;
+        const int kc = ks * kstep;
         // Streaming batches (decode) read every weight byte once: evict
         // first.  Prefill-sized batches keep the default policy (measured:
         // evict-last weights or evict-first tokens there cost ~4%).
@@ -480,6 +519,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                           tl.brow0 + bx * GEMM_B_BOX_ROWS);
           }
         }
+        if (f8) {
+          // scale atoms: W_gate's and W_up's 128 rows of this block, and the
+          // token tile's one or two atoms, for these 4 blocks of 32
+          uint8_t* sf = st + (SB - FP8_SF_STAGE_BYTES);
+          const int64_t wa =
+              (static_cast<int64_t>(tl.a0_row / GEMM_BM) * p.sf_kgroups + ks) * SF_ATOM_BYTES;
+          bulk_load(sf, p.sfa0 + wa, SF_ATOM_BYTES, &full_bar[stage]);
+          bulk_load(sf + SF_ATOM_BYTES, p.sfa1 + wa, SF_ATOM_BYTES, &full_bar[stage]);
+          const int64_t tb =
+              (static_cast<int64_t>(tl.ttile) * p.sf_kgroups + ks) * (2 * SF_ATOM_BYTES);
+          bulk_load(sf + 2 * SF_ATOM_BYTES, p.sfb + tb, sfb_atoms * SF_ATOM_BYTES,
+                    &full_bar[stage]);
+        }
         if (++stage == NST) { stage = 0; phase ^= 1; }
       }
     }
@@ -499,7 +551,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       const Tile tl = phase_tile<MODE>(p, p2, tph, t);
       const int buf = local % nbuf;
       const int use = local / nbuf;
-      (void)tph;
       const uint32_t par = static_cast<uint32_t>(use - 1) & 1u;
       const uint32_t acc0 = tmem + buf * 256;
       if (use > 0 && !mbar_wait(&acc_empty_bar[buf], par, p.wait_ns, p.err)) {
@@ -509,9 +560,36 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       tc_fence_after();
       const uint32_t idesc = idesc_bf16_f32(GEMM_BM, tl.nmma);
       const int nk = tl.k1 - tl.k0;
+      // FP8 gate/up tiles: block-scaled MMAs, the second accumulator FP8_BN
+      // columns on (two FP8_BN-token accumulators and the scale columns fill
+      // TMEM); bf16 tiles: 256 columns on
+      const bool f8 = FP8 && !(MODE == MODE_FUSED && tph == 1);
+      const uint32_t acc1 = acc0 + (f8 ? FP8_BN : 256);
+      const uint32_t sf_t = tmem + SF_TMEM_COL;
+      const bool two_tok = tl.nmma > 128;
+      constexpr uint32_t SF_OFF = SB - FP8_SF_STAGE_BYTES;
+      // first / second accumulator's k-step on the stage at st
+      auto kstep0 = [&](uint32_t st, bool first) {
+        if (f8) {
+          sf_to_tmem(sf_t, st + SF_OFF, two_tok);
+          mma_kstep_fp8(acc0, st, st + 2 * GEMM_A_BYTES, tl.nmma, sf_t, sf_t + 8, first);
+        } else {
+          mma_kstep(acc0, st, st + 2 * GEMM_A_BYTES, idesc, first);
+        }
+      };
+      auto kstep1 = [&](uint32_t st, bool first, bool copy_sf) {
+        if (f8) {
+          if (copy_sf) sf_to_tmem(sf_t, st + SF_OFF, two_tok);
+          mma_kstep_fp8(acc1, st + GEMM_A_BYTES, st + 2 * GEMM_A_BYTES, tl.nmma, sf_t + 4,
+                        sf_t + 8, first);
+        } else {
+          mma_kstep(acc1, st + GEMM_A_BYTES, st + 2 * GEMM_A_BYTES, idesc, first);
+        }
+      };
       // Two-block tile after the first: the first npre loaded stages feed the
       // first accumulator alone; they are freed once the second accumulator
-      // is back and has had its MMAs on them too.
+      // is back and has had its MMAs on them too (FP8: with their scale
+      // atoms copied into TMEM again).
       const bool stagger = nbuf == 1 && use > 0;
       const int npre = stagger ? min(nk, NST) : 0;
       bool ok = true;
@@ -519,8 +597,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       for (int i = 0; i < npre; ++i) {
         if (!mbar_wait(&full_bar[stage], phase, p.wait_ns, p.err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t st = smem_u32(smem + stage * SB);
-        mma_kstep(acc0, st, st + 2 * GEMM_A_BYTES, idesc, i == 0);
+        kstep0(smem_u32(smem + stage * SB), i == 0);
         if (++stage == NST) { stage = 0; phase ^= 1; }
       }
       if (ok && stagger) {
@@ -530,8 +607,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
           tc_fence_after();
           int s = stage0;
           for (int i = 0; i < npre; ++i) {
-            const uint32_t st = smem_u32(smem + s * SB);
-            if (tl.has_a1) mma_kstep(acc0 + 256, st + GEMM_A_BYTES, st + 2 * GEMM_A_BYTES, idesc, i == 0);
+            if (tl.has_a1) kstep1(smem_u32(smem + s * SB), i == 0, true);
             umma_commit(&empty_bar[s]);
             if (++s == NST) s = 0;
           }
@@ -541,8 +617,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         if (!mbar_wait(&full_bar[stage], phase, p.wait_ns, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = smem_u32(smem + stage * SB);
-        mma_kstep(acc0, st, st + 2 * GEMM_A_BYTES, idesc, i == 0);
-        if (tl.has_a1) mma_kstep(acc0 + 256, st + GEMM_A_BYTES, st + 2 * GEMM_A_BYTES, idesc, i == 0);
+        kstep0(st, i == 0);
+        if (tl.has_a1) kstep1(st, i == 0, false);
         umma_commit(&empty_bar[stage]);
         if (++stage == NST) { stage = 0; phase ^= 1; }
       }
@@ -592,7 +668,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         }
       } else if (MODE == MODE_GATEUP || (MODE == MODE_FUSED && !down_ph)) {
         uint32_t hp[3][16];
-        epi_read_bf16<MODE_GATEUP>(tacc, group, tl.nmma, hp);
+        epi_read_bf16<MODE_GATEUP>(tacc, group, tl.nmma, hp, FP8 ? FP8_BN : 256);
         tc_fence_before();
         mbar_arrive(&acc_empty_bar[0]);
         mbar_arrive(&acc_empty_bar[1]);
@@ -643,27 +719,27 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
 }
 
 // a2, b2, p2: MODE_FUSED's down phase (other modes: copies of a0, b, p).
-template <int MODE, int NST, int SB>
+template <int MODE, int NST, int SB, bool FP8 = false>
 cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                         const CUtensorMap& b_full, const CUtensorMap& a2, const CUtensorMap& b2,
                         GemmParams p, const GemmParams& p2, int grid, cudaStream_t stream) {
   constexpr int smem = NST * SB + GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024;
-  const cudaError_t e = smem_limit<gemm_kernel<MODE, NST, SB>>(smem);
+  const cudaError_t e = smem_limit<gemm_kernel<MODE, NST, SB, FP8>>(smem);
   if (e != cudaSuccess) return e;
   // pacing runs the grid as 2-CTA clusters: an even grid of at least two
   if (p.pair_tiles) {
     if (grid >= 2) {
-      return launch_pdl_pairs(gemm_kernel<MODE, NST, SB>, dim3(grid & ~1), dim3(GEMM_THREADS),
-                              smem, stream, a0, a1, b, b_full, a2, b2, p, p2);
+      return launch_pdl_pairs(gemm_kernel<MODE, NST, SB, FP8>, dim3(grid & ~1),
+                              dim3(GEMM_THREADS), smem, stream, a0, a1, b, b_full, a2, b2, p, p2);
     }
     p.pair_tiles = 0;
   }
   // a down tile of the one grid may wait for any other block's gate/up
   // tiles: every block must be resident at once
   if (MODE == MODE_FUSED)
-    return launch_pdl_coop(gemm_kernel<MODE, NST, SB>, dim3(grid), dim3(GEMM_THREADS), smem,
+    return launch_pdl_coop(gemm_kernel<MODE, NST, SB, FP8>, dim3(grid), dim3(GEMM_THREADS), smem,
                            stream, a0, a1, b, b_full, a2, b2, p, p2);
-  return launch_pdl(gemm_kernel<MODE, NST, SB>, dim3(grid), dim3(GEMM_THREADS), smem, stream,
+  return launch_pdl(gemm_kernel<MODE, NST, SB, FP8>, dim3(grid), dim3(GEMM_THREADS), smem, stream,
                     a0, a1, b, b_full, a2, b2, p, p2);
 }
 
@@ -722,14 +798,44 @@ cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, cons
 int fused_resident_blocks() {
   constexpr int smem = GEMM_SMALL_STAGES * GEMM_SMALL_STAGE_BYTES +
                        GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024;
-  if (smem_limit<gemm_kernel<MODE_FUSED, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>>(smem) !=
-      cudaSuccess) {
+  if (smem_limit<gemm_kernel<MODE_FUSED, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES, false>>(
+          smem) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
-  return blocks_per_sm<gemm_kernel<MODE_FUSED, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>>(
+  return blocks_per_sm<gemm_kernel<MODE_FUSED, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES, false>>(
              GEMM_THREADS, smem) *
          device_sms();
+}
+
+cudaError_t launch_gemm_gateup_fp8(const CUtensorMap& wg, const CUtensorMap& wu,
+                                   const CUtensorMap& xp8, const CUtensorMap& xp8_full,
+                                   const GemmParams& p, int grid, cudaStream_t stream) {
+  if (grid <= 0) return cudaSuccess;
+  if (p.tok_tile != FP8_BN || !p.sfa0 || !p.sfa1 || !p.sfb || p.sf_kgroups != p.ksteps)
+    return cudaErrorInvalidValue;
+  cudaError_t e;
+  if (p.small_b)
+    e = launch_mode<MODE_GATEUP, FP8_SMALL_STAGES, FP8_SMALL_STAGE_BYTES, true>(
+        wg, wu, xp8, xp8_full, wg, xp8, p, p, grid, stream);
+  else
+    e = launch_mode<MODE_GATEUP, GEMM_STAGES, FP8_STAGE_BYTES, true>(wg, wu, xp8, xp8_full, wg,
+                                                                      xp8, p, p, grid, stream);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_fused_fp8(const CUtensorMap& wg, const CUtensorMap& wu,
+                                  const CUtensorMap& xp8, const CUtensorMap& wd,
+                                  const CUtensorMap& h, const GemmParams& pg,
+                                  const GemmParams& pd, int grid, cudaStream_t stream) {
+  if (grid <= 0) return cudaSuccess;
+  if (grid > device_sms() || !pg.small_b || pg.pair_tiles || pg.b_box_full || pd.single_a ||
+      pg.done == nullptr || pg.tok_tile != FP8_BN || !pg.sfa0 || !pg.sfa1 || !pg.sfb ||
+      pg.sf_kgroups != pg.ksteps)
+    return cudaErrorInvalidValue;
+  return launch_mode<MODE_FUSED, FP8_SMALL_STAGES, FP8_SMALL_STAGE_BYTES, true>(
+      wg, wu, xp8, xp8, wd, h, pg, pd, grid, stream);
 }
 
 }  // namespace moezc

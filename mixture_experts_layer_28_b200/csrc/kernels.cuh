@@ -191,6 +191,14 @@ struct GemmParams {
   // first (about a gate/up tile's cost in down tiles).
   int* done;
   int down_lead;
+  // FP8 gate/up (block-scaled E4M3, FP8_BK contraction elements per stage):
+  // the UE8M0 scale atoms of W_gate and W_up (rows of the weight matrices,
+  // sf_atom_offset with kgroups = sf_kgroups) and of the token tiles (sfb:
+  // two atoms per tile and contraction group, as launch_permute_fp8 writes).
+  const uint8_t* sfa0;
+  const uint8_t* sfa1;
+  const uint8_t* sfb;
+  int sf_kgroups;         // contraction length / FP8_BK
 };
 
 // b: B map with GEMM_B_BOX_ROWS-row boxes; b_full: with GEMM_BN-row boxes,
@@ -209,9 +217,75 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
 cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, const CUtensorMap& xp,
                               const CUtensorMap& wd, const CUtensorMap& h, const GemmParams& pg,
                               const GemmParams& pd, int grid, cudaStream_t stream);
+// The FP8 gate/up GEMM (E4M3 maps of W_gate, W_up [N*I, d] with [128 x 128]
+// boxes and of the quantised tokens Xp8 with [128 x 32] boxes, b_full with
+// FP8_BN-row boxes; p.tok_tile = FP8_BN, p.grp_ttp the FP8_BN-tile prefix,
+// p.ksteps = d / FP8_BK, scale atoms in p.sfa0 / p.sfa1 / p.sfb).
+cudaError_t launch_gemm_gateup_fp8(const CUtensorMap& wg, const CUtensorMap& wu,
+                                   const CUtensorMap& xp8, const CUtensorMap& xp8_full,
+                                   const GemmParams& p, int grid, cudaStream_t stream);
+// launch_gemm_fused with the gate/up phase in FP8 (maps and parameters as for
+// launch_gemm_gateup_fp8); the down phase stays bf16.
+cudaError_t launch_gemm_fused_fp8(const CUtensorMap& wg, const CUtensorMap& wu,
+                                  const CUtensorMap& xp8, const CUtensorMap& wd,
+                                  const CUtensorMap& h, const GemmParams& pg,
+                                  const GemmParams& pd, int grid, cudaStream_t stream);
 // Blocks of the one-grid expert GEMM kernel the current device holds at once
 // (its occupancy times the multiprocessors).
 int fused_resident_blocks();
+
+// ------------------------------------------------------------------ FP8 gate/up
+// Block-scaled FP8 (E4M3 elements, one power-of-two scale per 32 elements
+// along the contraction, stored as a UE8M0 exponent byte: 2^(byte - 127)).
+// The gate/up GEMM's scale factors reach the tensor cores through TMEM in
+// 512-byte atoms: 128 rows x 4 consecutive 32-element blocks, the byte of row
+// r and block k at (r % 32) * 16 + (r / 32) * 4 + k.
+constexpr int FP8_BK = 128;            // contraction elements per pipeline stage (128-byte rows)
+constexpr int FP8_BN = 240;            // tokens per gate/up tile (2 x 240 accumulator columns
+                                       // + 16 scale-factor columns fill TMEM's 512)
+constexpr int SF_ATOM_BYTES = 512;
+constexpr int FP8_SF_STAGE_BYTES = 4 * SF_ATOM_BYTES;   // gate atom, up atom, two token atoms
+constexpr int FP8_STAGE_BYTES = 2 * GEMM_A_BYTES + FP8_BN * FP8_BK + FP8_SF_STAGE_BYTES;
+constexpr int FP8_SMALL_STAGES = 4;
+constexpr int FP8_SMALL_STAGE_BYTES =
+    ((2 * GEMM_A_BYTES + GEMM_SMALL_B * FP8_BK + 3 * SF_ATOM_BYTES) + 1023) & ~1023;
+static_assert(3 * FP8_STAGE_BYTES + GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024 <= 227 * 1024,
+              "FP8 stages exceed shared memory");
+static_assert(FP8_SMALL_STAGES * FP8_SMALL_STAGE_BYTES + GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024 <=
+                  227 * 1024,
+              "FP8 small-batch stages exceed shared memory");
+
+// Tokens per token tile of an expert with `count` tokens cut into ntt tiles of
+// at most tmax: the tiles share the tokens evenly (a multiple of 16 each),
+// unless that would leave the last tile empty.
+__host__ __device__ __forceinline__ int even_tile_size(int count, int ntt, int tmax) {
+  if (ntt > 1) {
+    const int even = (((count + ntt - 1) / ntt) + 15) & ~15;
+    if (static_cast<long long>(ntt - 1) * even < count) return even;
+  }
+  return tmax;
+}
+
+// Byte offset, in a matrix's scale-factor atoms, of row r and contraction
+// block kb (of 32 elements) when the matrix has kgroups = cols / 128 groups.
+__host__ __device__ __forceinline__ int64_t sf_atom_offset(int64_t r, int kb, int kgroups) {
+  return ((r / 128) * kgroups + kb / 4) * SF_ATOM_BYTES + (r % 32) * 16 + ((r % 128) / 32) * 4 +
+         (kb % 4);
+}
+
+// W [rows, cols] bf16 (rows % 128 == 0, cols % 128 == 0) -> E4M3 codes
+// [rows, cols] and UE8M0 scales in atoms (sf_atom_offset).
+cudaError_t launch_fp8_quantize_weights(const __nv_bfloat16* W, int64_t rows, int cols,
+                                        uint8_t* codes, uint8_t* sf, cudaStream_t stream);
+// The FP8 permute: each token row is quantised once (E4M3 codes, 1 x 32
+// blocks) and written to its FFN slots of Xp8; its scales go to the atoms of
+// the gate/up token tiles holding those slots: tile j of expert g (FP8_BN
+// token tiles, first tile grp_ttp8[g]) at sfx + (tile * d / 128 + kg) * 1024,
+// the tile's token n as atom row n (two atoms: tokens 0..127, 128..239).
+cudaError_t launch_permute_fp8(const __nv_bfloat16* x, const int* idx, const int* slot,
+                               const int* cnt, const int* grp_off, const int* grp_ttp8, int64_t T,
+                               int d, int K, int N, uint8_t* Xp8, uint8_t* sfx,
+                               cudaStream_t stream);
 
 // ------------------------------------------------------------------ router
 // softmax over E logits (+offset), + bias, top-K, zero-gate sums, histogram.
@@ -225,9 +299,10 @@ cudaError_t launch_route(const float* logits, const float* b, const float* offse
 // Slot assignment with the experts' row and tile offsets (grp_off, grp_ttp
 // [N + 1], written by CTA 0) computed from the histogram cnt; fill [N] must
 // be zero on entry (the router GEMM clears it).
+// grp_ttp8 (optional, [N + 1]): the same prefix for FP8_BN-token tiles.
 cudaError_t launch_assign_slots(const int* cnt, const int* idx, int64_t pairs, int N,
                                 int* grp_off, int* grp_ttp, int* fill, int* slot,
-                                cudaStream_t stream);
+                                cudaStream_t stream, int* grp_ttp8 = nullptr);
 // total[j] += cnt[j] for j < E (histogram summed over the chunks of a forward)
 cudaError_t launch_add_counts(const int* cnt, int E, int* total, cudaStream_t stream);
 cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, int d, int K,

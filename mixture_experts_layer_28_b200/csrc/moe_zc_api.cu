@@ -46,6 +46,9 @@ struct Ctx {
   bool init = false;
   int sms = 0;
   Buf logits, idx, gate, zsum, slot, cnt, fill, grp_off, grp_ttp, Xp, H, Y, err;
+  // FP8 gate/up forwards: quantised tokens, their scale atoms per token tile,
+  // and the experts' first FP8_BN-token tiles
+  Buf Xp8, sfx, grp_ttp8;
   // host-buffer forwards: device staging for two chunks in and out, the
   // histogram summed over chunks, copy streams and their events
   Buf xin[2], yout[2], cnt_total;
@@ -114,6 +117,20 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t k, uint3
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D E4M3 (one byte per element) tensor [rows, k], box [box_rows, 128]
+// (128-byte rows like the bf16 maps' 64 elements), 128-byte swizzle.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t k, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {k, rows};
+  cuuint64_t strides[1] = {k};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(FP8_BK), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -219,7 +236,8 @@ struct Plan {
 };
 bool g_one_grid_off = false;    // test hook: never use the one grid
 
-Plan make_plan(int64_t T, int d, int N, int Z, int K, int I, int sms, int64_t resident) {
+Plan make_plan(int64_t T, int d, int N, int Z, int K, int I, int sms, int64_t resident,
+               bool fp8 = false) {
   Plan pl;
   const int E = N + Z;
   pl.rp = router_plan(T, E, d / GEMM_BK, sms);
@@ -231,7 +249,9 @@ Plan make_plan(int64_t T, int d, int N, int Z, int K, int I, int sms, int64_t re
     return pl;
   }
   const int64_t tiles_ub = (T * K + GEMM_BN - 1) / GEMM_BN + N;
-  const int64_t g_ub = tiles_ub * (I / GEMM_BM);
+  // (the FP8 gate/up GEMM cuts tokens into FP8_BN-token tiles)
+  const int64_t g_tiles_ub = fp8 ? (T * K + FP8_BN - 1) / FP8_BN + N : tiles_ub;
+  const int64_t g_ub = g_tiles_ub * (I / GEMM_BM);
   const int64_t d_ub = tiles_ub * ((d + 2 * GEMM_BM - 1) / (2 * GEMM_BM));
   pl.gateup_grid = g_ub < sms ? g_ub : sms;
   pl.down_grid = d_ub < sms ? d_ub : sms;
@@ -241,7 +261,7 @@ Plan make_plan(int64_t T, int d, int N, int Z, int K, int I, int sms, int64_t re
   return pl;
 }
 
-int reserve_impl(Ctx& c, int64_t T, int d, int N, int Z, int K, int I) {
+int reserve_impl(Ctx& c, int64_t T, int d, int N, int Z, int K, int I, bool fp8 = false) {
   const int64_t E = static_cast<int64_t>(N) + Z;
   const int64_t pairs = T * K;
   const int64_t rows_cap = N > 0 ? pairs + 15LL * N + 16 : 16;
@@ -268,6 +288,15 @@ int reserve_impl(Ctx& c, int64_t T, int d, int N, int Z, int K, int I) {
     if ((s = ensure(c, c.Xp, static_cast<size_t>(rows_cap) * d * 2)) != MOE_ZC_OK) return s;
     if ((s = ensure(c, c.H, static_cast<size_t>(rows_cap) * I * 2)) != MOE_ZC_OK) return s;
     if ((s = ensure(c, c.Y, static_cast<size_t>(rows_cap) * d * 2)) != MOE_ZC_OK) return s;
+  }
+  if (fp8 && N > 0) {
+    const int64_t tiles8 = (pairs + FP8_BN - 1) / FP8_BN + N;
+    if ((s = ensure(c, c.Xp8, static_cast<size_t>(rows_cap) * d)) != MOE_ZC_OK) return s;
+    if ((s = ensure(c, c.sfx, static_cast<size_t>(tiles8) * (d / FP8_BK) * 2 * SF_ATOM_BYTES)) !=
+        MOE_ZC_OK)
+      return s;
+    if ((s = ensure(c, c.grp_ttp8, static_cast<size_t>(N + 1) * sizeof(int))) != MOE_ZC_OK)
+      return s;
   }
   c.rows_cap = rows_cap;
   return MOE_ZC_OK;
@@ -355,15 +384,35 @@ int queue_load_hints(Ctx& c, const int* cnt, int N, cudaStream_t st) {
   return MOE_ZC_OK;
 }
 
+// FP8 gate/up weights of moe_zc_forward_fp8: E4M3 codes of W_gate and W_up
+// (where the bf16 forward takes the bf16 matrices) and their scale atoms.
+struct Fp8Gates {
+  const uint8_t* gate_sf;
+  const uint8_t* up_sf;
+};
+
+int check_fp8(const Fp8Gates* f8, int d, int N) {
+  if (!f8 || N == 0) return MOE_ZC_OK;
+  if (!f8->gate_sf || !f8->up_sf) return MOE_ZC_ERR_INVALID_ARG;
+  if (d % FP8_BK != 0) return MOE_ZC_ERR_UNSUPPORTED;   // whole 128-element stages
+  if (!aligned16(f8->gate_sf) || !aligned16(f8->up_sf)) return MOE_ZC_ERR_UNSUPPORTED;
+  return MOE_ZC_OK;
+}
+
+// f8: NULL for the bf16 forward; else W_gate / W_up hold E4M3 codes and f8
+// their scales (the FP8 gate/up GEMM; the down projection stays bf16).
 int forward_impl(const void* x, const void* W_r, const float* b, const void* W_gate,
                  const void* W_up, const void* W_down, int64_t T, int32_t d, int32_t N,
-                 int32_t Z, int32_t K, int32_t I, const float* off, void* out, void* stream) {
+                 int32_t Z, int32_t K, int32_t I, const float* off, void* out, void* stream,
+                 const Fp8Gates* f8 = nullptr) {
   int s = check_args(x, W_r, b, W_gate, W_up, W_down, T, d, N, Z, K, I, off, out);
   if (s != MOE_ZC_OK) return s;
+  if ((s = check_fp8(f8, d, N)) != MOE_ZC_OK) return s;
+  if (N == 0) f8 = nullptr;
   Ctx* cp = nullptr;
   if ((s = get_ctx(&cp)) != MOE_ZC_OK) return s;
   Ctx& c = *cp;
-  if ((s = reserve_impl(c, T, d, N, Z, K, N > 0 ? I : 128)) != MOE_ZC_OK) return s;
+  if ((s = reserve_impl(c, T, d, N, Z, K, N > 0 ? I : 128, f8 != nullptr)) != MOE_ZC_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int E = N + Z;
   const long long wait_ns = g_wait_ns_next > 0 ? g_wait_ns_next : kWaitNs;
@@ -403,7 +452,9 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   const Plan plan = make_plan(T, d, N, Z, K, I, c.sms,
                               T > 0 && T <= GEMM_SMALL_B && N > 0 && !c.one_grid_refused
                                   ? fused_resident_blocks()
-                                  : 0);
+                                  : 0,
+                              f8 != nullptr);
+  int* grp_ttp8 = f8 ? static_cast<int*>(c.grp_ttp8.p) : nullptr;
   if (T > 0) {
     // 1  router GEMM
     CUtensorMap mWr, mX;
@@ -446,10 +497,17 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     rec.mark(2);
     if (N > 0) {
       // 3-4  dispatch
-      CK(launch_assign_slots(cnt, idx, T * K, N, grp_off, grp_ttp, fill, slot, st));
+      CK(launch_assign_slots(cnt, idx, T * K, N, grp_off, grp_ttp, fill, slot, st, grp_ttp8));
       rec.mark(3);
-      CK(launch_permute(static_cast<const __nv_bfloat16*>(x), slot, T, d, K,
-                        static_cast<__nv_bfloat16*>(c.Xp.p), st));
+      if (f8) {
+        // each token row quantised once (E4M3, 1 x 32 blocks) into its slots
+        CK(launch_permute_fp8(static_cast<const __nv_bfloat16*>(x), idx, slot, cnt, grp_off,
+                              grp_ttp8, T, d, K, N, static_cast<uint8_t*>(c.Xp8.p),
+                              static_cast<uint8_t*>(c.sfx.p), st));
+      } else {
+        CK(launch_permute(static_cast<const __nv_bfloat16*>(x), slot, T, d, K,
+                          static_cast<__nv_bfloat16*>(c.Xp.p), st));
+      }
       rec.mark(4);
       // 5  gate/up GEMM
       CUtensorMap mWg, mWu, mXp;
@@ -494,6 +552,25 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       pd.a_rows = d;
       pd.out = c.Y.p;
       pd.out_ld = d;
+      if (f8) {
+        // the FP8 gate/up GEMM: E4M3 operands with 128 contraction elements
+        // per stage, FP8_BN-token tiles, scale atoms (the down GEMM above
+        // keeps the bf16 parameters)
+        const bool full8 = c.rows_cap >= FP8_BN;
+        if (!make_map_u8(&mWg, W_gate, static_cast<uint64_t>(N) * I, d, GEMM_BM) ||
+            !make_map_u8(&mWu, W_up, static_cast<uint64_t>(N) * I, d, GEMM_BM) ||
+            !make_map_u8(&mXp, c.Xp8.p, c.rows_cap, d, GEMM_B_BOX_ROWS) ||
+            !make_map_u8(&mXpf, c.Xp8.p, c.rows_cap, d, full8 ? FP8_BN : GEMM_B_BOX_ROWS))
+          return MOE_ZC_ERR_CUDA;
+        pg.b_box_full = full8 ? 1 : 0;
+        pg.tok_tile = FP8_BN;
+        pg.grp_ttp = grp_ttp8;
+        pg.ksteps = d / FP8_BK;
+        pg.sf_kgroups = d / FP8_BK;
+        pg.sfa0 = f8->gate_sf;
+        pg.sfa1 = f8->up_sf;
+        pg.sfb = static_cast<const uint8_t*>(c.sfx.p);
+      }
       bool one_grid = plan.one_grid;
       if (one_grid) {
         // 5-6  at most 64 tokens: both expert GEMMs in one persistent grid,
@@ -505,8 +582,11 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
         pf.b_box_full = 0;
         pf.done = fill + N + 1;
         pf.down_lead = (d + I / 2) / I;
-        const cudaError_t e = launch_gemm_fused(mWg, mWu, mXp, mWd, mH, pf, pd,
-                                                static_cast<int>(plan.fused_grid), st);
+        const cudaError_t e =
+            f8 ? launch_gemm_fused_fp8(mWg, mWu, mXp, mWd, mH, pf, pd,
+                                       static_cast<int>(plan.fused_grid), st)
+               : launch_gemm_fused(mWg, mWu, mXp, mWd, mH, pf, pd,
+                                   static_cast<int>(plan.fused_grid), st);
         if (e != cudaSuccess) {
           // refused as a cooperative launch (its blocks cannot all be
           // resident): nothing was queued; run the two launches from now on
@@ -521,8 +601,12 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       }
       if (!one_grid) {
         // 5  gate/up GEMM
-        CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg, static_cast<int>(plan.gateup_grid),
-                       st));
+        if (f8)
+          CK(launch_gemm_gateup_fp8(mWg, mWu, mXp, mXpf, pg, static_cast<int>(plan.gateup_grid),
+                                    st));
+        else
+          CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg,
+                         static_cast<int>(plan.gateup_grid), st));
         rec.mark(5);
         // 6  down GEMM
         CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd, static_cast<int>(plan.down_grid), st));
@@ -713,6 +797,27 @@ int moe_zc_forward_ex(const void* x, const void* W_r, const float* b, const void
                       stream);
 }
 
+int moe_zc_forward_fp8(const void* x, const void* W_r, const float* b, const void* W_gate8,
+                       const void* W_gate_sf, const void* W_up8, const void* W_up_sf,
+                       const void* W_down, int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K,
+                       int32_t I, const float* logit_offset, void* out, void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const Fp8Gates f8{static_cast<const uint8_t*>(W_gate_sf), static_cast<const uint8_t*>(W_up_sf)};
+  return forward_impl(x, W_r, b, W_gate8, W_up8, W_down, T, d, N, Z, K, I, logit_offset, out,
+                      stream, &f8);
+}
+
+int moe_zc_fp8_quantize_weights(const void* W, int64_t rows, int32_t cols, void* codes,
+                                void* scales, void* stream) {
+  if (!W || !codes || !scales || rows < 1 || cols < 1) return MOE_ZC_ERR_INVALID_ARG;
+  if (rows % GEMM_BM != 0 || cols % FP8_BK != 0) return MOE_ZC_ERR_UNSUPPORTED;
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(scales)) return MOE_ZC_ERR_UNSUPPORTED;
+  CK(launch_fp8_quantize_weights(static_cast<const __nv_bfloat16*>(W), rows, cols,
+                                 static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                                 static_cast<cudaStream_t>(stream)));
+  return MOE_ZC_OK;
+}
+
 int moe_zc_forward_host(const void* x_host, const void* W_r, const float* b,
                         const void* W_gate, const void* W_up, const void* W_down, int64_t T,
                         int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I,
@@ -815,7 +920,8 @@ void moe_zc_release(void) {
     Buf* bufs[] = {&c.logits, &c.idx,     &c.gate,    &c.zsum,      &c.slot,
                    &c.cnt,    &c.fill,    &c.grp_off, &c.grp_ttp,   &c.Xp,
                    &c.H,      &c.Y,       &c.err,     &c.xin[0],    &c.xin[1],
-                   &c.yout[0], &c.yout[1], &c.cnt_total};
+                   &c.yout[0], &c.yout[1], &c.cnt_total, &c.Xp8,     &c.sfx,
+                   &c.grp_ttp8};
     for (Buf* b : bufs) {
       if (b->p) cudaFree(b->p);
       *b = Buf{};

@@ -210,6 +210,65 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N) {
          | ((M >> 4) << 24);  // M / 16
 }
 
+// ---------------------------------------------------------------- block-scaled FP8
+// D[tmem] (+)= (A * sa) * (B * sb)^T, kind::mxf8f6f4 with block scaling: A and
+// B E4M3, K-major, K = 32 per instruction; one UE8M0 scale per row of A and
+// per column of B for the 32 elements, read from TMEM at sfa / sfb (the byte
+// within each 32-bit TMEM word is chosen by the instruction descriptor).
+__device__ __forceinline__ void umma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+        "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor of umma_mxf8: E4M3 x E4M3 -> fp32, UE8M0 scales,
+// M x N, scale bytes sfa_id / sfb_id of the TMEM words (the 32-element block
+// of the 4 that one 32-bit word holds).
+__host__ __device__ constexpr uint32_t idesc_mxf8(uint32_t M, uint32_t N, uint32_t sfa_id,
+                                                 uint32_t sfb_id) {
+  return (sfb_id << 4)        // B scale-factor byte
+         | (0u << 7)          // A format: E4M3
+         | (0u << 10)         // B format: E4M3
+         | ((N >> 3) << 17)   // N / 8
+         | (1u << 23)         // scale format: UE8M0
+         | ((M >> 4) << 24)   // M / 16
+         | (sfa_id << 29);    // A scale-factor byte
+}
+
+// Copy 32 rows x 16 bytes of shared memory (a 512-byte scale atom) into 4
+// TMEM columns of all four lane quadrants (lane i % 32 of each quadrant gets
+// row i).  Asynchronous, ordered with this thread's later tcgen05.mma.
+__device__ __forceinline__ void tmem_cp_atom(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// Shared-memory descriptor of a 512-byte scale atom for tmem_cp_atom: 32
+// rows of 16 bytes, no swizzle (8-row core matrices 128 bytes apart).
+__device__ __forceinline__ uint64_t smem_desc_atom(uint32_t saddr) {
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);   // start address
+  desc |= static_cast<uint64_t>(128 >> 4) << 32;           // stride byte offset (8-row groups)
+  desc |= static_cast<uint64_t>(1) << 46;                  // descriptor version (sm100)
+  return desc;                                             // layout: no swizzle
+}
+
+// Untiled bulk copy global -> shared (this CTA), completing on `bar`: both
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ---------------------------------------------------------------- clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -105,6 +105,11 @@ def lib() -> ctypes.CDLL:
         L.moe_zc_plan.restype = ctypes.c_int
         L.moe_zc_test_one_grid.argtypes = [i32]
         L.moe_zc_test_one_grid.restype = None
+        L.moe_zc_fp8_quantize_weights.argtypes = [vp, i64, i32, vp, vp, vp]
+        L.moe_zc_fp8_quantize_weights.restype = ctypes.c_int
+        L.moe_zc_forward_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, i32,
+                                         i32, i32, vp, vp, vp]
+        L.moe_zc_forward_fp8.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -158,6 +163,50 @@ def forward(x: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor,
         st = lib().moe_zc_forward_ex(*args, _dev_ptr(logit_offset, torch.float32, "logit_offset"),
                                      o, s)
     _check(st, "moe_zc_forward")
+    return out
+
+
+class Fp8Weight:
+    """A weight matrix quantised by moe_zc_fp8_quantize_weights: E4M3 codes
+    (uint8, the matrix's shape) and UE8M0 scales in 512-byte atoms (uint8)."""
+
+    def __init__(self, codes: torch.Tensor, scales: torch.Tensor):
+        self.codes, self.scales = codes, scales
+
+
+def fp8_quantize_weights(W: torch.Tensor, stream=None) -> Fp8Weight:
+    """moe_zc_fp8_quantize_weights of a CUDA bf16 tensor, taken as [rows, cols]
+    with cols its last dimension (e.g. W_gate [N, I, d] as [N * I, d])."""
+    cols = int(W.shape[-1])
+    rows = W.numel() // cols
+    codes = torch.empty(W.shape, dtype=torch.uint8, device=W.device)
+    scales = torch.empty(rows * cols // 32, dtype=torch.uint8, device=W.device)
+    _check(lib().moe_zc_fp8_quantize_weights(_dev_ptr(W, torch.bfloat16, "W"), rows, cols,
+                                             codes.data_ptr(), scales.data_ptr(),
+                                             _stream_ptr(stream)),
+           "moe_zc_fp8_quantize_weights")
+    return Fp8Weight(codes, scales)
+
+
+def forward_fp8(x: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor, W_gate: Fp8Weight,
+                W_up: Fp8Weight, W_down: torch.Tensor, N: int, Z: int, K: int,
+                out: Optional[torch.Tensor] = None,
+                logit_offset: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """moe_zc_forward_fp8: gate/up in block-scaled FP8 (weights from
+    fp8_quantize_weights), down in bf16; returns out [T, d] bf16."""
+    T, d = x.shape
+    I = int(W_gate.codes.shape[1]) if N > 0 else 0
+    if out is None:
+        out = torch.empty_like(x)
+    bf, u8 = torch.bfloat16, torch.uint8
+    st = lib().moe_zc_forward_fp8(
+        _dev_ptr(x, bf, "x"), _dev_ptr(W_r, bf, "W_r"), _dev_ptr(b, torch.float32, "b"),
+        _dev_ptr(W_gate.codes, u8, "W_gate codes"), _dev_ptr(W_gate.scales, u8, "W_gate scales"),
+        _dev_ptr(W_up.codes, u8, "W_up codes"), _dev_ptr(W_up.scales, u8, "W_up scales"),
+        _dev_ptr(W_down, bf, "W_down"), T, d, N, Z, K, I,
+        _dev_ptr(logit_offset, torch.float32, "logit_offset"), _dev_ptr(out, bf, "out"),
+        _stream_ptr(stream))
+    _check(st, "moe_zc_forward_fp8")
     return out
 
 
