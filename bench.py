@@ -333,11 +333,11 @@ def config_of(w, extra=None):
 
 def bf16_peak(pk, region_s, clk=None):
     """The bf16 peak a kernel timed inside a region of region_s seconds is held
-    to: the burst figure for a short region at full clocks, the sustained one
-    (seconds of back-to-back GEMMs under the power cap) for a long region or
-    one whose sampled SM clock sat below 90% of its maximum."""
-    capped = bool(clk and clk.get("sm_max_mhz") and clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"])
-    if region_s >= SUSTAINED_REGION_S or capped:
+    to: the burst figure for a region under SUSTAINED_REGION_S, the sustained
+    one (seconds of back-to-back GEMMs under the power cap) for a longer one.
+    The clocks sampled in the region are reported beside the fraction, not
+    used to pick the peak (the burst figure is the stricter one)."""
+    if region_s >= SUSTAINED_REGION_S:
         return pk["bf16_sus"], f"bf16 dense, sustained ({pk['src']}, MEASURED_PEAKS.json)"
     return pk["bf16"], f"bf16 dense, burst ({pk['src']}, MEASURED_PEAKS.json)"
 

@@ -112,3 +112,22 @@ def test_clock_samples_outside_the_region_are_dropped():
     s = c.summary(t0, t1)
     assert s["samples"] == 2 and s["sm_mhz"] == (1965 + 1900) / 2
     assert s["reasons"] == ["sw_power_cap"] and s["samples_outside_region"] == 2
+
+
+def test_fp8_layer_bytes_and_peak():
+    """FP8 gate/up: weights and tokens at one byte plus a scale byte per 32
+    elements; the down projection stays bf16.  The decode layer with 30 hit
+    experts then touches 30 x (2 x 2048 x 6144 x 33/32 + 6144 x 2048 x 2)
+    bytes of expert weights; its gate/up kernel is held to twice the bf16
+    peak."""
+    w = wl.get("decode")
+    rf = bench.roofline_numbers(w, dict(ffn_pairs=460, experts_hit=30), None, fp8=True)
+    weights = 30 * (2 * 2048 * 6144 * 33 / 32 + 6144 * 2048 * 2)
+    assert rf["B_layer"] == weights + 768 * 6144 * 2 + 768 * 4 + 2 * 64 * 6144 * 2
+    assert rf["B_gateup"] == 30 * 2 * 2048 * 6144 * 33 / 32 + 460 * 6144 * 33 / 32 + 460 * 2048 * 2
+    assert bench.tensor_peak(_pk(), 0.5, fp8=True)[0] == 2 * 1662.4
+    # the layer's tensor bound counts gate/up FLOPs at the FP8 rate
+    lr = bench.layer_roofline(rf, _pk(), 1.0, 0.5)
+    t_f = (rf["F_gateup"] / 2 + rf["F_down"]) / 1662.4e12
+    t_b = rf["B_layer"] / 6457.4e9
+    assert abs(lr["roofline_ms"] - max(t_f, t_b) * 1e3) < 1e-12

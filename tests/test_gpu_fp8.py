@@ -196,9 +196,20 @@ def test_decode_sized_fp8_one_grid_and_fallback_agree():
 
 
 def test_fp8_rejects_widths_off_128():
-    case = Fp8Case(wl.get("tiny", d=192, I=128, T=16))
+    """d = 192 is refused (a stage takes 128 contraction elements) before any
+    launch; the quantiser refuses such matrices too."""
+    w = wl.get("tiny", d=192, I=128, T=16)
+    case = Case(w)
     with pytest.raises(mz.MoeZcError) as ei:
-        case.run_fp8()
+        mz.fp8_quantize_weights(case.ew.W_gate)
+    assert ei.value.status == mz.ERR_UNSUPPORTED
+    codes = torch.zeros(w.N, w.I, w.d, dtype=torch.uint8, device="cuda")
+    scales = torch.zeros(w.N * w.I * w.d // 32, dtype=torch.uint8, device="cuda")
+    stand_in = mz.Fp8Weight(codes, scales)
+    d = case.dev
+    with pytest.raises(mz.MoeZcError) as ei:
+        mz.forward_fp8(d["x"], d["W_r"], d["b"], stand_in, stand_in, case.ew.W_down,
+                       w.N, w.Z, w.K)
     assert ei.value.status == mz.ERR_UNSUPPORTED
 
 
