@@ -108,6 +108,8 @@ def parse():
                     help="time replays of one forward captured into a CUDA graph")
     ap.add_argument("--shape", default="",
                     help="override workload sizes, e.g. T=4096,N=32,Z=16 (for profiling runs)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the forward with FP8 gate/up projections (moe_zc_forward_fp8)")
     ap.add_argument("--workloads", default=EXTRA_WORKLOADS,
                     help="comma-separated workloads also timed in the same run and reported "
                          "under `workloads` ('none': only the headline)")
@@ -568,7 +570,7 @@ def measure(args, dist, w, steps, e2e_steps, headline, fp8=False):
 
 
 def run_ours(args, dist, w):
-    res = measure(args, dist, w, args.steps, args.e2e_steps, headline=True)
+    res = measure(args, dist, w, args.steps, args.e2e_steps, headline=True, fp8=args.fp8)
     ri, b, ew = res.pop("_keep")
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
@@ -578,7 +580,8 @@ def run_ours(args, dist, w):
     line = {
         "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": dist.world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8 gate/up (E4M3, 1x32 UE8M0 blocks), bf16 down" if args.fp8 else "bf16",
         "data": "synthetic: seeded inputs, random-init weights of the workload's shapes",
         "config": config_of(w, {
             "global_batch": w.T * dist.world, "parallelism": f"replicas{dist.world}",
