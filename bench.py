@@ -77,7 +77,14 @@ def kernels_per_forward(w, sms=148):
 # launch processes); null when the sources have changed since the capture.
 GEMM_SOURCES = ["gemm_tcgen05.cu", "ptx.cuh", "epilogue.cuh", "kernels.cuh"]
 NCU_TRAFFIC_RATIO = {
-    # workload: (dominant kernel, DRAM bytes / algorithmic bytes, sources sha16, case)
+    # workload (+ "_fp8" for the FP8 forward): (dominant kernel,
+    # DRAM bytes / algorithmic bytes, GEMM sources sha16, the captured case)
+    "prefill": ("gateup_gemm", 2.9935e9 / 2.1829e9, "a50c95bdfa12e9fe",
+                "T=4096, N=32, Z=16 prefill-shaped layer (profiles/traffic_gemm_small_cases.md)"),
+    "prefill_fp8": ("gateup_gemm", 1.2903e9 / 1.1949e9, "a50c95bdfa12e9fe",
+                    "T=4096, N=32, Z=16 prefill-shaped layer (profiles/traffic_gemm_small_cases.md)"),
+    "decode_fp8": ("gateup_down_gemm (one kernel)", 0.98234e9 / 0.98599e9, "a50c95bdfa12e9fe",
+                   "T=64, N=32, Z=16 decode-shaped layer (profiles/traffic_gemm_small_cases.md)"),
 }
 SUSTAINED_REGION_S = 2.0   # timed regions at least this long use the sustained bf16 peak
 NOMINAL_HBM_GBS = 7700.0   # B200 HBM3e, HGX figure (context beside the measured copy peak)
@@ -385,7 +392,7 @@ def kernel_roofline(w, rf, plan, per, pk, region_s, clk=None):
     roof["ms_per_launch"] = per[dom]
     roof["algorithmic_bytes"] = B
     roof["algorithmic_flops"] = F
-    tr = NCU_TRAFFIC_RATIO.get(w.name)
+    tr = NCU_TRAFFIC_RATIO.get(w.name + ("_fp8" if rf.get("fp8") else ""))
     roof["traffic"] = None
     if tr and tr[0] == roof["kernel"] and tr[2] == gemm_sources_sha16():
         roof["traffic"] = tr[1] * B
