@@ -285,6 +285,59 @@ int moe_zc_forward_fp8(const void* x, const void* W_r, const float* b, const voi
                        const void* W_down, int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K,
                        int32_t I, const float* logit_offset, void* out, void* stream);
 
+/*
+ * The forward's steps as separate calls, for expert parallelism across GPUs
+ * (write-up, section "Shortcut-connected MoE": the expert computation sits
+ * between a dispatch and a combine communication step; "System-level
+ * optimisation": expert parallelism over many GPUs).  With the FFN experts
+ * split into contiguous ranges, one per rank, a rank runs
+ *   moe_zc_route     its tokens' picks, gates, zero-gate sums, histogram
+ *   moe_zc_dispatch  its FFN picks' rows packed by expert, so the rows for
+ *                    each rank's expert range are contiguous
+ *   (the caller exchanges rows, their expert ids and counts between ranks)
+ *   moe_zc_experts   the SwiGLU experts of its range on the rows it received
+ *   (the caller sends the result rows back, in the order received)
+ *   moe_zc_combine   out_t = zsum_t x_t + sum_k gate_{t,k} Y[slot_{t,k}]
+ * Zero-expert picks never leave the rank: they are folded into zsum by
+ * moe_zc_route.  All pointers are device memory (bf16 rows, int32 / fp32
+ * arrays, 16-byte aligned row buffers); every call is asynchronous on
+ * `stream`; device-side wait timeouts are reported by moe_zc_synchronize.
+ * On one rank, route -> dispatch -> experts -> combine gives moe_zc_forward's
+ * output bit for bit (the experts' rows are computed by the same GEMMs in the
+ * same reduction order).
+ *
+ * moe_zc_route: x [T, d], W_r [E, d], b [E], logit_offset [E] or NULL as for
+ *   moe_zc_forward_ex; writes idx [T*K], gate [T*K] (the unbiased softmax
+ *   probabilities), zsum [T] (sum of the gates on zero experts) and counts
+ *   [E] (histogram of all picks).  Uses the device workspace for logits.
+ * moe_zc_dispatch: x [T, d], idx [T*K] and counts [>= N] from moe_zc_route;
+ *   writes slot [T*K] (row of pick (t, k) in `send`, or -1 for a zero-expert
+ *   pick), send [sum(counts[0..N-1]), d] (x rows grouped by expert, expert 0
+ *   first, no padding; the order inside an expert is not fixed) and
+ *   send_expert [same rows] (each row's expert).  N >= 1, d % 8 == 0.
+ * moe_zc_experts: x_rows [R, d] and expert [R]: row i goes to FFN expert
+ *   expert[i] - expert_base of the N given (W_gate [N, I, d], W_up, W_down
+ *   [N, d, I]); y [R, d] receives E_e(x_i) in bf16 (rows whose expert lies
+ *   outside [expert_base, expert_base + N) get zeros).  Conditions on d and
+ *   I as for moe_zc_forward.  Runs the forward's dispatch, GEMMs and
+ *   combine with gate 1, so moe_zc_last_routing, moe_zc_last_expert and
+ *   moe_zc_expert_load describe this call afterwards.
+ * moe_zc_combine: x [T, d], y_rows (the rows slot indexes), slot, gate
+ *   [T*K], zsum [T] -> out [T, d] bf16: fp32 accumulation in k order, one
+ *   rounding.  d % 8 == 0.
+ */
+int moe_zc_route(const void* x, const void* W_r, const float* b, const float* logit_offset,
+                 int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t* idx,
+                 float* gate, float* zsum, int32_t* counts, void* stream);
+int moe_zc_dispatch(const void* x, const int32_t* idx, const int32_t* counts, int64_t T,
+                    int32_t d, int32_t N, int32_t K, int32_t* slot, void* send,
+                    int32_t* send_expert, void* stream);
+int moe_zc_experts(const void* x_rows, const int32_t* expert, int32_t expert_base, int64_t R,
+                   int32_t d, int32_t N, int32_t I, const void* W_gate, const void* W_up,
+                   const void* W_down, void* y, void* stream);
+int moe_zc_combine(const void* x, const void* y_rows, const int32_t* slot, const float* gate,
+                   const float* zsum, int64_t T, int32_t d, int32_t K, void* out, void* stream);
+
 /* Wait for the last forward; report (and clear) a device-side timeout. */
 int moe_zc_synchronize(void);
 

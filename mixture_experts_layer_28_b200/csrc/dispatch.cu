@@ -9,8 +9,10 @@
 //             FFN expert's rows (count rounded up to 16) and token tiles
 //             (ceil(count / 256), and for the FP8 gate/up GEMM ceil(count /
 //             240)); exclusive prefix sums give the expert's first row in the
-//             permuted buffers (grp_off) and its first GEMM token tile
-//             (grp_ttp, grp_ttp8), which CTA 0 also stores for the GEMMs
+//             permuted buffers (rows rounded up to 16 per expert, or not at
+//             all for a dispatch to other ranks, whose rows travel packed)
+//             (grp_off) and its first GEMM token tile (grp_ttp, grp_ttp8),
+//             which CTA 0 also stores for the GEMMs
 //             (the GEMM grid walks grp_ttp).  Then one thread per (token,
 //             pick): lanes of a warp that picked the same expert are grouped
 //             with __match_any_sync and take their slots with one atomicAdd
@@ -60,7 +62,8 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total
 __global__ void __launch_bounds__(ASSIGN_THREADS)
 assign_slots_kernel(const int* __restrict__ cnt, const int* __restrict__ idx, int64_t pairs,
                     int N, int* __restrict__ grp_off, int* __restrict__ grp_ttp,
-                    int* __restrict__ fill, int* __restrict__ slot, int* __restrict__ grp_ttp8) {
+                    int* __restrict__ fill, int* __restrict__ slot, int* __restrict__ grp_ttp8,
+                    int pad, int* __restrict__ row_expert) {
   __shared__ int off_s[MOE_MAX_E_INTERNAL];
   __shared__ int warp_sums[32];
   griddep_wait();
@@ -70,7 +73,7 @@ assign_slots_kernel(const int* __restrict__ cnt, const int* __restrict__ idx, in
     const int g = base + threadIdx.x;
     const int c = g < N ? cnt[g] : 0;
     int tot_rows, tot_tiles = 0, tot_tiles8 = 0;
-    const int off = block_excl_scan((c + 15) & ~15, warp_sums, &tot_rows);
+    const int off = block_excl_scan((c + pad - 1) / pad * pad, warp_sums, &tot_rows);
     if (g < N) off_s[g] = carry_rows + off;
     if (blockIdx.x == 0) {
       const int ttp = block_excl_scan((c + GEMM_BN - 1) / GEMM_BN, warp_sums, &tot_tiles);
@@ -109,6 +112,7 @@ assign_slots_kernel(const int* __restrict__ cnt, const int* __restrict__ idx, in
     if (lane == leader) base = atomicAdd(&fill[e], __popc(peers));
     base = __shfl_sync(peers, base, leader);
     s = off_s[e] + base + rank;
+    if (row_expert) row_expert[s] = e;
   }
   if (valid) slot[i] = s;
   griddep_launch_dependents();   // as the last CTAs finish (several waves)
@@ -138,6 +142,25 @@ __global__ void permute_kernel(const uint4* __restrict__ x, const int* __restric
   griddep_launch_dependents();
 }
 
+// Caller-given routing of R rows, one pick each: idx = expert - base, gate
+// 1, zsum 0, and the histogram (cnt zeroed before the launch).  A row whose
+// expert lies outside [base, base + N) is not dispatched (its output row is
+// zero).
+__global__ void given_routing_kernel(const int* __restrict__ expert, int64_t R, int base, int N,
+                                     int* __restrict__ idx, float* __restrict__ gate,
+                                     float* __restrict__ zsum, int* __restrict__ cnt) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= R) return;
+  const int e = expert[i] - base;
+  const bool ok = e >= 0 && e < N;
+  idx[i] = ok ? e : -1;
+  gate[i] = 1.0f;
+  zsum[i] = 0.0f;
+  if (ok) atomicAdd(cnt + e, 1);
+}
+
 __global__ void add_counts_kernel(const int* __restrict__ cnt, int E, int* __restrict__ total) {
   griddep_wait();
   griddep_launch_dependents();
@@ -153,10 +176,18 @@ cudaError_t launch_add_counts(const int* cnt, int E, int* total, cudaStream_t st
 
 cudaError_t launch_assign_slots(const int* cnt, const int* idx, int64_t pairs, int N,
                                 int* grp_off, int* grp_ttp, int* fill, int* slot,
-                                cudaStream_t stream, int* grp_ttp8) {
+                                cudaStream_t stream, int* grp_ttp8, int pad, int* row_expert) {
   const int64_t blocks = pairs > 0 ? (pairs + ASSIGN_THREADS - 1) / ASSIGN_THREADS : 1;
   return launch_pdl(assign_slots_kernel, dim3(static_cast<unsigned>(blocks)), dim3(ASSIGN_THREADS),
-                    0, stream, cnt, idx, pairs, N, grp_off, grp_ttp, fill, slot, grp_ttp8);
+                    0, stream, cnt, idx, pairs, N, grp_off, grp_ttp, fill, slot, grp_ttp8, pad,
+                    row_expert);
+}
+
+cudaError_t launch_given_routing(const int* expert, int64_t R, int base, int N, int* idx,
+                                 float* gate, float* zsum, int* cnt, cudaStream_t stream) {
+  if (R <= 0) return cudaSuccess;
+  return launch_pdl(given_routing_kernel, dim3(static_cast<unsigned>((R + 255) / 256)), dim3(256),
+                    0, stream, expert, R, base, N, idx, gate, zsum, cnt);
 }
 
 cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, int d, int K,

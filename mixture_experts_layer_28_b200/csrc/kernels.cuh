@@ -300,9 +300,18 @@ cudaError_t launch_route(const float* logits, const float* b, const float* offse
 // [N + 1], written by CTA 0) computed from the histogram cnt; fill [N] must
 // be zero on entry (the router GEMM clears it).
 // grp_ttp8 (optional, [N + 1]): the same prefix for FP8_BN-token tiles.
+// pad: each expert's rows rounded up to a multiple of pad (16 for the GEMM
+// buffers, 1 for packed rows); row_expert (optional): the expert of every
+// assigned row.
 cudaError_t launch_assign_slots(const int* cnt, const int* idx, int64_t pairs, int N,
                                 int* grp_off, int* grp_ttp, int* fill, int* slot,
-                                cudaStream_t stream, int* grp_ttp8 = nullptr);
+                                cudaStream_t stream, int* grp_ttp8 = nullptr, int pad = 16,
+                                int* row_expert = nullptr);
+// Routing given by the caller for R rows with one pick each (expert[i] -
+// base; rows outside [0, N) are not dispatched): idx, gate 1, zsum 0 and
+// the histogram cnt (zeroed by the caller).
+cudaError_t launch_given_routing(const int* expert, int64_t R, int base, int N, int* idx,
+                                 float* gate, float* zsum, int* cnt, cudaStream_t stream);
 // total[j] += cnt[j] for j < E (histogram summed over the chunks of a forward)
 cudaError_t launch_add_counts(const int* cnt, int E, int* total, cudaStream_t stream);
 cudaError_t launch_permute(const __nv_bfloat16* x, const int* slot, int64_t T, int d, int K,

@@ -401,10 +401,17 @@ int check_fp8(const Fp8Gates* f8, int d, int N) {
 
 // f8: NULL for the bf16 forward; else W_gate / W_up hold E4M3 codes and f8
 // their scales (the FP8 gate/up GEMM; the down projection stays bf16).
+// Routing given by the caller (moe_zc_experts): row i goes, with gate 1, to
+// FFN expert expert[i] - base; there is no router (K = 1, Z = 0).
+struct GivenRouting {
+  const int32_t* expert;
+  int base;
+};
+
 int forward_impl(const void* x, const void* W_r, const float* b, const void* W_gate,
                  const void* W_up, const void* W_down, int64_t T, int32_t d, int32_t N,
                  int32_t Z, int32_t K, int32_t I, const float* off, void* out, void* stream,
-                 const Fp8Gates* f8 = nullptr) {
+                 const Fp8Gates* f8 = nullptr, const GivenRouting* given = nullptr) {
   int s = check_args(x, W_r, b, W_gate, W_up, W_down, T, d, N, Z, K, I, off, out);
   if (s != MOE_ZC_OK) return s;
   if ((s = check_fp8(f8, d, N)) != MOE_ZC_OK) return s;
@@ -455,7 +462,16 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
                                   : 0,
                               f8 != nullptr);
   int* grp_ttp8 = f8 ? static_cast<int*>(c.grp_ttp8.p) : nullptr;
+  if (T > 0 && given) {
+    // 1-2  the caller's routing: one pick per row, gate 1, no zero experts
+    CK(cudaMemsetAsync(cnt, 0, sizeof(int) * E, st));
+    CK(cudaMemsetAsync(fill, 0, sizeof(int) * (2 * N + 2), st));
+    CK(launch_given_routing(given->expert, T, given->base, N, idx, gate, zsum, cnt, st));
+    rec.mark(1);
+    rec.mark(2);
+  }
   if (T > 0) {
+   if (!given) {
     // 1  router GEMM
     CUtensorMap mWr, mX;
     const RouterPlan rp = plan.rp;
@@ -495,6 +511,7 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     CK(launch_route(static_cast<const float*>(c.logits.p), b, off, T, E, N, K, idx, gate, zsum,
                     cnt, st, splits));
     rec.mark(2);
+   }
     if (N > 0) {
       // 3-4  dispatch
       CK(launch_assign_slots(cnt, idx, T * K, N, grp_off, grp_ttp, fill, slot, st, grp_ttp8));
@@ -795,6 +812,120 @@ int moe_zc_forward_ex(const void* x, const void* W_r, const float* b, const void
   std::lock_guard<std::mutex> lk(g_mu);
   return forward_impl(x, W_r, b, W_gate, W_up, W_down, T, d, N, Z, K, I, logit_offset, out,
                       stream);
+}
+
+int moe_zc_route(const void* x, const void* W_r, const float* b, const float* logit_offset,
+                 int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t* idx,
+                 float* gate, float* zsum, int32_t* counts, void* stream) {
+  const void* f = reinterpret_cast<const void*>(16);   // stand-ins: no expert weights here
+  int s = check_args(x, W_r, b, f, f, f, T, d, N, Z, K, 128, logit_offset, f);
+  if (s != MOE_ZC_OK) return s;
+  if (!counts || (T > 0 && (!idx || !gate || !zsum))) return MOE_ZC_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Ctx* cp = nullptr;
+  if ((s = get_ctx(&cp)) != MOE_ZC_OK) return s;
+  Ctx& c = *cp;
+  const int E = N + Z;
+  const RouterPlan rp = router_plan(T, E, d / GEMM_BK, c.sms);
+  const bool fresh_err = c.err.p == nullptr;
+  if ((s = ensure(c, c.err, sizeof(int))) != MOE_ZC_OK) return s;
+  if (fresh_err && cudaMemset(c.err.p, 0, sizeof(int)) != cudaSuccess) return MOE_ZC_ERR_CUDA;
+  if ((s = ensure(c, c.logits, static_cast<size_t>(T * E * rp.splits) * sizeof(float))) !=
+      MOE_ZC_OK)
+    return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long wait_ns = g_wait_ns_next > 0 ? g_wait_ns_next : kWaitNs;
+  g_wait_ns_next = 0;
+  if (T == 0) {
+    CK(cudaMemsetAsync(counts, 0, sizeof(int) * E, st));
+  } else {
+    CUtensorMap mWr, mX, mXf;
+    const bool full_ok = T >= rp.tok_tile;
+    if (!make_map(&mWr, W_r, E, d, GEMM_BM) || !make_map(&mX, x, T, d, GEMM_B_BOX_ROWS) ||
+        !make_map(&mXf, x, T, d, full_ok ? rp.tok_tile : GEMM_B_BOX_ROWS))
+      return MOE_ZC_ERR_CUDA;
+    GemmParams pr{};
+    pr.G = 1;
+    pr.T = static_cast<int>(T);
+    pr.ksteps = d / GEMM_BK;
+    pr.a_rows = E;
+    pr.out = c.logits.p;
+    pr.out_ld = E;
+    pr.err = static_cast<int*>(c.err.p);
+    pr.wait_ns = wait_ns;
+    pr.mblocks = rp.mblocks;
+    pr.single_a = rp.single_a;
+    pr.tok_tile = rp.tok_tile;
+    pr.ksplit = rp.splits;
+    pr.split_stride = T * E;
+    pr.b_box_full = full_ok ? 1 : 0;
+    pr.small_b = T <= GEMM_SMALL_B ? 1 : 0;
+    pr.zero0 = counts;   // the router GEMM clears the histogram
+    pr.nzero0 = E;
+    const int64_t rg = rp.tiles * rp.splits;
+    CK(launch_gemm(MODE_ROUTER, mWr, mWr, mX, mXf, pr, static_cast<int>(rg < c.sms ? rg : c.sms),
+                   st));
+    CK(launch_route(static_cast<const float*>(c.logits.p), b, logit_offset, T, E, N, K, idx, gate,
+                    zsum, counts, st, rp.splits));
+  }
+  CK(cudaEventRecord(c.done, st));
+  c.done_valid = true;
+  c.has_result = true;
+  return MOE_ZC_OK;
+}
+
+int moe_zc_dispatch(const void* x, const int32_t* idx, const int32_t* counts, int64_t T,
+                    int32_t d, int32_t N, int32_t K, int32_t* slot, void* send,
+                    int32_t* send_expert, void* stream) {
+  if (T < 0 || N < 1 || K < 1 || K > MOE_ZC_MAX_K || N > MOE_ZC_MAX_E || d <= 0)
+    return MOE_ZC_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !idx || !counts || !slot || !send || !send_expert))
+    return MOE_ZC_ERR_INVALID_ARG;
+  if (d % 8 != 0 || !aligned16(x) || !aligned16(send)) return MOE_ZC_ERR_UNSUPPORTED;
+  if (T * K > (1LL << 31) - 1) return MOE_ZC_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_ZC_OK;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Ctx* cp = nullptr;
+  int s = get_ctx(&cp);
+  if (s != MOE_ZC_OK) return s;
+  Ctx& c = *cp;
+  if ((s = ensure(c, c.fill, static_cast<size_t>(2 * N + 2) * sizeof(int))) != MOE_ZC_OK) return s;
+  if ((s = ensure(c, c.grp_off, static_cast<size_t>(N + 1) * sizeof(int))) != MOE_ZC_OK) return s;
+  if ((s = ensure(c, c.grp_ttp, static_cast<size_t>(N + 1) * sizeof(int))) != MOE_ZC_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* fill = static_cast<int*>(c.fill.p);
+  CK(cudaMemsetAsync(fill, 0, sizeof(int) * (N + 1), st));
+  // packed rows (no padding): expert e's rows follow expert e - 1's, so the
+  // rows bound for each rank's contiguous range of experts are contiguous
+  CK(launch_assign_slots(counts, idx, T * K, N, static_cast<int*>(c.grp_off.p),
+                         static_cast<int*>(c.grp_ttp.p), fill, slot, st, nullptr, 1, send_expert));
+  CK(launch_permute(static_cast<const __nv_bfloat16*>(x), slot, T, d, K,
+                    static_cast<__nv_bfloat16*>(send), st));
+  return MOE_ZC_OK;
+}
+
+int moe_zc_experts(const void* x_rows, const int32_t* expert, int32_t expert_base, int64_t R,
+                   int32_t d, int32_t N, int32_t I, const void* W_gate, const void* W_up,
+                   const void* W_down, void* y, void* stream) {
+  if (R > 0 && !expert) return MOE_ZC_ERR_INVALID_ARG;
+  if (N < 1) return MOE_ZC_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  const void* f = reinterpret_cast<const void*>(16);   // no router: stand-ins
+  const GivenRouting given{expert, expert_base};
+  return forward_impl(x_rows, f, static_cast<const float*>(f), W_gate, W_up, W_down, R, d, N, 0,
+                      1, I, nullptr, y, stream, nullptr, &given);
+}
+
+int moe_zc_combine(const void* x, const void* y_rows, const int32_t* slot, const float* gate,
+                   const float* zsum, int64_t T, int32_t d, int32_t K, void* out, void* stream) {
+  if (T < 0 || K < 1 || K > MOE_ZC_MAX_K || d <= 0) return MOE_ZC_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !slot || !gate || !zsum || !out)) return MOE_ZC_ERR_INVALID_ARG;
+  if (d % 8 != 0 || !aligned16(x) || !aligned16(y_rows) || !aligned16(out))
+    return MOE_ZC_ERR_UNSUPPORTED;
+  CK(launch_combine(static_cast<const __nv_bfloat16*>(x),
+                    static_cast<const __nv_bfloat16*>(y_rows), slot, gate, zsum, T, d, K,
+                    static_cast<__nv_bfloat16*>(out), static_cast<cudaStream_t>(stream)));
+  return MOE_ZC_OK;
 }
 
 int moe_zc_forward_fp8(const void* x, const void* W_r, const float* b, const void* W_gate8,

@@ -110,6 +110,14 @@ def lib() -> ctypes.CDLL:
         L.moe_zc_forward_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, i32,
                                          i32, i32, vp, vp, vp]
         L.moe_zc_forward_fp8.restype = ctypes.c_int
+        L.moe_zc_route.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+        L.moe_zc_route.restype = ctypes.c_int
+        L.moe_zc_dispatch.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, vp]
+        L.moe_zc_dispatch.restype = ctypes.c_int
+        L.moe_zc_experts.argtypes = [vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, vp, vp]
+        L.moe_zc_experts.restype = ctypes.c_int
+        L.moe_zc_combine.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, vp, vp]
+        L.moe_zc_combine.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -207,6 +215,76 @@ def forward_fp8(x: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor, W_gate: Fp8
         _dev_ptr(logit_offset, torch.float32, "logit_offset"), _dev_ptr(out, bf, "out"),
         _stream_ptr(stream))
     _check(st, "moe_zc_forward_fp8")
+    return out
+
+
+def route(x: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor, N: int, Z: int, K: int,
+          logit_offset: Optional[torch.Tensor] = None, stream=None):
+    """moe_zc_route: (idx int32 [T, K], gate fp32 [T, K], zsum fp32 [T],
+    counts int32 [E]) as CUDA tensors."""
+    T, d = x.shape
+    dev = x.device
+    idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+    gate = torch.empty(T, K, dtype=torch.float32, device=dev)
+    zsum = torch.empty(T, dtype=torch.float32, device=dev)
+    counts = torch.empty(N + Z, dtype=torch.int32, device=dev)
+    _check(lib().moe_zc_route(_dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(W_r, torch.bfloat16, "W_r"),
+                              _dev_ptr(b, torch.float32, "b"),
+                              _dev_ptr(logit_offset, torch.float32, "logit_offset"), T, d, N, Z, K,
+                              idx.data_ptr(), gate.data_ptr(), zsum.data_ptr(), counts.data_ptr(),
+                              _stream_ptr(stream)), "moe_zc_route")
+    return idx, gate, zsum, counts
+
+
+def dispatch(x: torch.Tensor, idx: torch.Tensor, counts: torch.Tensor, N: int, rows: int,
+             stream=None):
+    """moe_zc_dispatch: (slot int32 [T, K], send bf16 [rows, d], send_expert
+    int32 [rows]); rows = the FFN picks, sum(counts[:N]) (known to the caller
+    from the histogram)."""
+    T, d = x.shape
+    K = int(idx.shape[1])
+    slot = torch.empty(T, K, dtype=torch.int32, device=x.device)
+    send = torch.empty(max(rows, 1), d, dtype=torch.bfloat16, device=x.device)
+    send_expert = torch.empty(max(rows, 1), dtype=torch.int32, device=x.device)
+    _check(lib().moe_zc_dispatch(_dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(idx, torch.int32, "idx"),
+                                 _dev_ptr(counts, torch.int32, "counts"), T, d, N, K,
+                                 slot.data_ptr(), send.data_ptr(), send_expert.data_ptr(),
+                                 _stream_ptr(stream)), "moe_zc_dispatch")
+    return slot, send[:rows], send_expert[:rows]
+
+
+def experts(x_rows: torch.Tensor, expert: torch.Tensor, expert_base: int, W_gate: torch.Tensor,
+            W_up: torch.Tensor, W_down: torch.Tensor, stream=None) -> torch.Tensor:
+    """moe_zc_experts: y [R, d], row i = SwiGLU expert (expert[i] - expert_base)
+    of the given shard applied to x_rows[i]."""
+    R, d = x_rows.shape
+    N, I = int(W_gate.shape[0]), int(W_gate.shape[1])
+    y = torch.empty_like(x_rows)
+    bf = torch.bfloat16
+    _check(lib().moe_zc_experts(_dev_ptr(x_rows, bf, "x_rows") if R else None,
+                                _dev_ptr(expert, torch.int32, "expert") if R else None,
+                                expert_base, R, d, N, I, _dev_ptr(W_gate, bf, "W_gate"),
+                                _dev_ptr(W_up, bf, "W_up"), _dev_ptr(W_down, bf, "W_down"),
+                                y.data_ptr() if R else None, _stream_ptr(stream)), "moe_zc_experts")
+    return y
+
+
+def combine(x: torch.Tensor, y_rows: torch.Tensor, slot: torch.Tensor, gate: torch.Tensor,
+            zsum: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """moe_zc_combine: out_t = zsum_t x_t + sum_k gate_{t,k} y_rows[slot_{t,k}]."""
+    T, d = x.shape
+    K = int(slot.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    yp = y_rows.data_ptr() if y_rows.numel() else None
+    if yp is not None:
+        _dev_ptr(y_rows, torch.bfloat16, "y_rows")
+    _check(lib().moe_zc_combine(_dev_ptr(x, torch.bfloat16, "x"), yp,
+                                _dev_ptr(slot, torch.int32, "slot"),
+                                _dev_ptr(gate, torch.float32, "gate"),
+                                _dev_ptr(zsum, torch.float32, "zsum"), T, d, K,
+                                _dev_ptr(out, torch.bfloat16, "out"), _stream_ptr(stream)),
+           "moe_zc_combine")
     return out
 
 
