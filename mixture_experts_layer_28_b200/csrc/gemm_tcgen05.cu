@@ -43,6 +43,12 @@
 // down tiles run in one persistent grid (MODE_FUSED, see gemm_kernel), so the
 // SMs that the last, part-filled round of gate/up tiles leaves idle stream
 // down weights of the experts whose H rows are already complete.
+// Prefill-sized gate/up and down launches take their tiles in order from a
+// global counter (the producer takes each and hands it to the MMA issuer and
+// the epilogue through a small shared-memory queue), so the tiles running
+// at any moment are neighbours in tile order -- those that share a weight
+// block or a token tile overlap in time and re-read it from L2 -- and the
+// last round is shared out evenly.
 // Every wait is time-bounded (ptx.cuh); on running out the CTA drains its
 // in-flight copies and MMAs, frees TMEM and returns with the error flag set.
 #include "epilogue.cuh"
@@ -54,6 +60,7 @@ namespace {
 
 constexpr long long DRAIN_NS = 2000000000LL;  // bound of the drain waits at exit
 constexpr long long PACE_NS = 50000LL;        // longest wait for the partner CTA's tile start
+constexpr int TILE_Q = 4;                      // depth of the producer's tile queue
 
 struct Tile {
   int k0, k1;   // k-step range of this tile
@@ -361,6 +368,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
   __shared__ uint32_t peer_tile_sh;   // p.pair_tiles: paced tiles the partner CTA has begun
+  // Tiles taken from p.tile_counter: the producer takes each and hands it to
+  // the MMA issuer and the epilogue warps through this queue (-1: no more).
+  __shared__ volatile int tile_q[TILE_Q];
+  __shared__ __align__(8) uint64_t tq_full[TILE_Q];
+  __shared__ __align__(8) uint64_t tq_empty[TILE_Q];
+  const bool dyn =
+      (MODE == MODE_GATEUP || MODE == MODE_DOWN) && p.tile_counter != nullptr && !p.pair_tiles;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -377,6 +391,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       mbar_init(&acc_empty_bar[b], GEMM_EPI_THREADS);
     }
     mbar_init(&drain_bar, 1);
+    for (int i = 0; i < TILE_Q; ++i) {
+      mbar_init(&tq_full[i], 1);
+      mbar_init(&tq_empty[i], 1 + GEMM_EPI_WARPS);
+    }
     abort_sh = 0;
     peer_tile_sh = 0;
     fence_mbar_init();
@@ -442,7 +460,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     uint32_t begun = 0;
     for (int it = 0; !abort_sh; ++it) {
       int tph, t;
-      if (!tile_at<MODE>(p, it, ntiles, ntiles2, tph, t)) break;
+      if (dyn) {
+        // take the next tile of the grid and hand it to the other roles
+        const int qs = it % TILE_Q;
+        if (!mbar_wait(&tq_empty[qs], ((it / TILE_Q) & 1) ^ 1, p.wait_ns, p.err)) {
+          abort_sh = 1;
+          break;
+        }
+        t = atomicAdd(p.tile_counter, 1);
+        if (t >= ntiles) t = -1;
+        tph = 0;
+        tile_q[qs] = t;
+        mbar_arrive(&tq_full[qs]);
+        if (t < 0) break;
+      } else if (!tile_at<MODE>(p, it, ntiles, ntiles2, tph, t)) {
+        break;
+      }
       const Tile tl = phase_tile<MODE>(p, p2, tph, t);
       const bool down_ph = MODE == MODE_FUSED && tph == 1;
       if (down_ph) {
@@ -547,7 +580,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     uint32_t phase = 0;
     for (int local = 0; !abort_sh; ++local) {
       int tph, t;
-      if (!tile_at<MODE>(p, local, ntiles, ntiles2, tph, t)) break;
+      if (dyn) {
+        const int qs = local % TILE_Q;
+        if (!mbar_wait(&tq_full[qs], (local / TILE_Q) & 1, p.wait_ns, p.err)) {
+          abort_sh = 1;
+          break;
+        }
+        t = tile_q[qs];
+        tph = 0;
+        mbar_arrive(&tq_empty[qs]);
+        if (t < 0) break;
+      } else if (!tile_at<MODE>(p, local, ntiles, ntiles2, tph, t)) {
+        break;
+      }
       const Tile tl = phase_tile<MODE>(p, p2, tph, t);
       const int buf = local % nbuf;
       const int use = local / nbuf;
@@ -645,7 +690,20 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     const uint64_t pol_out = p.l2_stream ? l2_policy_evict_first() : 0;
     for (int local = 0; !abort_sh; ++local) {
       int tph, t;
-      if (!tile_at<MODE>(p, local, ntiles, ntiles2, tph, t)) break;
+      if (dyn) {
+        const int qs = local % TILE_Q;
+        if (!mbar_wait(&tq_full[qs], (local / TILE_Q) & 1, p.wait_ns, p.err)) {
+          abort_sh = 1;
+          break;
+        }
+        t = tile_q[qs];
+        tph = 0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tq_empty[qs]);
+        if (t < 0) break;
+      } else if (!tile_at<MODE>(p, local, ntiles, ntiles2, tph, t)) {
+        break;
+      }
       const Tile tl = phase_tile<MODE>(p, p2, tph, t);
       const int buf = local % nbuf;
       if (!mbar_wait(&acc_full_bar[buf], (local / nbuf) & 1, p.wait_ns, p.err)) {

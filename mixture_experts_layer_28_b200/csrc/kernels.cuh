@@ -199,6 +199,12 @@ struct GemmParams {
   const uint8_t* sfa1;
   const uint8_t* sfb;
   int sf_kgroups;         // contraction length / FP8_BK
+  // Gate/up and down launches without tile pacing: CTAs take tiles in order
+  // from this counter (zero before the launch) instead of every G-th tile,
+  // so the tiles running at any moment are neighbours in tile order (those
+  // sharing a weight block or token tile overlap in time, and their reads
+  // hit L2) and no CTA is left with a longer share; nullptr: fixed shares.
+  int* tile_counter;
 };
 
 // b: B map with GEMM_B_BOX_ROWS-row boxes; b_full: with GEMM_BN-row boxes,
