@@ -194,29 +194,25 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
         }
       }
     } else if (SLICED) {
-      constexpr int U = 4;   // values per thread per pass: U x 4 loads in flight
+      // Few tokens: every thread sums some of the block's logits over the
+      // slices, in slice order.  The loads of SLICE_GROUP slices are issued
+      // together before their adds, so a logit waits for ceil(splits /
+      // SLICE_GROUP) round trips to L2 rather than one per slice.
+      constexpr int SLICE_GROUP = 8;
       const int V = static_cast<int>(T - t0 < tps ? T - t0 : tps) * E;
       const float* base = logits + t0 * E;
-      for (int vb = threadIdx.x; vb < V; vb += U * blockDim.x) {
-        float a[U];
+      for (int v = threadIdx.x; v < V; v += blockDim.x) {
+        float acc = base[v];
+        for (int sp = 1; sp < splits; sp += SLICE_GROUP) {
+          float a[SLICE_GROUP];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int v = vb + u * blockDim.x;
-          a[u] = v < V ? base[v] : 0.f;
-        }
-#pragma unroll 4
-        for (int sp = 1; sp < splits; ++sp) {
+          for (int u = 0; u < SLICE_GROUP; ++u)
+            a[u] = sp + u < splits ? base[static_cast<int64_t>(sp + u) * split_stride + v] : 0.f;
 #pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int v = vb + u * blockDim.x;
-            if (v < V) a[u] += base[sp * split_stride + v];
-          }
+          for (int u = 0; u < SLICE_GROUP; ++u)
+            if (sp + u < splits) acc += a[u];
         }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int v = vb + u * blockDim.x;
-          if (v < V) lsum[v] = a[u];
-        }
+        lsum[v] = acc;
       }
       __syncthreads();
       if (mine) {
