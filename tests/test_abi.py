@@ -123,3 +123,49 @@ def test_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError):
         mz.forward(x, torch.zeros(6, 128, dtype=torch.bfloat16), torch.zeros(6), None, None, None,
                    N=0, Z=6, K=2)
+
+
+def test_fp8_entry_points_argument_checks(L):
+    f = FAKE
+    fwd8 = lambda **kw: L.moe_zc_forward_fp8(
+        kw.get("x", f), f, f, kw.get("wg", f), kw.get("wg_sf", f), kw.get("wu", f),
+        kw.get("wu_sf", f), f, 16, kw.get("d", 256), 4, 2, 2, 128, None, f, None)
+    assert fwd8(wg_sf=None) == mz.ERR_INVALID_ARG           # scales are required
+    assert fwd8(wu_sf=None) == mz.ERR_INVALID_ARG
+    assert fwd8(d=192) == mz.ERR_UNSUPPORTED                # 128 contraction elements a stage
+    assert fwd8(wg_sf=f + 4) == mz.ERR_UNSUPPORTED          # misaligned scales
+    q = L.moe_zc_fp8_quantize_weights
+    assert q(None, 128, 128, f, f, None) == mz.ERR_INVALID_ARG
+    assert q(f, 0, 128, f, f, None) == mz.ERR_INVALID_ARG
+    assert q(f, 130, 128, f, f, None) == mz.ERR_UNSUPPORTED  # rows % 128
+    assert q(f, 128, 96, f, f, None) == mz.ERR_UNSUPPORTED   # cols % 128
+    assert q(f, 128, 128, f + 8, f, None) == mz.ERR_UNSUPPORTED
+
+
+def test_expert_parallel_steps_argument_checks(L):
+    f = FAKE
+    # moe_zc_route: as the forward's router arguments
+    r = lambda **kw: L.moe_zc_route(f, f, f, None, kw.get("T", 16), kw.get("d", 128), 4, 2,
+                                    kw.get("K", 2), f, f, f, kw.get("counts", f), None)
+    assert r(counts=None) == mz.ERR_INVALID_ARG
+    assert r(K=0) == mz.ERR_INVALID_ARG
+    assert r(d=96) == mz.ERR_UNSUPPORTED
+    # moe_zc_dispatch
+    dsp = lambda **kw: L.moe_zc_dispatch(kw.get("x", f), f, f, 16, kw.get("d", 128),
+                                         kw.get("N", 4), 2, f, kw.get("send", f), f, None)
+    assert dsp(N=0) == mz.ERR_INVALID_ARG
+    assert dsp(send=None) == mz.ERR_INVALID_ARG
+    assert dsp(d=100) == mz.ERR_UNSUPPORTED
+    assert dsp(x=f + 2) == mz.ERR_UNSUPPORTED
+    # moe_zc_experts: given routing of R rows over N local experts
+    ex = lambda **kw: L.moe_zc_experts(f, kw.get("expert", f), 0, 16, kw.get("d", 128),
+                                       kw.get("N", 4), 128, f, f, f, f, None)
+    assert ex(expert=None) == mz.ERR_INVALID_ARG
+    assert ex(N=0) == mz.ERR_INVALID_ARG
+    assert ex(d=96) == mz.ERR_UNSUPPORTED
+    # moe_zc_combine
+    cb = lambda **kw: L.moe_zc_combine(kw.get("x", f), f, f, f, f, 16, kw.get("d", 128),
+                                       kw.get("K", 2), f, None)
+    assert cb(x=None) == mz.ERR_INVALID_ARG
+    assert cb(K=0) == mz.ERR_INVALID_ARG
+    assert cb(d=100) == mz.ERR_UNSUPPORTED

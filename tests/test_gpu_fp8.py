@@ -218,3 +218,38 @@ def test_full_size_fp8(name):
     case = Fp8Case(wl.get(name))
     rows = wl.tokens_sample(case.T, 128, case.w.seed).numpy()
     _check_fp8(case, rows=rows if case.T > 128 else None, n_expert_checks=3)
+
+
+def test_logit_offset_fp8():
+    """The skewed workload's Zipf logit offset, with FP8 gate/up."""
+    _check_fp8(Fp8Case(wl.get("skewed40", T=2048, d=512, I=256)))
+
+
+def test_fp8_forward_graph_replay():
+    """After one eager FP8 forward has sized the workspace, the forward can
+    be captured into a CUDA graph; replays equal the eager call bit for bit,
+    also after new token values are written into the captured input."""
+    case = Fp8Case(wl.get("small", T=512))
+    w, d = case.w, case.dev
+    out = torch.empty_like(d["x"])
+    run = lambda: mz.forward_fp8(d["x"], d["W_r"], d["b"], case.q_gate, case.q_up, case.ew.W_down,
+                                 w.N, w.Z, w.K, out=out)
+    run()
+    torch.cuda.synchronize()
+    eager = out.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager)
+    x2 = (torch.randn(w.T, w.d, generator=torch.Generator().manual_seed(9))).to(torch.bfloat16)
+    d["x"].copy_(x2.cuda())
+    g.replay()
+    torch.cuda.synchronize()
+    replayed = out.clone()
+    run()
+    torch.cuda.synchronize()
+    assert torch.equal(replayed, out)
+    del g
