@@ -22,7 +22,7 @@ own weight replica (tokens are independent: no collective in the step), so
 The JSON line also carries `workloads`: the decode, small and skewed40
 workloads and the decode and prefill layers with FP8 gate/up projections
 (moe_zc_forward_fp8, `dtype` says so) (--workloads), each timed the same way
-in the same run, with its own ms_per_step, tokens/s, e2e (bf16 only),
+in the same run, with its own ms_per_step, tokens/s, e2e,
 roofline, layer_roofline and clocks (each timed region lasts at least about
 a second, so the clocks are sampled inside it).
 Also: `e2e` (the same metric through moe_zc_forward_host: the
@@ -428,8 +428,9 @@ def measure(args, dist, w, steps, e2e_steps, headline, fp8=False):
     """Time `steps` forwards of workload w (device-resident inputs), then the
     same with per-stage events, then e2e through the host-buffer entry point.
     steps <= 0: as many as fill about one second (at least 20).  fp8: the
-    forward with FP8 gate/up (moe_zc_forward_fp8; weights quantised on the
-    device before timing; no host-buffer entry point, so no e2e)."""
+    forward with FP8 gate/up (moe_zc_forward_fp8, e2e through
+    moe_zc_forward_host_fp8; weights quantised on the device before
+    timing)."""
     from mixture_experts_layer_28_b200 import moe_zc as mz
     pk = peaks()
     ri, b, ew, dev = make_inputs(w)
@@ -529,12 +530,15 @@ def measure(args, dist, w, steps, e2e_steps, headline, fp8=False):
     # ---- end to end through the host-buffer entry point: the step's input
     # goes from pinned host memory to the device and its output comes back,
     # in chunks whose copies overlap the kernels (moe_zc_forward_host)
-    if fp8:
-        e2e_steps = 0
     x_host = ri.x.pin_memory()
     out_host = torch.empty_like(x_host).pin_memory()
 
     def step_host():
+        if fp8:
+            mz.forward_host_fp8(x_host, dev["W_r"], dev["b"], q_gate, q_up, ew.W_down,
+                                w.N, w.Z, w.K, out_host=out_host, logit_offset=dev["off"],
+                                chunk_tokens=args.chunk_tokens, stream=stream)
+            return
         mz.forward_host(x_host, dev["W_r"], dev["b"], ew.W_gate, ew.W_up, ew.W_down,
                         w.N, w.Z, w.K, out_host=out_host, logit_offset=dev["off"],
                         chunk_tokens=args.chunk_tokens, stream=stream)

@@ -338,6 +338,19 @@ int moe_zc_experts(const void* x_rows, const int32_t* expert, int32_t expert_bas
 int moe_zc_combine(const void* x, const void* y_rows, const int32_t* slot, const float* gate,
                    const float* zsum, int64_t T, int32_t d, int32_t K, void* out, void* stream);
 
+/*
+ * moe_zc_forward_fp8 on HOST buffers: x_host and out_host as for
+ * moe_zc_forward_host (chunks whose copies overlap the kernels of their
+ * neighbours), the weights as for moe_zc_forward_fp8.  Each chunk's rows
+ * equal those of moe_zc_forward_fp8 on the same chunk bit for bit.
+ */
+int moe_zc_forward_host_fp8(const void* x_host, const void* W_r, const float* b,
+                            const void* W_gate8, const void* W_gate_sf, const void* W_up8,
+                            const void* W_up_sf, const void* W_down, int64_t T, int32_t d,
+                            int32_t N, int32_t Z, int32_t K, int32_t I,
+                            const float* logit_offset, void* out_host, int64_t chunk_tokens,
+                            void* stream);
+
 /* Wait for the last forward; report (and clear) a device-side timeout. */
 int moe_zc_synchronize(void);
 

@@ -685,13 +685,14 @@ int host_streams(Ctx& c) {
 int forward_host_impl(const void* x_host, const void* W_r, const float* b, const void* W_gate,
                       const void* W_up, const void* W_down, int64_t T, int32_t d, int32_t N,
                       int32_t Z, int32_t K, int32_t I, const float* off, void* out_host,
-                      int64_t chunk, void* stream) {
+                      int64_t chunk, void* stream, const Fp8Gates* f8 = nullptr) {
   if (T < 0) return MOE_ZC_ERR_INVALID_ARG;
   if (T > 0 && (!x_host || !out_host)) return MOE_ZC_ERR_INVALID_ARG;
   // the device-side checks of one chunk (fake aligned buffers stand in)
   int s = check_args(reinterpret_cast<const void*>(16), W_r, b, W_gate, W_up, W_down, T, d, N,
                      Z, K, I, off, reinterpret_cast<void*>(16));
   if (s != MOE_ZC_OK) return s;
+  if ((s = check_fp8(f8, d, N)) != MOE_ZC_OK) return s;
   Ctx* cp = nullptr;
   if ((s = get_ctx(&cp)) != MOE_ZC_OK) return s;
   Ctx& c = *cp;
@@ -757,7 +758,7 @@ int forward_host_impl(const void* x_host, const void* W_r, const float* b, const
     CK(cudaStreamWaitEvent(st, c.ev_in[bi], 0));
     if (ci >= 2) CK(cudaStreamWaitEvent(st, c.ev_out[bi], 0));
     s = forward_impl(c.xin[bi].p, W_r, b, W_gate, W_up, W_down, n, d, N, Z, K, I, off,
-                     c.yout[bi].p, stream);
+                     c.yout[bi].p, stream, f8);
     if (s != MOE_ZC_OK) return s;
     CK(launch_add_counts(static_cast<const int*>(c.cnt.p), E,
                          static_cast<int*>(c.cnt_total.p), st));
@@ -945,6 +946,18 @@ int moe_zc_forward_fp8(const void* x, const void* W_r, const float* b, const voi
   const Fp8Gates f8{static_cast<const uint8_t*>(W_gate_sf), static_cast<const uint8_t*>(W_up_sf)};
   return forward_impl(x, W_r, b, W_gate8, W_up8, W_down, T, d, N, Z, K, I, logit_offset, out,
                       stream, &f8);
+}
+
+int moe_zc_forward_host_fp8(const void* x_host, const void* W_r, const float* b,
+                            const void* W_gate8, const void* W_gate_sf, const void* W_up8,
+                            const void* W_up_sf, const void* W_down, int64_t T, int32_t d,
+                            int32_t N, int32_t Z, int32_t K, int32_t I,
+                            const float* logit_offset, void* out_host, int64_t chunk_tokens,
+                            void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const Fp8Gates f8{static_cast<const uint8_t*>(W_gate_sf), static_cast<const uint8_t*>(W_up_sf)};
+  return forward_host_impl(x_host, W_r, b, W_gate8, W_up8, W_down, T, d, N, Z, K, I,
+                           logit_offset, out_host, chunk_tokens, stream, &f8);
 }
 
 int moe_zc_fp8_quantize_weights(const void* W, int64_t rows, int32_t cols, void* codes,

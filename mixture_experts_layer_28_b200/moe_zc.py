@@ -110,6 +110,9 @@ def lib() -> ctypes.CDLL:
         L.moe_zc_forward_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, i32,
                                          i32, i32, vp, vp, vp]
         L.moe_zc_forward_fp8.restype = ctypes.c_int
+        L.moe_zc_forward_host_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i32, i32,
+                                              i32, i32, i32, vp, vp, i64, vp]
+        L.moe_zc_forward_host_fp8.restype = ctypes.c_int
         L.moe_zc_route.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp]
         L.moe_zc_route.restype = ctypes.c_int
         L.moe_zc_dispatch.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, vp]
@@ -216,6 +219,33 @@ def forward_fp8(x: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor, W_gate: Fp8
         _stream_ptr(stream))
     _check(st, "moe_zc_forward_fp8")
     return out
+
+
+def forward_host_fp8(x_host: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor,
+                     W_gate: Fp8Weight, W_up: Fp8Weight, W_down: torch.Tensor, N: int, Z: int,
+                     K: int, out_host: Optional[torch.Tensor] = None,
+                     logit_offset: Optional[torch.Tensor] = None, chunk_tokens: int = 0,
+                     stream=None) -> torch.Tensor:
+    """moe_zc_forward_host_fp8: forward_fp8 on CPU tensors x_host / out_host
+    (pin them for overlap).  Asynchronous on `stream`."""
+    if x_host.is_cuda or x_host.dtype != torch.bfloat16 or not x_host.is_contiguous():
+        raise ValueError("x_host must be a contiguous bf16 CPU tensor")
+    T, d = x_host.shape
+    I = int(W_gate.codes.shape[1]) if N > 0 else 0
+    if out_host is None:
+        out_host = torch.empty_like(x_host, pin_memory=x_host.is_pinned())
+    if out_host.is_cuda or out_host.dtype != torch.bfloat16 or not out_host.is_contiguous():
+        raise ValueError("out_host must be a contiguous bf16 CPU tensor")
+    bf, u8 = torch.bfloat16, torch.uint8
+    st = lib().moe_zc_forward_host_fp8(
+        x_host.data_ptr(), _dev_ptr(W_r, bf, "W_r"), _dev_ptr(b, torch.float32, "b"),
+        _dev_ptr(W_gate.codes, u8, "W_gate codes"), _dev_ptr(W_gate.scales, u8, "W_gate scales"),
+        _dev_ptr(W_up.codes, u8, "W_up codes"), _dev_ptr(W_up.scales, u8, "W_up scales"),
+        _dev_ptr(W_down, bf, "W_down"), T, d, N, Z, K, I,
+        _dev_ptr(logit_offset, torch.float32, "logit_offset"), out_host.data_ptr(),
+        chunk_tokens, _stream_ptr(stream))
+    _check(st, "moe_zc_forward_host_fp8")
+    return out_host
 
 
 def route(x: torch.Tensor, W_r: torch.Tensor, b: torch.Tensor, N: int, Z: int, K: int,

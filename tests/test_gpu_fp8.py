@@ -253,3 +253,25 @@ def test_fp8_forward_graph_replay():
     torch.cuda.synchronize()
     assert torch.equal(replayed, out)
     del g
+
+
+@pytest.mark.parametrize("chunk", [0, 256])
+def test_fp8_host_buffer_forward(chunk):
+    """moe_zc_forward_host_fp8: with one chunk it equals moe_zc_forward_fp8
+    bit for bit; with 256-token chunks each chunk equals moe_zc_forward_fp8
+    of that chunk."""
+    case = Fp8Case(wl.get("small", T=1000))
+    w, d = case.w, case.dev
+    x_host = case.x.clone().pin_memory()
+    out_host = torch.full_like(x_host, 7.0).pin_memory()
+    mz.forward_host_fp8(x_host, d["W_r"], d["b"], case.q_gate, case.q_up, case.ew.W_down,
+                        w.N, w.Z, w.K, out_host=out_host, chunk_tokens=chunk or w.T)
+    torch.cuda.synchronize()
+    mz.synchronize()
+    step = chunk or w.T
+    for t0 in range(0, w.T, step):
+        xs = d["x"][t0:t0 + step].contiguous()
+        want = mz.forward_fp8(xs, d["W_r"], d["b"], case.q_gate, case.q_up, case.ew.W_down,
+                              w.N, w.Z, w.K)
+        torch.cuda.synchronize()
+        assert torch.equal(out_host[t0:t0 + step], want.cpu()), t0
