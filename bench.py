@@ -79,11 +79,13 @@ GEMM_SOURCES = ["gemm_tcgen05.cu", "ptx.cuh", "epilogue.cuh", "kernels.cuh"]
 NCU_TRAFFIC_RATIO = {
     # workload (+ "_fp8" for the FP8 forward): (dominant kernel,
     # DRAM bytes / algorithmic bytes, GEMM sources sha16, the captured case)
-    "prefill": ("gateup_gemm", 2.9935e9 / 2.1829e9, "a50c95bdfa12e9fe",
-                "T=4096, N=32, Z=16 prefill-shaped layer (profiles/traffic_gemm_small_cases.md)"),
-    "prefill_fp8": ("gateup_gemm", 1.2903e9 / 1.1949e9, "a50c95bdfa12e9fe",
-                    "T=4096, N=32, Z=16 prefill-shaped layer (profiles/traffic_gemm_small_cases.md)"),
-    "decode_fp8": ("gateup_down_gemm (one kernel)", 0.98234e9 / 0.98599e9, "a50c95bdfa12e9fe",
+    "prefill": ("gateup_gemm", 3.5935e9 / 2.5460e9, "d892549a292a33dd",
+                "T=8192, N=32, Z=16 prefill-shaped layer (profiles/traffic_gemm_small_cases.md)"),
+    "prefill_fp8": ("gateup_gemm", 1.4650e9 / 1.4260e9, "d892549a292a33dd",
+                    "T=8192, N=32, Z=16 prefill-shaped layer (profiles/traffic_gemm_small_cases.md)"),
+    "decode": ("gateup_down_gemm (one kernel)", 1.4530e9 / 1.4525e9, "d892549a292a33dd",
+               "T=64, N=32, Z=16 decode-shaped layer (profiles/traffic_gemm_small_cases.md)"),
+    "decode_fp8": ("gateup_down_gemm (one kernel)", 0.9799e9 / 0.9860e9, "d892549a292a33dd",
                    "T=64, N=32, Z=16 decode-shaped layer (profiles/traffic_gemm_small_cases.md)"),
 }
 SUSTAINED_REGION_S = 2.0   # timed regions at least this long use the sustained bf16 peak
