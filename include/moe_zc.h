@@ -432,13 +432,6 @@ void moe_zc_test_inject(int32_t fail_allocs, int64_t wait_limit);
  */
 void moe_zc_test_one_grid(int32_t one_grid_off);
 
-/*
- * Test hook: with pair_off != 0, forwards never run the expert GEMMs on CTA
- * pairs (the single-SM kernels instead, same bits); 0 restores the default.
- * Not for production use.
- */
-void moe_zc_test_pair_off(int32_t pair_off);
-
 #ifdef __cplusplus
 }
 #endif

@@ -776,285 +776,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   }
 }
 
-// ---------------------------------------------------------------- CTA-pair expert GEMMs
-// The prefill-sized gate/up and down GEMMs on 2-CTA clusters (the two SMs of
-// a TPC), each MMA of M = 256 weight rows issued once for the pair
-// (tcgen05.mma.cta_group::2): CTA r holds rows r*128..+127 of every 256-row
-// weight block and half of the token tile's rows, and keeps its 128 rows of
-// each accumulator in its own TMEM.  A tile is (expert, token tile, 256-row
-// block pair): gate/up: W_gate and W_up rows m*256..+255 (two MMAs per K
-// step); down: W_down rows m*512..+255 and +256..+511.  Per CTA and 64-wide K
-// step that is 32 KB of weights and N/2 tokens (<= 16 KB) for 128 x N x 64 x 2
-// MMA work -- 48 KB where the single-SM kernel needs 64 KB -- so four 48 KB
-// stages fit, and the shared-memory and L2 feed per FLOP drops by a quarter.
-// Roles as in gemm_kernel; the even CTA's warp 1 issues the MMAs, both CTAs'
-// producers load into their own stages with completion counted on the even
-// CTA's barriers, the even CTA's commits release both CTAs' stages and
-// accumulators, and both CTAs' epilogue warps release the accumulators on
-// the even CTA's barriers.
-constexpr int PAIR_STAGES = 4;
-constexpr int PAIR_B_ROWS = GEMM_BN / 2;                        // tokens per CTA at most
-constexpr int PAIR_STAGE_BYTES = 2 * GEMM_A_BYTES + PAIR_B_ROWS * GEMM_BK * 2;
-constexpr int PAIR_SMEM_BYTES =
-    PAIR_STAGES * PAIR_STAGE_BYTES + GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024;
-static_assert(PAIR_SMEM_BYTES <= 227 * 1024, "pair stages exceed shared memory");
-
-struct PairTile {
-  int g, m, tok0, ntok, nmma, half, count, ntt;
-  int brow;            // this CTA's first token row of the tile
-  int a0_row, a1_row;  // this CTA's first weight row of each A block
-  bool has_a1;
-};
-
-// Pair tile t: (expert, token tile, block pair) with the block fastest; an
-// expert's token tiles share its tokens evenly (multiples of 16 tokens).
-template <int MODE>
-__device__ __forceinline__ PairTile pair_tile(const GemmParams& p, int t, uint32_t rank) {
-  PairTile tl;
-  const int lo = group_of_tile(p, t);
-  const int ttp0 = __ldg(p.grp_ttp + lo);
-  tl.ntt = __ldg(p.grp_ttp + lo + 1) - ttp0;
-  tl.g = lo;
-  const int u = t - ttp0 * p.mblocks;
-  const int j = u / p.mblocks;
-  tl.m = u - j * p.mblocks;
-  tl.count = __ldg(p.grp_count + lo);
-  const int tsz = even_tile_size(tl.count, tl.ntt, GEMM_BN);
-  tl.tok0 = j * tsz;
-  tl.ntok = min(tsz, tl.count - tl.tok0);
-  tl.nmma = (tl.ntok + 15) & ~15;
-  tl.half = tl.nmma >> 1;
-  tl.brow = __ldg(p.grp_off + lo) + tl.tok0 + static_cast<int>(rank) * tl.half;
-  const int r128 = static_cast<int>(rank) * GEMM_BM;
-  if (MODE == MODE_GATEUP) {
-    tl.a0_row = tl.g * p.a_rows + tl.m * 2 * GEMM_BM + r128;   // W_gate and W_up rows
-    tl.a1_row = tl.a0_row;
-    tl.has_a1 = true;
-  } else {
-    const int r = tl.m * 4 * GEMM_BM;
-    tl.a0_row = tl.g * p.a_rows + r + r128;
-    tl.a1_row = tl.a0_row + 2 * GEMM_BM;
-    tl.has_a1 = r + 2 * GEMM_BM < p.a_rows;
-  }
-  return tl;
-}
-
-template <int MODE>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                 const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[PAIR_STAGES];
-  __shared__ __align__(8) uint64_t empty_bar[PAIR_STAGES];
-  __shared__ __align__(8) uint64_t acc_full_bar;
-  __shared__ __align__(8) uint64_t acc_empty_bar[2];
-  __shared__ __align__(8) uint64_t drain_bar;
-  __shared__ uint32_t tmem_base_sh;
-  __shared__ volatile int abort_sh;
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < PAIR_STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
-    }
-    mbar_init(&acc_full_bar, 1);
-    for (int b = 0; b < 2; ++b) mbar_init(&acc_empty_bar[b], 2 * GEMM_EPI_WARPS);
-    mbar_init(&drain_bar, 1);
-    abort_sh = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tmA0);
-    tma_prefetch_desc(&tmA1);
-    tma_prefetch_desc(&tmB);
-  }
-  __syncwarp();
-  if (warp == 2) {
-    tmem_alloc_pair(&tmem_base_sh, 512);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();   // both CTAs' barriers exist before any cross-CTA use
-  tc_fence_after();
-  griddep_wait();
-  griddep_launch_dependents();
-  const uint32_t tmem = tmem_base_sh;
-  const int ntiles = __ldg(p.grp_ttp + p.G) * p.mblocks;
-  const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
-
-  if (warp == 0) {
-   if (lane == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
-    int stage = 0;
-    uint32_t phase = 0, armed = 0, last_par = 0;
-    for (int t = cl; t < ntiles && !abort_sh; t += ncl) {
-      const PairTile tl = pair_tile<MODE>(p, t, rank);
-      const int nbox = (tl.half + GEMM_B_BOX_ROWS - 1) / GEMM_B_BOX_ROWS;
-      // (both CTAs load the same number of bytes; the even CTA expects both)
-      const uint32_t cta_bytes =
-          GEMM_A_BYTES * (tl.has_a1 ? 2 : 1) + nbox * GEMM_B_BOX_ROWS * GEMM_BK * 2;
-      for (int ks = 0; ks < p.ksteps; ++ks) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1, p.wait_ns, p.err)) {
-          abort_sh = 1;
-          break;
-        }
-        uint8_t* st = smem + stage * PAIR_STAGE_BYTES;
-        const uint32_t bar = mapa_shared(smem_u32(&full_bar[stage]), 0);
-        if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * cta_bytes);
-        armed |= 1u << stage;
-        last_par = (last_par & ~(1u << stage)) | (phase << stage);
-        const int kc = ks * GEMM_BK;
-        tma_load_2d_pair(st, &tmA0, bar, kc, tl.a0_row);
-        if (tl.has_a1) tma_load_2d_pair(st + GEMM_A_BYTES, &tmA1, bar, kc, tl.a1_row);
-        uint8_t* sb = st + 2 * GEMM_A_BYTES;
-        for (int bx = 0; bx < nbox; ++bx)
-          tma_load_2d_pair(sb + bx * GEMM_B_BOX_ROWS * GEMM_BK * 2, &tmB, bar, kc,
-                           tl.brow + bx * GEMM_B_BOX_ROWS);
-        if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1; }
-      }
-    }
-    // Drain: the even CTA's full barriers count both CTAs' copies; the odd
-    // CTA sees its copies consumed through its empty barriers.
-    for (int s = 0; s < PAIR_STAGES; ++s)
-      if (armed & (1u << s))
-        mbar_wait(leader ? &full_bar[s] : &empty_bar[s], (last_par >> s) & 1, DRAIN_NS, p.err);
-   }
-   __syncwarp();
-  } else if (warp == 1) {
-   if (lane == 0 && leader) {
-    // ------------------------------------------------------------ MMA issuer (even CTA)
-    // commits reach the barrier at this offset in both CTAs
-    auto commit_both = [](uint64_t* bar) {
-      umma_commit_pair(smem_u32(bar));
-      umma_commit_pair(mapa_shared(smem_u32(bar), 1));
-    };
-    int stage = 0;
-    uint32_t phase = 0;
-    int local = 0;
-    for (int t = cl; t < ntiles && !abort_sh; t += ncl, ++local) {
-      const PairTile tl = pair_tile<MODE>(p, t, rank);
-      const uint32_t par = static_cast<uint32_t>(local - 1) & 1u;
-      if (local > 0 && !mbar_wait(&acc_empty_bar[0], par, p.wait_ns, p.err)) {
-        abort_sh = 1;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(2 * GEMM_BM, tl.nmma);
-      const int nk = p.ksteps;
-      // as in gemm_kernel: after the first tile, the first stages feed the
-      // first accumulator alone until the second is handed back
-      const int npre = local > 0 ? min(nk, PAIR_STAGES) : 0;
-      bool ok = true;
-      const int stage0 = stage;
-      auto kstep = [&](uint32_t d, uint32_t a_smem, uint32_t b_smem, bool first) {
-        const uint64_t ad = smem_desc_sw128(a_smem);
-        const uint64_t bd = smem_desc_sw128(b_smem);
-#pragma unroll
-        for (int kk = 0; kk < GEMM_BK / 16; ++kk)
-          umma_bf16_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, (first && kk == 0) ? 0u : 1u);
-      };
-      for (int i = 0; i < npre; ++i) {
-        if (!mbar_wait(&full_bar[stage], phase, p.wait_ns, p.err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t st = smem_u32(smem + stage * PAIR_STAGE_BYTES);
-        kstep(tmem, st, st + 2 * GEMM_A_BYTES, i == 0);
-        if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1; }
-      }
-      if (ok && npre > 0) {
-        if (!mbar_wait(&acc_empty_bar[1], par, p.wait_ns, p.err)) {
-          ok = false;
-        } else {
-          tc_fence_after();
-          int s = stage0;
-          for (int i = 0; i < npre; ++i) {
-            const uint32_t st = smem_u32(smem + s * PAIR_STAGE_BYTES);
-            if (tl.has_a1) kstep(tmem + 256, st + GEMM_A_BYTES, st + 2 * GEMM_A_BYTES, i == 0);
-            commit_both(&empty_bar[s]);
-            if (++s == PAIR_STAGES) s = 0;
-          }
-        }
-      }
-      for (int i = npre; ok && i < nk; ++i) {
-        if (!mbar_wait(&full_bar[stage], phase, p.wait_ns, p.err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t st = smem_u32(smem + stage * PAIR_STAGE_BYTES);
-        kstep(tmem, st, st + 2 * GEMM_A_BYTES, i == 0);
-        if (tl.has_a1) kstep(tmem + 256, st + GEMM_A_BYTES, st + 2 * GEMM_A_BYTES, i == 0);
-        commit_both(&empty_bar[stage]);
-        if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1; }
-      }
-      if (!ok) { abort_sh = 1; break; }
-      commit_both(&acc_full_bar);
-    }
-    // Drain: all MMAs issued by this thread finish before TMEM is freed.
-    umma_commit_pair(smem_u32(&drain_bar));
-    mbar_wait(&drain_bar, 0, DRAIN_NS, p.err);
-   }
-   __syncwarp();
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;
-    const int group = (warp - 4) >> 2;
-    const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    uint8_t* stg = smem + PAIR_STAGES * PAIR_STAGE_BYTES + (warp - 4) * GEMM_STG_BYTES;
-    const uint32_t empty0 = mapa_shared(smem_u32(&acc_empty_bar[0]), 0);
-    const uint32_t empty1 = mapa_shared(smem_u32(&acc_empty_bar[1]), 0);
-    // each warp releases an accumulator on the even CTA's barrier
-    auto release = [&](uint32_t cl_addr) {
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(cl_addr);
-    };
-    int local = 0;
-    for (int t = cl; t < ntiles && !abort_sh; t += ncl, ++local) {
-      const PairTile pt = pair_tile<MODE>(p, t, rank);
-      if (!mbar_wait(&acc_full_bar, local & 1, p.wait_ns, p.err)) {
-        abort_sh = 1;
-        break;
-      }
-      tc_fence_after();
-      // the epilogue helpers take a Tile: its token range and output rows
-      Tile tl;
-      tl.tok0 = pt.tok0;
-      tl.nmma = pt.nmma;
-      tl.count = pt.count;
-      tl.brow0 = __ldg(p.grp_off + pt.g) + pt.tok0;
-      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-      uint32_t hp[3][16];
-      if (MODE == MODE_GATEUP) {
-        epi_read_bf16<MODE_GATEUP>(tq, group, tl.nmma, hp, 256);
-        release(empty0);
-        release(empty1);
-        // H columns of this CTA's rows of the block pair
-        const int f = pt.m * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM + q * 32;
-        epi_store_bf16(stg, lane, group, tl, hp, out + f, p.out_ld, 0);
-      } else {
-        const int f = pt.m * 4 * GEMM_BM + static_cast<int>(rank) * GEMM_BM + q * 32;
-        epi_read_bf16<MODE_DOWN>(tq, group, tl.nmma, hp);
-        release(empty0);
-        epi_store_bf16(stg, lane, group, tl, hp, out + f, p.out_ld, 0);
-        if (pt.has_a1) epi_read_bf16<MODE_DOWN>(tq + 256, group, tl.nmma, hp);
-        release(empty1);
-        if (pt.has_a1) epi_store_bf16(stg, lane, group, tl, hp, out + f + 2 * GEMM_BM, p.out_ld, 0);
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();   // the pair's MMAs, copies and remote arrivals are over
-  if (warp == 2) {
-    tc_fence_after();
-    tmem_dealloc_pair(tmem, 512);
-  }
-}
-
 // a2, b2, p2: MODE_FUSED's down phase (other modes: copies of a0, b, p).
 template <int MODE, int NST, int SB, bool FP8 = false>
 cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
@@ -1130,26 +851,6 @@ cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, cons
   // is returned as is, without cudaGetLastError, for the caller to clear)
   return launch_mode<MODE_FUSED, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>(
       wg, wu, xp, xp, wd, h, pg, pd, grid, stream);
-}
-
-cudaError_t launch_gemm_pair(GemmMode mode, const CUtensorMap& a0, const CUtensorMap& a1,
-                             const CUtensorMap& b, const GemmParams& p, int clusters,
-                             cudaStream_t stream) {
-  if (clusters <= 0) return cudaSuccess;
-  cudaError_t e;
-  if (mode == MODE_GATEUP) {
-    if ((e = smem_limit<gemm_pair_kernel<MODE_GATEUP>>(PAIR_SMEM_BYTES)) != cudaSuccess) return e;
-    e = launch_pdl_pairs(gemm_pair_kernel<MODE_GATEUP>, dim3(2 * clusters), dim3(GEMM_THREADS),
-                         PAIR_SMEM_BYTES, stream, a0, a1, b, p);
-  } else if (mode == MODE_DOWN) {
-    if ((e = smem_limit<gemm_pair_kernel<MODE_DOWN>>(PAIR_SMEM_BYTES)) != cudaSuccess) return e;
-    e = launch_pdl_pairs(gemm_pair_kernel<MODE_DOWN>, dim3(2 * clusters), dim3(GEMM_THREADS),
-                         PAIR_SMEM_BYTES, stream, a0, a1, b, p);
-  } else {
-    return cudaErrorInvalidValue;
-  }
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
 }
 
 int fused_resident_blocks() {

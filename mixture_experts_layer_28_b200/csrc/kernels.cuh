@@ -236,14 +236,6 @@ cudaError_t launch_gemm_fused_fp8(const CUtensorMap& wg, const CUtensorMap& wu,
                                   const CUtensorMap& xp8, const CUtensorMap& wd,
                                   const CUtensorMap& h, const GemmParams& pg,
                                   const GemmParams& pd, int grid, cudaStream_t stream);
-// The prefill-sized gate/up (I % 256 == 0) or down (d % 256 == 0) GEMM on
-// 2-CTA clusters with pair MMAs (cta_group::2, M = 256): maps a0 / a1 of
-// W_gate / W_up (gate/up) or W_down twice (down) with 128-row boxes, b with
-// 32-row boxes; p.mblocks = I / 256 (gate/up) or ceil(d / 512) (down),
-// p.grp_ttp the GEMM_BN-token tile prefix; `clusters` pairs are launched.
-cudaError_t launch_gemm_pair(GemmMode mode, const CUtensorMap& a0, const CUtensorMap& a1,
-                             const CUtensorMap& b, const GemmParams& p, int clusters,
-                             cudaStream_t stream);
 // Blocks of the one-grid expert GEMM kernel the current device holds at once
 // (its occupancy times the multiprocessors).
 int fused_resident_blocks();

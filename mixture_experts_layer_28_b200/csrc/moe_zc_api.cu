@@ -235,7 +235,6 @@ struct Plan {
   int kernels = 0;
 };
 bool g_one_grid_off = false;    // test hook: never use the one grid
-bool g_pair_off = false;        // test hook: never use the CTA-pair expert GEMMs
 
 Plan make_plan(int64_t T, int d, int N, int Z, int K, int I, int sms, int64_t resident,
                bool fp8 = false) {
@@ -598,12 +597,6 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
         pg.sfa1 = f8->up_sf;
         pg.sfb = static_cast<const uint8_t*>(c.sfx.p);
       }
-      // Prefill-sized bf16 batches run the expert GEMMs on CTA pairs (pair
-      // MMAs of M = 256: a quarter less operand feed per FLOP), unless the
-      // tiles are being paced on clusters of the single-SM kernel
-      const bool pair = !f8 && !g_pair_off && T >= 8192 && !pace_tiles;
-      const bool pair_gu = pair && I % (2 * GEMM_BM) == 0;
-      const bool pair_dn = pair && d % (2 * GEMM_BM) == 0;
       bool one_grid = plan.one_grid;
       if (one_grid) {
         // 5-6  at most 64 tokens: both expert GEMMs in one persistent grid,
@@ -634,32 +627,15 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       }
       if (!one_grid) {
         // 5  gate/up GEMM
-        const int64_t tiles_ub = (T * K + GEMM_BN - 1) / GEMM_BN + N;
-        const int64_t pair_max = c.sms / 2;
-        if (f8) {
+        if (f8)
           CK(launch_gemm_gateup_fp8(mWg, mWu, mXp, mXpf, pg, static_cast<int>(plan.gateup_grid),
                                     st));
-        } else if (pair_gu) {
-          GemmParams pp = pg;
-          pp.mblocks = I / (2 * GEMM_BM);
-          const int64_t ub = tiles_ub * pp.mblocks;
-          CK(launch_gemm_pair(MODE_GATEUP, mWg, mWu, mXp, pp,
-                              static_cast<int>(ub < pair_max ? ub : pair_max), st));
-        } else {
+        else
           CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg,
                          static_cast<int>(plan.gateup_grid), st));
-        }
         rec.mark(5);
         // 6  down GEMM
-        if (pair_dn) {
-          GemmParams pp = pd;
-          pp.mblocks = (d + 4 * GEMM_BM - 1) / (4 * GEMM_BM);
-          const int64_t ub = tiles_ub * pp.mblocks;
-          CK(launch_gemm_pair(MODE_DOWN, mWd, mWd, mH, pp,
-                              static_cast<int>(ub < pair_max ? ub : pair_max), st));
-        } else {
-          CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd, static_cast<int>(plan.down_grid), st));
-        }
+        CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd, static_cast<int>(plan.down_grid), st));
         rec.mark(6);
       }
     } else {
@@ -1187,11 +1163,6 @@ int moe_zc_plan(int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I
   plan->expert_gemms_one_grid = pl.one_grid ? 1 : 0;
   plan->expert_grid = static_cast<int32_t>(pl.one_grid ? pl.fused_grid : pl.gateup_grid);
   return MOE_ZC_OK;
-}
-
-void moe_zc_test_pair_off(int32_t pair_off) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  g_pair_off = pair_off != 0;
 }
 
 void moe_zc_test_one_grid(int32_t one_grid_off) {

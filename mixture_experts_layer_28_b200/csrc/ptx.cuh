@@ -341,62 +341,6 @@ __device__ __forceinline__ bool wait_count_geq(const int* p, int target, long lo
   }
 }
 
-// ---------------------------------------------------------------- CTA pairs (cta_group::2)
-// The two CTAs of a 2-CTA cluster (the two SMs of a TPC) run one MMA of
-// M = 256 rows together: each holds 128 rows of A and half of B's columns in
-// its shared memory (same offsets) and 128 rows of the accumulator in its
-// TMEM.  The even CTA issues the MMAs.
-
-// Arrive on an mbarrier given by its cluster-window address (may be the peer's).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr)
-               : "memory");
-}
-
-// TMA load into this CTA's shared memory whose completion is counted on an
-// mbarrier of either CTA of the pair (cluster-window address).
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map,
-                                                 uint32_t bar_cl, int32_t c0, int32_t c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cl), "r"(c0), "r"(c1)
-      : "memory");
-}
-
-// TMEM allocation shared by the pair: issued by the same warp in both CTAs.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
-               ::"r"(smem_u32(dst)), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
-// Pair MMA (issued by the even CTA): D[256 x N] over both CTAs' TMEM, A rows
-// 0..127 from this CTA's shared memory and 128..255 from the peer's, B
-// columns N/2 + N/2 the same way; bf16 in, fp32 accumulate.
-__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                               uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive on the mbarrier at cluster-window address cl_addr (this CTA's or
-// the peer's) once the pair MMAs issued so far by this thread are done.
-__device__ __forceinline__ void umma_commit_pair(uint32_t cl_addr) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-               ::"r"(cl_addr) : "memory");
-}
-
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 

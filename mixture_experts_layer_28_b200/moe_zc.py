@@ -105,8 +105,6 @@ def lib() -> ctypes.CDLL:
         L.moe_zc_plan.restype = ctypes.c_int
         L.moe_zc_test_one_grid.argtypes = [i32]
         L.moe_zc_test_one_grid.restype = None
-        L.moe_zc_test_pair_off.argtypes = [i32]
-        L.moe_zc_test_pair_off.restype = None
         L.moe_zc_fp8_quantize_weights.argtypes = [vp, i64, i32, vp, vp, vp]
         L.moe_zc_fp8_quantize_weights.restype = ctypes.c_int
         L.moe_zc_forward_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, i32,
@@ -491,11 +489,6 @@ def plan(T: int, d: int, N: int, Z: int, K: int, I: int, sms: int = 148,
     _check(lib().moe_zc_plan(T, d, N, Z, K, I, sms, resident_blocks, ctypes.byref(p)),
            "moe_zc_plan")
     return {name: getattr(p, name) for name, _ in LaunchPlan._fields_}
-
-
-def test_pair_off(off: bool) -> None:
-    """Test hook: keep the expert GEMMs off CTA pairs (single-SM kernels)."""
-    lib().moe_zc_test_pair_off(1 if off else 0)
 
 
 def test_one_grid(off: bool) -> None:

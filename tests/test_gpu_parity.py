@@ -370,33 +370,3 @@ def test_device_wait_timeout_is_reported(T):
         mz.synchronize()
     assert ei.value.status == mz.ERR_TIMEOUT
     _full_check(case)
-
-
-@pytest.mark.parametrize("case_id", ["small9000", "one_block_pair", "half_down_pair", "hot_expert"])
-def test_cta_pair_gemms_match_single_sm(case_id):
-    """Batches of >= 8192 tokens run the expert GEMMs on 2-CTA clusters with
-    pair MMAs (M = 256).  Against the single-SM kernels (forced by the test
-    hook) every output, routing and histogram bit is equal, and the oracle
-    agrees.  Cases: ragged token tiles; I = d = 256 (one 256-row block pair
-    for gate/up, one single block for down); d = 768 (the last down tile has
-    one 256-row block); one expert holding 8500 tokens (34 token tiles)."""
-    if case_id == "small9000":
-        case = Case(wl.get("small", T=9000))
-    elif case_id == "one_block_pair":
-        case = Case(wl.get("tiny", T=8200, d=256, I=256))
-    elif case_id == "half_down_pair":
-        case = Case(wl.get("tiny", T=8192, d=768, I=512))
-    else:
-        w = wl.get("small", T=8500)
-        case = Case(w, T=8500, bias=_bias_hot_expert(w, 3, 8500))
-    o1, i1, g1, c1 = _gpu_result(case)
-    mz.test_pair_off(True)
-    try:
-        o2, i2, g2, c2 = _gpu_result(case)
-    finally:
-        mz.test_pair_off(False)
-    assert np.array_equal(i1, i2) and np.array_equal(c1, c2)
-    assert np.array_equal(o1, o2)
-    _sampled_check(case, n_rows=192, n_expert_checks=4)
-    if case_id == "hot_expert":
-        assert check_expert_rows(case, 3, max_rows=600) > 0
