@@ -80,13 +80,13 @@ NCU_TRAFFIC_RATIO = {
     # workload (+ "_fp8" for the FP8 forward): (dominant kernel,
     # DRAM bytes / algorithmic bytes, GEMM sources sha16, the captured case)
     "prefill": ("gateup_gemm", 3.5935e9 / 2.5460e9, "d892549a292a33dd",
-                "T=8192, N=32, Z=16 prefill-shaped layer (profiles/traffic_gemm_small_cases.md)"),
+                "T=8192, N=32, Z=16 prefill-shaped layer, ncu DRAM counters of two launches"),
     "prefill_fp8": ("gateup_gemm", 1.4650e9 / 1.4260e9, "d892549a292a33dd",
-                    "T=8192, N=32, Z=16 prefill-shaped layer (profiles/traffic_gemm_small_cases.md)"),
+                    "T=8192, N=32, Z=16 prefill-shaped layer, ncu DRAM counters of two launches"),
     "decode": ("gateup_down_gemm (one kernel)", 1.4530e9 / 1.4525e9, "d892549a292a33dd",
-               "T=64, N=32, Z=16 decode-shaped layer (profiles/traffic_gemm_small_cases.md)"),
+               "T=64, N=32, Z=16 decode-shaped layer, ncu DRAM counters of two launches"),
     "decode_fp8": ("gateup_down_gemm (one kernel)", 0.9799e9 / 0.9860e9, "d892549a292a33dd",
-                   "T=64, N=32, Z=16 decode-shaped layer (profiles/traffic_gemm_small_cases.md)"),
+                   "T=64, N=32, Z=16 decode-shaped layer, ncu DRAM counters of two launches"),
 }
 SUSTAINED_REGION_S = 2.0   # timed regions at least this long use the sustained bf16 peak
 NOMINAL_HBM_GBS = 7700.0   # B200 HBM3e, HGX figure (context beside the measured copy peak)
