@@ -75,7 +75,7 @@ def kernels_per_forward(w, sms=148):
 # the GEMM engine's sources at the capture.  `traffic` = ratio x the
 # algorithmic bytes of this run's launch (traffic scales with the units a
 # launch processes); null when the sources have changed since the capture.
-GEMM_SOURCES = ["gemm_tcgen05.cu", "ptx.cuh", "epilogue.cuh", "kernels.cuh"]
+GEMM_SOURCES = ["gemm_tcgen05.cu", "ptx.cuh", "epilogue.cuh", "kernels.cuh", "step.cuh"]
 NCU_TRAFFIC_RATIO = {
     # workload (+ "_fp8" for the FP8 forward): (dominant kernel,
     # DRAM bytes / algorithmic bytes, GEMM sources sha16, the captured case)
@@ -279,10 +279,11 @@ def routing_stats(w, cnt):
                 max_load=int(ffn.max()) if w.N else 0)
 
 
-def roofline_numbers(w, st, pk, fp8=False):
+def roofline_numbers(w, st, pk, fp8=False, splits=1):
     """Algorithmic FLOPs and bytes of the layer and of its kernels.  fp8: the
     gate/up weights and permuted tokens are E4M3 bytes plus one scale byte
-    per 32 elements; the down projection stays bf16."""
+    per 32 elements; the down projection stays bf16.  splits: the router
+    GEMM's K slices."""
     P, hit = st["ffn_pairs"], st["experts_hit"]
     d, I, T, E = w.d, w.I, w.T, w.E
     gu = (1.0 + 1.0 / 32) if fp8 else 2.0      # bytes per gate/up weight or token element
@@ -292,8 +293,14 @@ def roofline_numbers(w, st, pk, fp8=False):
     B_down = hit * 1.0 * I * d * 2 + P * I * 2 + P * d * 2        # weights + H in + Y out
     F_layer = F_gateup + F_down
     B_layer = hit * (2.0 * d * I * gu + d * I * 2) + E * d * 2 + E * 4 + 2.0 * T * d * 2
+    # the rest of the forward, for a kernel that also routes, dispatches and
+    # combines (the decode step's one grid): the router's K slices of partial
+    # logits read; picks, gates, slots and zsum written; x read twice (copy
+    # and combine), the permuted tokens written, Y read back, out written
+    B_phases = (splits * T * E * 4 + T * w.K * 12 + T * 4 + 2.0 * T * d * 2 + P * d * gu
+                + P * d * 2 + T * d * 2)
     return dict(F_gateup=F_gateup, F_down=F_down, B_gateup=B_gateup, B_down=B_down,
-                F_layer=F_layer, B_layer=B_layer, fp8=fp8)
+                F_layer=F_layer, B_layer=B_layer, B_phases=B_phases, fp8=fp8)
 
 
 # ----------------------------------------------------------------- oracle timing
@@ -366,9 +373,12 @@ def kernel_roofline(w, rf, plan, per, pk, region_s, clk=None):
     """The dominant stage's achieved rate against its bound."""
     dom = max(per, key=per.get)
     # (with the one-grid expert GEMMs the gate/up stage is the kernel that
-    # runs both)
+    # runs both; with the decode step in that grid, also route, dispatch and
+    # combine, whose bytes it then moves too)
     one_grid = bool(plan["expert_gemms_one_grid"])
-    kern = {"gateup_gemm": ((rf["F_gateup"] + rf["F_down"], rf["B_gateup"] + rf["B_down"])
+    step = bool(plan.get("one_grid_step"))
+    kern = {"gateup_gemm": ((rf["F_gateup"] + rf["F_down"],
+                             rf["B_gateup"] + rf["B_down"] + (rf["B_phases"] if step else 0.0))
                             if one_grid else (rf["F_gateup"], rf["B_gateup"])),
             "down_gemm": (rf["F_down"], rf["B_down"])}.get(dom)
     if not kern or per[dom] <= 0:
@@ -390,7 +400,10 @@ def kernel_roofline(w, rf, plan, per, pk, region_s, clk=None):
                 "frac": ach / pk["hbm"],
                 "peak_kind": f"HBM copy, read + write ({pk['src']}, MEASURED_PEAKS.json)",
                 "frac_of_nominal_hbm": ach / NOMINAL_HBM_GBS}
-    roof["kernel"] = "gateup_down_gemm (one kernel)" if one_grid and dom == "gateup_gemm" else dom
+    roof["kernel"] = dom
+    if one_grid and dom == "gateup_gemm":
+        roof["kernel"] = ("decode_step (route, dispatch, gate/up + down GEMMs, combine: one kernel)"
+                          if step else "gateup_down_gemm (one kernel)")
     roof["ms_per_launch"] = per[dom]
     roof["algorithmic_bytes"] = B
     roof["algorithmic_flops"] = F
@@ -460,7 +473,7 @@ def measure(args, dist, w, steps, e2e_steps, headline, fp8=False):
     torch.cuda.synchronize()
     mz.synchronize()
     st = routing_stats(w, mz.expert_load(w.E))
-    rf = roofline_numbers(w, st, pk, fp8=fp8)
+    rf = roofline_numbers(w, st, pk, fp8=fp8, splits=plan["router_k_slices"])
     if steps <= 0:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)

@@ -225,6 +225,11 @@ int moe_zc_fp8_quantize(const void* W, int64_t rows, int64_t cols, int32_t mode,
  *                           (batches of at most 64 tokens whose grid can be
  *                           resident at once), 0: two launches
  *   expert_grid             blocks of that one grid, or of the gate/up GEMM
+ *   one_grid_step           1: that grid also routes the tokens, assigns their
+ *                           slots, copies them into the GEMM's token buffer
+ *                           and combines the outputs (phases separated by grid
+ *                           barriers), so the forward is two kernels: the
+ *                           router GEMM and that grid
  * Returns the forward's argument-check status (nothing is written unless
  * MOE_ZC_OK), or MOE_ZC_ERR_INVALID_ARG for a NULL plan or sms < 1.
  */
@@ -235,6 +240,7 @@ typedef struct moe_zc_launch_plan {
   int32_t router_k_slices;
   int32_t expert_gemms_one_grid;
   int32_t expert_grid;
+  int32_t one_grid_step;
 } moe_zc_launch_plan;
 int moe_zc_plan(int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I,
                 int32_t sms, int32_t resident_blocks, moe_zc_launch_plan* plan);
@@ -426,11 +432,14 @@ int moe_zc_route_noalloc(const void* x, const void* W_r, const float* b,
 void moe_zc_test_inject(int32_t fail_allocs, int64_t wait_limit);
 
 /*
- * Test hook: with one_grid_off != 0, forwards never run the two expert GEMMs
- * of small batches in one grid (the fallback path, same bits); 0 restores
- * the default.  Not for production use.
+ * Test hook for the launch paths of batches of at most 64 tokens (all give
+ * the same bits): mode 1 never runs the two expert GEMMs in one grid (the
+ * fallback path); mode 2 runs them in one grid but routes, dispatches and
+ * combines in kernels of their own; 0 (or any other value) restores the
+ * default, where the one grid does all but the router GEMM.  Not for
+ * production use.
  */
-void moe_zc_test_one_grid(int32_t one_grid_off);
+void moe_zc_test_one_grid(int32_t mode);
 
 #ifdef __cplusplus
 }

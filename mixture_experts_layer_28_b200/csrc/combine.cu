@@ -15,18 +15,10 @@
 // with 16-byte loads.
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "step.cuh"
 
 namespace moezc {
 namespace {
-
-__device__ __forceinline__ void acc8(float (&a)[8], const uint4& v, float g) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    a[2 * i] = fmaf(g, __uint_as_float(w[i] << 16), a[2 * i]);
-    a[2 * i + 1] = fmaf(g, __uint_as_float(w[i] & 0xFFFF0000u), a[2 * i + 1]);
-  }
-}
 
 __global__ void combine_kernel(const uint4* __restrict__ x, const uint4* __restrict__ Y,
                                const int* __restrict__ slot, const float* __restrict__ gate,
@@ -51,21 +43,8 @@ __global__ void combine_kernel(const uint4* __restrict__ x, const uint4* __restr
   __syncthreads();
   const float z = zsum[t];
   const int n = nffn;
-  for (int c = c_begin + threadIdx.x; c < c_end; c += blockDim.x) {
-    float a[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] = 0.f;
-    acc8(a, x[t * d8 + c], z);
-    for (int k = 0; k < n; ++k) acc8(a, Y[static_cast<int64_t>(sl[k]) * d8 + c], gt[k]);
-    uint4 o;
-    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __nv_bfloat162 h = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
-      ow[i] = *reinterpret_cast<const uint32_t*>(&h);
-    }
-    out[t * d8 + c] = o;
-  }
+  for (int c = c_begin + threadIdx.x; c < c_end; c += blockDim.x)
+    out[t * d8 + c] = combine_chunk(x, Y, t, c, d8, z, sl, gt, n);
   // many waves of CTAs: let dependents launch only as the last ones finish
   griddep_launch_dependents();
 }

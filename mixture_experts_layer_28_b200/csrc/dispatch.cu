@@ -24,40 +24,12 @@
 // The histogram itself is integer and comes from the router, so it is exact.
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "step.cuh"
 
 namespace moezc {
 namespace {
 
 constexpr int ASSIGN_THREADS = 256;
-
-// Exclusive prefix sum of v over the CTA (ASSIGN_THREADS threads), with the
-// CTA's total in *total.
-__device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total) {
-  constexpr int W = ASSIGN_THREADS / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < W ? warp_sums[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < W; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += u;
-    }
-    if (lane < W) warp_sums[lane] = w;   // inclusive prefix over warps
-  }
-  __syncthreads();
-  const int base = warp ? warp_sums[warp - 1] : 0;
-  *total = warp_sums[W - 1];
-  __syncthreads();
-  return base + incl - v;
-}
 
 __global__ void __launch_bounds__(ASSIGN_THREADS)
 assign_slots_kernel(const int* __restrict__ cnt, const int* __restrict__ idx, int64_t pairs,
@@ -73,16 +45,16 @@ assign_slots_kernel(const int* __restrict__ cnt, const int* __restrict__ idx, in
     const int g = base + threadIdx.x;
     const int c = g < N ? cnt[g] : 0;
     int tot_rows, tot_tiles = 0, tot_tiles8 = 0;
-    const int off = block_excl_scan((c + pad - 1) / pad * pad, warp_sums, &tot_rows);
+    const int off = block_excl_scan<ASSIGN_THREADS>((c + pad - 1) / pad * pad, warp_sums, &tot_rows);
     if (g < N) off_s[g] = carry_rows + off;
     if (blockIdx.x == 0) {
-      const int ttp = block_excl_scan((c + GEMM_BN - 1) / GEMM_BN, warp_sums, &tot_tiles);
+      const int ttp = block_excl_scan<ASSIGN_THREADS>((c + GEMM_BN - 1) / GEMM_BN, warp_sums, &tot_tiles);
       if (g < N) {
         grp_off[g] = carry_rows + off;
         grp_ttp[g] = carry_tiles + ttp;
       }
       if (grp_ttp8) {   // (uniform over the CTA)
-        const int t8 = block_excl_scan((c + FP8_BN - 1) / FP8_BN, warp_sums, &tot_tiles8);
+        const int t8 = block_excl_scan<ASSIGN_THREADS>((c + FP8_BN - 1) / FP8_BN, warp_sums, &tot_tiles8);
         if (g < N) grp_ttp8[g] = carry_tiles8 + t8;
       }
     }

@@ -19,72 +19,12 @@
 //   permute (FP8)      each token row is quantised once, its codes go to the
 //                      token's FFN slots of Xp8 and its scales to the atoms
 //                      of the gate/up token tiles that hold those slots
-#include <cuda_fp8.h>
-
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "step.cuh"
 
 namespace moezc {
 namespace {
-
-// UE8M0 byte of the smallest power of two 2^k with amax <= 448 * 2^k (amax > 0,
-// finite).  With amax = (1 + m / 2^23) 2^(E - 127) and 448 = 1.75 * 2^8:
-// k = E - 135, plus one when the significand exceeds 1.75 (m > 0x600000).
-// Subnormal amax (and anything needing k < -127) takes the floor 2^-127.
-__device__ __forceinline__ uint32_t ue8m0_of_amax(float amax) {
-  const uint32_t bits = __float_as_uint(amax);
-  const int E = static_cast<int>((bits >> 23) & 0xFF);
-  if (amax == 0.f || E == 0xFF) return 127u;   // zero, or a NaN / infinity in the block
-  if (E == 0) return 0u;
-  int k = E - 135 + ((bits & 0x7FFFFF) > 0x600000u ? 1 : 0);
-  k = k < -127 ? -127 : (k > 127 ? 127 : k);
-  return static_cast<uint32_t>(k + 127);
-}
-
-// 2^-k as a float, exactly (k in [-127, 127]).
-__device__ __forceinline__ float inv_pow2(int k) {
-  return k <= 126 ? __uint_as_float(static_cast<uint32_t>(127 - k) << 23)
-                  : __uint_as_float(0x00400000u);   // 2^-127 (subnormal)
-}
-
-// 32 bf16 values (8 per uint4) -> their E4M3 codes (4 per uint32) and the
-// block's UE8M0 scale byte.  value / 2^k is exact in fp32, and the
-// conversion rounds to nearest, ties to even (it never saturates:
-// |value| / 2^k <= 448).
-__device__ __forceinline__ uint32_t quantize32(const uint4 (&v)[4], uint32_t (&codes)[8]) {
-  float f[32];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[q * 8 + 2 * i] = bf16_lo(w[i]);
-      f[q * 8 + 2 * i + 1] = bf16_hi(w[i]);
-    }
-  }
-  float amax = 0.f;
-  bool finite = true;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float a = fabsf(f[i]);
-    finite = finite && (__float_as_uint(a) < 0x7F800000u);
-    amax = fmaxf(amax, a);
-  }
-  const uint32_t sf = finite ? ue8m0_of_amax(amax) : 127u;
-  const float inv = inv_pow2(static_cast<int>(sf) - 127);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __nv_fp8_storage_t c =
-          __nv_cvt_float_to_fp8(f[4 * i + j] * inv, __NV_SATFINITE, __NV_E4M3);
-      word |= static_cast<uint32_t>(c) << (8 * j);
-    }
-    codes[i] = word;
-  }
-  return sf;
-}
 
 __global__ void fp8_quantize_weights_kernel(const uint4* __restrict__ W, int64_t rows, int cols,
                                             uint4* __restrict__ codes, uint8_t* __restrict__ sf) {
@@ -132,8 +72,7 @@ __global__ void permute_fp8_kernel(const uint4* __restrict__ x, const int* __res
       const int pos = u - j * tsz;                 // the token's place in its tile
       const int64_t tile = ttp0 + j;
       row_s[n] = static_cast<int64_t>(s) * d;
-      sf_s[n] = tile * (d / 128) * (2 * SF_ATOM_BYTES) + (pos / 128) * SF_ATOM_BYTES +
-                (pos % 32) * 16 + ((pos % 128) / 32) * 4;
+      sf_s[n] = token_sf_base(tile, pos, d);
       ++n;
     }
     npick = n;

@@ -54,6 +54,7 @@
 #include "epilogue.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "step.cuh"
 
 namespace moezc {
 namespace {
@@ -78,32 +79,43 @@ struct Tile {
   int ttile;    // expert GEMMs: the tile's index among all token tiles (FP8 scale atoms)
 };
 
+// The expert offsets and counts a tile is decoded from: written by earlier
+// kernels (read-only here: the non-coherent path), or -- in the one grid
+// that runs the whole decode step -- by this grid's own assign phase (COH):
+// plain loads, which after the grid barrier's acquire see those writes and
+// then hit in L1 (no block reads these words before that barrier).
+template <bool COH>
+__device__ __forceinline__ int ld_meta(const int* p) {
+  return COH ? *p : __ldg(p);
+}
+
 __device__ __forceinline__ int router_tok_tile(const GemmParams& p) {
   return p.tok_tile > 0 ? p.tok_tile : GEMM_BN;
 }
 
-template <int MODE>
+template <int MODE, bool COH = false>
 __device__ __forceinline__ int total_tiles(const GemmParams& p) {
   if (MODE == MODE_ROUTER) {
     const int tt = router_tok_tile(p);
     return ((p.T + tt - 1) / tt) * p.mblocks * (p.ksplit > 1 ? p.ksplit : 1);
   }
-  return __ldg(p.grp_ttp + p.G) * p.mblocks;
+  return ld_meta<COH>(p.grp_ttp + p.G) * p.mblocks;
 }
 
 // Group (expert) of expert-GEMM tile t: the largest g with ttp[g] <= t / mblocks
 // (a group's tiles start at ttp[g] * mblocks).
+template <bool COH = false>
 __device__ __forceinline__ int group_of_tile(const GemmParams& p, int t) {
   const int tt = t / p.mblocks;
   int lo = 0, hi = p.G - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(p.grp_ttp + mid) <= tt) lo = mid; else hi = mid - 1;
+    if (ld_meta<COH>(p.grp_ttp + mid) <= tt) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
 
-template <int MODE>
+template <int MODE, bool COH = false>
 __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   Tile tl;
   tl.split = 0;
@@ -126,15 +138,15 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
     tl.count = p.T;
     tl.brow0 = 0;
   } else {
-    const int lo = group_of_tile(p, t);
+    const int lo = group_of_tile<COH>(p, t);
     tl.g = lo;
     // Order inside the group: weight block fastest, so that the tiles of a
     // round of the persistent grid share a few weight blocks and token
     // tiles; but an expert with two token tiles goes weight block by weight
     // block with its two token tiles adjacent (tiles 2i and 2i + 1 read the
     // same weight block).
-    const int ttp0 = __ldg(p.grp_ttp + lo);
-    const int ntt = __ldg(p.grp_ttp + lo + 1) - ttp0;
+    const int ttp0 = ld_meta<COH>(p.grp_ttp + lo);
+    const int ntt = ld_meta<COH>(p.grp_ttp + lo + 1) - ttp0;
     tl.ntt = ntt;
     const int u = t - ttp0 * p.mblocks;
     if (ntt == 2) {
@@ -144,8 +156,8 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
       j = u / p.mblocks;
       tl.m = u - j * p.mblocks;
     }
-    tl.count = __ldg(p.grp_count + lo);
-    tl.brow0 = __ldg(p.grp_off + lo);
+    tl.count = ld_meta<COH>(p.grp_count + lo);
+    tl.brow0 = ld_meta<COH>(p.grp_off + lo);
   }
   // An expert's ntt = ceil(count / tile) token tiles share its tokens evenly
   // (sizes a multiple of 16): two tiles of similar size run side by side in
@@ -156,7 +168,7 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   tl.ttile = 0;
   if (MODE != MODE_ROUTER) {
     tsz = even_tile_size(tl.count, tl.ntt, tsz);
-    tl.ttile = __ldg(p.grp_ttp + tl.g) + j;
+    tl.ttile = ld_meta<COH>(p.grp_ttp + tl.g) + j;
   }
   tl.tok0 = j * tsz;
   tl.ntok = min(tsz, tl.count - tl.tok0);
@@ -212,7 +224,8 @@ __device__ __forceinline__ bool tile_at(const GemmParams& p, int it, int n0, int
 template <int MODE>
 __device__ __forceinline__ Tile phase_tile(const GemmParams& p, const GemmParams& p2, int tph,
                                            int t) {
-  if (MODE == MODE_FUSED) return tph ? decode_tile<MODE_DOWN>(p2, t) : decode_tile<MODE_GATEUP>(p, t);
+  if (MODE == MODE_FUSED)
+    return tph ? decode_tile<MODE_DOWN, true>(p2, t) : decode_tile<MODE_GATEUP, true>(p, t);
   return decode_tile<MODE>(p, t);
 }
 
@@ -356,7 +369,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
             const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBf,
             const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-            const GemmParams p, const GemmParams p2) {
+            const GemmParams p, const GemmParams p2, const __grid_constant__ StepParams sp) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[NST];
   __shared__ __align__(8) uint64_t empty_bar[NST];
@@ -373,6 +386,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   __shared__ volatile int tile_q[TILE_Q];
   __shared__ __align__(8) uint64_t tq_full[TILE_Q];
   __shared__ __align__(8) uint64_t tq_empty[TILE_Q];
+  __shared__ volatile int bar_ok_sh;   // grid barriers of the decode step
   const bool dyn =
       (MODE == MODE_GATEUP || MODE == MODE_DOWN) && p.tile_counter != nullptr && !p.pair_tiles;
 
@@ -426,9 +440,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     for (int i = threadIdx.x; i < p.nzero0; i += blockDim.x) p.zero0[i] = 0;
     for (int i = threadIdx.x; i < p.nzero1; i += blockDim.x) p.zero1[i] = 0;
   }
+  // The whole decode step (sp.on): route, then assign and permute, each
+  // followed by a grid barrier, before the expert tiles; the combine after
+  // them.  Every block passes every barrier (a wait that runs out records
+  // DEV_TIMEOUT), but the work after a failed one is skipped.
+  uint8_t* ws = smem + NST * SB;   // the epilogue staging area
+  bool step_ok = true;
+  int nbar = 0;
+  if (MODE == MODE_FUSED && sp.on) {
+    const int G = static_cast<int>(gridDim.x);
+    step_route<GEMM_THREADS>(sp, ws);
+    step_ok = grid_barrier(sp.gbar, ++nbar * G, p.wait_ns, p.err, &bar_ok_sh, step_ok);
+    if (step_ok) step_assign_permute<GEMM_THREADS, FP8>(sp, ws);
+    step_ok = grid_barrier(sp.gbar, ++nbar * G, p.wait_ns, p.err, &bar_ok_sh, step_ok);
+    if (!step_ok && threadIdx.x == 0) abort_sh = 1;
+    __syncthreads();
+  }
   const uint32_t tmem = tmem_base_sh;
-  const int ntiles = total_tiles<MODE == MODE_FUSED ? MODE_GATEUP : MODE>(p);
-  const int ntiles2 = MODE == MODE_FUSED ? total_tiles<MODE_DOWN>(p2) : 0;
+  const int ntiles = total_tiles<MODE == MODE_FUSED ? MODE_GATEUP : MODE, MODE == MODE_FUSED>(p);
+  const int ntiles2 = MODE == MODE_FUSED ? total_tiles<MODE_DOWN, true>(p2) : 0;
   // gate/up tiles always hold two blocks; router and down tiles hold one
   // when p.single_a is set (1 buffer of 512 columns, or 2 of 256)
   // (MODE_FUSED: both phases hold two blocks)
@@ -483,7 +513,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         // gate/up tiles has counted itself; the acquire and the proxy fence
         // order this CTA's bulk copies of them after those stores
         const int need =
-            GEMM_EPI_WARPS * p.mblocks * (__ldg(p.grp_ttp + tl.g + 1) - __ldg(p.grp_ttp + tl.g));
+            GEMM_EPI_WARPS * p.mblocks *
+            (ld_meta<true>(p.grp_ttp + tl.g + 1) - ld_meta<true>(p.grp_ttp + tl.g));
         if (!wait_count_geq(p.done + tl.g, need, p.wait_ns, p.err)) {
           abort_sh = 1;
           break;
@@ -687,7 +718,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
     uint8_t* stg = smem + NST * SB + (warp - 4) * GEMM_STG_BYTES;
     // H / Y rows are written once here; hint them only for streaming batches
-    const uint64_t pol_out = p.l2_stream ? l2_policy_evict_first() : 0;
+    // whose next reader is another kernel (the one grid reads H back, and
+    // the combine reads Y right after it: default policy)
+    const uint64_t pol_out = p.l2_stream && MODE != MODE_FUSED ? l2_policy_evict_first() : 0;
     for (int local = 0; !abort_sh; ++local) {
       int tph, t;
       if (dyn) {
@@ -774,13 +807,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (MODE == MODE_FUSED && sp.on) {
+    // every Y row is stored once all blocks are here
+    step_ok = grid_barrier(sp.gbar, ++nbar * static_cast<int>(gridDim.x), p.wait_ns, p.err,
+                           &bar_ok_sh, step_ok && !abort_sh);
+    if (step_ok) step_combine<GEMM_THREADS>(sp, ws);
+  }
 }
 
 // a2, b2, p2: MODE_FUSED's down phase (other modes: copies of a0, b, p).
+// sp: the decode step's phases (MODE_FUSED; off elsewhere).
 template <int MODE, int NST, int SB, bool FP8 = false>
 cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                         const CUtensorMap& b_full, const CUtensorMap& a2, const CUtensorMap& b2,
-                        GemmParams p, const GemmParams& p2, int grid, cudaStream_t stream) {
+                        GemmParams p, const GemmParams& p2, int grid, cudaStream_t stream,
+                        const StepParams& sp = StepParams{}) {
   constexpr int smem = NST * SB + GEMM_EPI_WARPS * GEMM_STG_BYTES + 1024;
   const cudaError_t e = smem_limit<gemm_kernel<MODE, NST, SB, FP8>>(smem);
   if (e != cudaSuccess) return e;
@@ -788,7 +829,8 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   if (p.pair_tiles) {
     if (grid >= 2) {
       return launch_pdl_pairs(gemm_kernel<MODE, NST, SB, FP8>, dim3(grid & ~1),
-                              dim3(GEMM_THREADS), smem, stream, a0, a1, b, b_full, a2, b2, p, p2);
+                              dim3(GEMM_THREADS), smem, stream, a0, a1, b, b_full, a2, b2, p, p2,
+                              StepParams{});
     }
     p.pair_tiles = 0;
   }
@@ -796,9 +838,9 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   // tiles: every block must be resident at once
   if (MODE == MODE_FUSED)
     return launch_pdl_coop(gemm_kernel<MODE, NST, SB, FP8>, dim3(grid), dim3(GEMM_THREADS), smem,
-                           stream, a0, a1, b, b_full, a2, b2, p, p2);
+                           stream, a0, a1, b, b_full, a2, b2, p, p2, sp);
   return launch_pdl(gemm_kernel<MODE, NST, SB, FP8>, dim3(grid), dim3(GEMM_THREADS), smem, stream,
-                    a0, a1, b, b_full, a2, b2, p, p2);
+                    a0, a1, b, b_full, a2, b2, p, p2, StepParams{});
 }
 
 // The stage shapes: prefill (3 x 64 KB) and at most 64 tokens (5 x 40 KB).
@@ -840,17 +882,29 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
   return cudaGetLastError();
 }
 
+// A decode step (step.on) wants the barrier counter, sizes the phases can
+// hold in the staging area (N + Z <= MOE_MAX_E_INTERNAL, K <= 32) and its
+// output buffers.
+static bool step_args_ok(const StepParams& s, const GemmParams& pg, bool fp8) {
+  if (!s.on) return true;
+  return s.gbar && s.T > 0 && s.T <= GEMM_SMALL_B && s.E <= MOE_MAX_E_INTERNAL && s.N > 0 &&
+         s.N <= s.E && s.K > 0 && s.K <= 32 && s.splits >= 1 && s.logits && s.bias && s.idx &&
+         s.gate && s.zsum && s.cnt == pg.grp_count && s.slot && s.fill && s.grp_off == pg.grp_off &&
+         s.grp_ttp && s.x && s.Y && s.out && (fp8 ? (s.Xp8 && s.sfx && s.grp_ttp8) : s.Xp != nullptr);
+}
+
 cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, const CUtensorMap& xp,
                               const CUtensorMap& wd, const CUtensorMap& h, const GemmParams& pg,
-                              const GemmParams& pd, int grid, cudaStream_t stream) {
+                              const GemmParams& pd, int grid, cudaStream_t stream,
+                              const StepParams& step) {
   if (grid <= 0) return cudaSuccess;
   if (grid > device_sms() || !pg.small_b || pg.pair_tiles || pg.b_box_full || pd.single_a ||
-      pg.done == nullptr)
+      pg.done == nullptr || !step_args_ok(step, pg, false))
     return cudaErrorInvalidValue;
   // (a refused cooperative launch leaves nothing queued: launch_mode's error
   // is returned as is, without cudaGetLastError, for the caller to clear)
   return launch_mode<MODE_FUSED, GEMM_SMALL_STAGES, GEMM_SMALL_STAGE_BYTES>(
-      wg, wu, xp, xp, wd, h, pg, pd, grid, stream);
+      wg, wu, xp, xp, wd, h, pg, pd, grid, stream, step);
 }
 
 int fused_resident_blocks() {
@@ -886,14 +940,15 @@ cudaError_t launch_gemm_gateup_fp8(const CUtensorMap& wg, const CUtensorMap& wu,
 cudaError_t launch_gemm_fused_fp8(const CUtensorMap& wg, const CUtensorMap& wu,
                                   const CUtensorMap& xp8, const CUtensorMap& wd,
                                   const CUtensorMap& h, const GemmParams& pg,
-                                  const GemmParams& pd, int grid, cudaStream_t stream) {
+                                  const GemmParams& pd, int grid, cudaStream_t stream,
+                                  const StepParams& step) {
   if (grid <= 0) return cudaSuccess;
   if (grid > device_sms() || !pg.small_b || pg.pair_tiles || pg.b_box_full || pd.single_a ||
       pg.done == nullptr || pg.tok_tile != FP8_BN || !pg.sfa0 || !pg.sfa1 || !pg.sfb ||
-      pg.sf_kgroups != pg.ksteps)
+      pg.sf_kgroups != pg.ksteps || !step_args_ok(step, pg, true))
     return cudaErrorInvalidValue;
   return launch_mode<MODE_FUSED, FP8_SMALL_STAGES, FP8_SMALL_STAGE_BYTES, true>(
-      wg, wu, xp8, xp8, wd, h, pg, pd, grid, stream);
+      wg, wu, xp8, xp8, wd, h, pg, pd, grid, stream, step);
 }
 
 }  // namespace moezc

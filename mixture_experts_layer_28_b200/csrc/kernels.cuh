@@ -207,6 +207,43 @@ struct GemmParams {
   int* tile_counter;
 };
 
+// The rest of a forward of at most GEMM_SMALL_B tokens, run by the one-grid
+// expert GEMMs (launch_gemm_fused with step.on) around their tiles, as
+// phases separated by grid barriers (the grid is resident as a whole):
+//   route    the router's K slices summed and each token routed (softmax,
+//            biased top-K, gates, zsum, histogram), as launch_route does
+//   assign   expert offsets from the histogram (grp_off, grp_ttp and, for
+//            FP8, grp_ttp8 stored for the tiles), a slot for each FFN pick
+//            and the token copied into its slots (bf16 rows, or FP8 codes
+//            and scale atoms), as launch_assign_slots and launch_permute(_fp8)
+//   experts  the gate/up and down tiles
+//   combine  out_t = zsum_t x_t + sum_k gate_{t,k} Y[slot_{t,k}], as launch_combine
+// The histogram, fill counters and *gbar are zero at launch.
+struct StepParams {
+  int on;
+  int T, E, N, K, d;
+  const float* logits;       // [splits][T, E] partial router logits
+  int splits;
+  const float* bias;         // [E]
+  const float* offset;       // [E] or null
+  int* idx;                  // [T, K] out
+  float* gate;               // [T, K] out
+  float* zsum;               // [T] out
+  int* cnt;                  // [E] histogram out
+  int* slot;                 // [T, K] out
+  int* fill;                 // [N] slot counters
+  int* grp_off;              // [N + 1] out
+  int* grp_ttp;              // [N + 1] out (GEMM_BN-token tiles)
+  int* grp_ttp8;             // [N + 1] out (FP8_BN-token tiles), FP8 only
+  const __nv_bfloat16* x;    // [T, d]
+  __nv_bfloat16* Xp;         // bf16 permuted rows, or
+  uint8_t* Xp8;              // FP8 codes and
+  uint8_t* sfx;              //   scale atoms of the token tiles
+  const __nv_bfloat16* Y;    // [rows, d] the down tiles' output
+  __nv_bfloat16* out;        // [T, d]
+  int* gbar;                 // grid barrier counter
+};
+
 // b: B map with GEMM_B_BOX_ROWS-row boxes; b_full: with GEMM_BN-row boxes,
 // used for full token tiles when p.b_box_full is set.  With p.pair_tiles the
 // grid (rounded down to even) runs as 2-CTA clusters.
@@ -222,7 +259,8 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
 // separate launches instead.
 cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, const CUtensorMap& xp,
                               const CUtensorMap& wd, const CUtensorMap& h, const GemmParams& pg,
-                              const GemmParams& pd, int grid, cudaStream_t stream);
+                              const GemmParams& pd, int grid, cudaStream_t stream,
+                              const StepParams& step);
 // The FP8 gate/up GEMM (E4M3 maps of W_gate, W_up [N*I, d] with [128 x 128]
 // boxes and of the quantised tokens Xp8 with [128 x 32] boxes, b_full with
 // FP8_BN-row boxes; p.tok_tile = FP8_BN, p.grp_ttp the FP8_BN-tile prefix,
@@ -235,7 +273,8 @@ cudaError_t launch_gemm_gateup_fp8(const CUtensorMap& wg, const CUtensorMap& wu,
 cudaError_t launch_gemm_fused_fp8(const CUtensorMap& wg, const CUtensorMap& wu,
                                   const CUtensorMap& xp8, const CUtensorMap& wd,
                                   const CUtensorMap& h, const GemmParams& pg,
-                                  const GemmParams& pd, int grid, cudaStream_t stream);
+                                  const GemmParams& pd, int grid, cudaStream_t stream,
+                                  const StepParams& step);
 // Blocks of the one-grid expert GEMM kernel the current device holds at once
 // (its occupancy times the multiprocessors).
 int fused_resident_blocks();

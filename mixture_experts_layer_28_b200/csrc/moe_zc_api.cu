@@ -231,10 +231,16 @@ struct Plan {
   RouterPlan rp;
   int64_t router_grid = 0;
   bool one_grid = false;        // gate/up and down GEMMs in one persistent grid
+  bool step = false;            // ... which also routes, dispatches and combines
   int64_t gateup_grid = 0, down_grid = 0, fused_grid = 0;
   int kernels = 0;
 };
-bool g_one_grid_off = false;    // test hook: never use the one grid
+// test hook: 0 default, 1 never the one grid, 2 the one grid for the expert
+// GEMMs only (route, dispatch and combine in their own kernels)
+int g_one_grid_mode = 0;
+
+// Counters that the router GEMM clears for each forward (see reserve_impl).
+constexpr int kFillInts(int N) { return 2 * N + 5; }
 
 Plan make_plan(int64_t T, int d, int N, int Z, int K, int I, int sms, int64_t resident,
                bool fp8 = false) {
@@ -256,8 +262,11 @@ Plan make_plan(int64_t T, int d, int N, int Z, int K, int I, int sms, int64_t re
   pl.gateup_grid = g_ub < sms ? g_ub : sms;
   pl.down_grid = d_ub < sms ? d_ub : sms;
   pl.fused_grid = g_ub + d_ub < sms ? g_ub + d_ub : sms;
-  pl.one_grid = T <= GEMM_SMALL_B && !g_one_grid_off && pl.fused_grid <= resident;
-  pl.kernels = pl.one_grid ? 6 : 7;
+  pl.one_grid = T <= GEMM_SMALL_B && g_one_grid_mode != 1 && pl.fused_grid <= resident;
+  // the one grid also runs route, assign, permute and combine: the router
+  // GEMM and that grid are the whole forward
+  pl.step = pl.one_grid && g_one_grid_mode != 2;
+  pl.kernels = pl.step ? 2 : (pl.one_grid ? 6 : 7);
   return pl;
 }
 
@@ -280,9 +289,10 @@ int reserve_impl(Ctx& c, int64_t T, int d, int N, int Z, int K, int I, bool fp8 
   if ((s = ensure(c, c.slot, static_cast<size_t>(pairs) * sizeof(int))) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.zsum, static_cast<size_t>(T) * sizeof(float))) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.cnt, static_cast<size_t>(E) * sizeof(int))) != MOE_ZC_OK) return s;
-  // fill: [N + 1] slot counters, [N + 1] gate/up completion counters, then
-  // the gate/up and down GEMMs' tile counters
-  if ((s = ensure(c, c.fill, static_cast<size_t>(2 * N + 4) * sizeof(int))) != MOE_ZC_OK) return s;
+  // fill: [N + 1] slot counters, [N + 1] gate/up completion counters, the
+  // gate/up and down GEMMs' tile counters, the decode step's grid barrier
+  if ((s = ensure(c, c.fill, static_cast<size_t>(kFillInts(N)) * sizeof(int))) != MOE_ZC_OK)
+    return s;
   if ((s = ensure(c, c.grp_off, static_cast<size_t>(N + 1) * sizeof(int))) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.grp_ttp, static_cast<size_t>(N + 1) * sizeof(int))) != MOE_ZC_OK) return s;
   if (N > 0) {
@@ -466,16 +476,17 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
   if (T > 0 && given) {
     // 1-2  the caller's routing: one pick per row, gate 1, no zero experts
     CK(cudaMemsetAsync(cnt, 0, sizeof(int) * E, st));
-    CK(cudaMemsetAsync(fill, 0, sizeof(int) * (2 * N + 4), st));
+    CK(cudaMemsetAsync(fill, 0, sizeof(int) * kFillInts(N), st));
     CK(launch_given_routing(given->expert, T, given->base, N, idx, gate, zsum, cnt, st));
     rec.mark(1);
     rec.mark(2);
   }
   if (T > 0) {
+    const RouterPlan rp = plan.rp;
+    const int splits = rp.splits;
    if (!given) {
     // 1  router GEMM
     CUtensorMap mWr, mX;
-    const RouterPlan rp = plan.rp;
     // x in boxes of 32 tokens, and of one full token tile (rp.tok_tile)
     CUtensorMap mXf;
     const bool full_ok = T >= rp.tok_tile;
@@ -493,11 +504,10 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     pr.wait_ns = wait_ns;
     // Few token tiles (decode): single blocks and K slices so that every SM
     // streams a part of W_r; the slices' partial logits are summed in slice
-    // order by the route kernel.
+    // order by the route kernel (or the decode step's route phase).
     pr.mblocks = rp.mblocks;
     pr.single_a = rp.single_a;
     pr.tok_tile = rp.tok_tile;
-    const int splits = rp.splits;
     pr.ksplit = splits;
     pr.split_stride = T * E;
     pr.b_box_full = full_ok ? 1 : 0;
@@ -505,29 +515,27 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
     pr.zero0 = cnt;
     pr.nzero0 = E;
     pr.zero1 = fill;
-    pr.nzero1 = 2 * N + 4;
+    pr.nzero1 = kFillInts(N);
     CK(launch_gemm(MODE_ROUTER, mWr, mWr, mX, mXf, pr, static_cast<int>(plan.router_grid), st));
     rec.mark(1);
-    // 2  route
-    CK(launch_route(static_cast<const float*>(c.logits.p), b, off, T, E, N, K, idx, gate, zsum,
-                    cnt, st, splits));
-    rec.mark(2);
    }
+    // 2  route (unless the decode step's one grid does it)
+    auto route = [&]() -> int {
+      if (given) return MOE_ZC_OK;
+      CK(launch_route(static_cast<const float*>(c.logits.p), b, off, T, E, N, K, idx, gate, zsum,
+                      cnt, st, splits));
+      rec.mark(2);
+      return MOE_ZC_OK;
+    };
+    // 7  combine
+    auto combine = [&]() -> int {
+      CK(launch_combine(static_cast<const __nv_bfloat16*>(x),
+                        static_cast<const __nv_bfloat16*>(c.Y.p), slot, gate, zsum, T, d, K,
+                        static_cast<__nv_bfloat16*>(out), st));
+      return MOE_ZC_OK;
+    };
     if (N > 0) {
-      // 3-4  dispatch
-      CK(launch_assign_slots(cnt, idx, T * K, N, grp_off, grp_ttp, fill, slot, st, grp_ttp8));
-      rec.mark(3);
-      if (f8) {
-        // each token row quantised once (E4M3, 1 x 32 blocks) into its slots
-        CK(launch_permute_fp8(static_cast<const __nv_bfloat16*>(x), idx, slot, cnt, grp_off,
-                              grp_ttp8, T, d, K, N, static_cast<uint8_t*>(c.Xp8.p),
-                              static_cast<uint8_t*>(c.sfx.p), st));
-      } else {
-        CK(launch_permute(static_cast<const __nv_bfloat16*>(x), slot, T, d, K,
-                          static_cast<__nv_bfloat16*>(c.Xp.p), st));
-      }
-      rec.mark(4);
-      // 5  gate/up GEMM
+      // the expert GEMMs' maps and parameters (host only)
       CUtensorMap mWg, mWu, mXp;
       if (!make_map(&mWg, W_gate, static_cast<uint64_t>(N) * I, d, GEMM_BM) ||
           !make_map(&mWu, W_up, static_cast<uint64_t>(N) * I, d, GEMM_BM) ||
@@ -597,55 +605,115 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
         pg.sfa1 = f8->up_sf;
         pg.sfb = static_cast<const uint8_t*>(c.sfx.p);
       }
-      bool one_grid = plan.one_grid;
-      if (one_grid) {
-        // 5-6  at most 64 tokens: both expert GEMMs in one persistent grid,
-        // the down tiles of an expert starting as soon as its H rows are
-        // stored (the SMs that the last round of gate/up tiles leaves idle
-        // stream down weights meanwhile); a gate/up tile costs about d / I
-        // down tiles
-        GemmParams pf = pg;
-        pf.b_box_full = 0;
-        pf.done = fill + N + 1;
-        pf.down_lead = (d + I / 2) / I;
-        const cudaError_t e =
-            f8 ? launch_gemm_fused_fp8(mWg, mWu, mXp, mWd, mH, pf, pd,
-                                       static_cast<int>(plan.fused_grid), st)
-               : launch_gemm_fused(mWg, mWu, mXp, mWd, mH, pf, pd,
-                                   static_cast<int>(plan.fused_grid), st);
-        if (e != cudaSuccess) {
-          // refused as a cooperative launch (its blocks cannot all be
-          // resident): nothing was queued; run the two launches from now on
-          cudaGetLastError();
-          if (captured) return MOE_ZC_ERR_CUDA;   // (the capture is invalidated)
-          c.one_grid_refused = true;
-          one_grid = false;
-        } else {
-          rec.mark(5);
-          rec.mark(6);
+      // At most 64 tokens: both expert GEMMs in one persistent grid, the
+      // down tiles of an expert starting as soon as its H rows are stored
+      // (the SMs that the last round of gate/up tiles leaves idle stream down
+      // weights meanwhile); a gate/up tile costs about d / I down tiles.
+      GemmParams pf = pg;
+      pf.b_box_full = 0;
+      pf.done = fill + N + 1;
+      pf.down_lead = (d + I / 2) / I;
+      auto one_grid_launch = [&](const StepParams& sp) {
+        return f8 ? launch_gemm_fused_fp8(mWg, mWu, mXp, mWd, mH, pf, pd,
+                                          static_cast<int>(plan.fused_grid), st, sp)
+                  : launch_gemm_fused(mWg, mWu, mXp, mWd, mH, pf, pd,
+                                      static_cast<int>(plan.fused_grid), st, sp);
+      };
+      // a refused cooperative launch (its blocks cannot all be resident)
+      // queues nothing: the forward goes on with separate launches, and so do
+      // the later ones
+      auto refused = [&]() -> int {
+        cudaGetLastError();
+        if (captured) return MOE_ZC_ERR_CUDA;   // (the capture is invalidated)
+        c.one_grid_refused = true;
+        return MOE_ZC_OK;
+      };
+      bool stepped = false;
+      if (plan.step && !given) {
+        // 2-7  the rest of the forward in the one grid: route, assign and
+        // permute, the expert tiles, combine
+        StepParams sp{};
+        sp.on = 1;
+        sp.T = static_cast<int>(T);
+        sp.E = E;
+        sp.N = N;
+        sp.K = K;
+        sp.d = d;
+        sp.logits = static_cast<const float*>(c.logits.p);
+        sp.splits = splits;
+        sp.bias = b;
+        sp.offset = off;
+        sp.idx = idx;
+        sp.gate = gate;
+        sp.zsum = zsum;
+        sp.cnt = cnt;
+        sp.slot = slot;
+        sp.fill = fill;
+        sp.grp_off = grp_off;
+        sp.grp_ttp = grp_ttp;
+        sp.grp_ttp8 = grp_ttp8;
+        sp.x = static_cast<const __nv_bfloat16*>(x);
+        sp.Xp = static_cast<__nv_bfloat16*>(c.Xp.p);
+        sp.Xp8 = f8 ? static_cast<uint8_t*>(c.Xp8.p) : nullptr;
+        sp.sfx = f8 ? static_cast<uint8_t*>(c.sfx.p) : nullptr;
+        sp.Y = static_cast<const __nv_bfloat16*>(c.Y.p);
+        sp.out = static_cast<__nv_bfloat16*>(out);
+        sp.gbar = fill + 2 * N + 4;
+        for (int i = 2; i <= 4; ++i) rec.mark(i);
+        if (one_grid_launch(sp) == cudaSuccess) {
+          for (int i = 5; i <= 6; ++i) rec.mark(i);
+          stepped = true;
+        } else if ((s = refused()) != MOE_ZC_OK) {
+          return s;
         }
       }
-      if (!one_grid) {
-        // 5  gate/up GEMM
-        if (f8)
-          CK(launch_gemm_gateup_fp8(mWg, mWu, mXp, mXpf, pg, static_cast<int>(plan.gateup_grid),
-                                    st));
-        else
-          CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg,
-                         static_cast<int>(plan.gateup_grid), st));
-        rec.mark(5);
-        // 6  down GEMM
-        CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd, static_cast<int>(plan.down_grid), st));
-        rec.mark(6);
+      if (!stepped) {
+        if ((s = route()) != MOE_ZC_OK) return s;
+        // 3-4  dispatch
+        CK(launch_assign_slots(cnt, idx, T * K, N, grp_off, grp_ttp, fill, slot, st, grp_ttp8));
+        rec.mark(3);
+        if (f8) {
+          // each token row quantised once (E4M3, 1 x 32 blocks) into its slots
+          CK(launch_permute_fp8(static_cast<const __nv_bfloat16*>(x), idx, slot, cnt, grp_off,
+                                grp_ttp8, T, d, K, N, static_cast<uint8_t*>(c.Xp8.p),
+                                static_cast<uint8_t*>(c.sfx.p), st));
+        } else {
+          CK(launch_permute(static_cast<const __nv_bfloat16*>(x), slot, T, d, K,
+                            static_cast<__nv_bfloat16*>(c.Xp.p), st));
+        }
+        rec.mark(4);
+        bool one_grid = plan.one_grid && !c.one_grid_refused;
+        if (one_grid) {
+          // 5-6  the expert GEMMs in the one grid
+          if (one_grid_launch(StepParams{}) == cudaSuccess) {
+            rec.mark(5);
+            rec.mark(6);
+          } else {
+            if ((s = refused()) != MOE_ZC_OK) return s;
+            one_grid = false;
+          }
+        }
+        if (!one_grid) {
+          // 5  gate/up GEMM
+          if (f8)
+            CK(launch_gemm_gateup_fp8(mWg, mWu, mXp, mXpf, pg, static_cast<int>(plan.gateup_grid),
+                                      st));
+          else
+            CK(launch_gemm(MODE_GATEUP, mWg, mWu, mXp, mXpf, pg,
+                           static_cast<int>(plan.gateup_grid), st));
+          rec.mark(5);
+          // 6  down GEMM
+          CK(launch_gemm(MODE_DOWN, mWd, mWd, mH, mHf, pd, static_cast<int>(plan.down_grid), st));
+          rec.mark(6);
+        }
+        if ((s = combine()) != MOE_ZC_OK) return s;
       }
     } else {
+      if ((s = route()) != MOE_ZC_OK) return s;
       CK(launch_assign_slots(cnt, idx, T * K, N, grp_off, grp_ttp, fill, slot, st));
       for (int i = 3; i <= 6; ++i) rec.mark(i);
+      if ((s = combine()) != MOE_ZC_OK) return s;
     }
-    // 7  combine
-    CK(launch_combine(static_cast<const __nv_bfloat16*>(x),
-                      static_cast<const __nv_bfloat16*>(c.Y.p), slot, gate, zsum, T, d, K,
-                      static_cast<__nv_bfloat16*>(out), st));
   } else {
     for (int i = 1; i <= 6; ++i) rec.mark(i);
   }
@@ -1162,12 +1230,13 @@ int moe_zc_plan(int64_t T, int32_t d, int32_t N, int32_t Z, int32_t K, int32_t I
   plan->router_k_slices = pl.rp.splits;
   plan->expert_gemms_one_grid = pl.one_grid ? 1 : 0;
   plan->expert_grid = static_cast<int32_t>(pl.one_grid ? pl.fused_grid : pl.gateup_grid);
+  plan->one_grid_step = pl.step ? 1 : 0;
   return MOE_ZC_OK;
 }
 
-void moe_zc_test_one_grid(int32_t one_grid_off) {
+void moe_zc_test_one_grid(int32_t mode) {
   std::lock_guard<std::mutex> lk(g_mu);
-  g_one_grid_off = one_grid_off != 0;
+  g_one_grid_mode = (mode == 1 || mode == 2) ? mode : 0;
 }
 
 void moe_zc_test_inject(int32_t fail_allocs, int64_t wait_limit) {

@@ -46,7 +46,8 @@ class LaunchPlan(ctypes.Structure):
     """moe_zc_launch_plan (include/moe_zc.h)."""
     _fields_ = [("kernels", ctypes.c_int32), ("router_grid", ctypes.c_int32),
                 ("router_token_tile", ctypes.c_int32), ("router_k_slices", ctypes.c_int32),
-                ("expert_gemms_one_grid", ctypes.c_int32), ("expert_grid", ctypes.c_int32)]
+                ("expert_gemms_one_grid", ctypes.c_int32), ("expert_grid", ctypes.c_int32),
+                ("one_grid_step", ctypes.c_int32)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -491,9 +492,11 @@ def plan(T: int, d: int, N: int, Z: int, K: int, I: int, sms: int = 148,
     return {name: getattr(p, name) for name, _ in LaunchPlan._fields_}
 
 
-def test_one_grid(off: bool) -> None:
-    """Test hook: keep small batches off the one-grid expert GEMMs."""
-    lib().moe_zc_test_one_grid(1 if off else 0)
+def test_one_grid(off: bool = False, step: bool = True) -> None:
+    """Test hook for batches of at most 64 tokens: off keeps them off the
+    one-grid expert GEMMs; step=False keeps route, dispatch and combine out
+    of that grid."""
+    lib().moe_zc_test_one_grid(1 if off else (0 if step else 2))
 
 
 def declared_symbols() -> list[str]:

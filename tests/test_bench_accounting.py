@@ -16,9 +16,10 @@ from mixture_experts_layer_28_b200 import workloads as wl  # noqa: E402
 def test_launches_per_forward():
     # router GEMM, route, assign, permute, gate/up, down, combine
     assert bench.kernels_per_forward(wl.get("prefill")) == 7
-    # at most 64 tokens: the two expert GEMMs are one kernel
-    assert bench.kernels_per_forward(wl.get("decode")) == 6
-    assert bench.kernels_per_forward(wl.get("tiny", T=64)) == 6
+    # at most 64 tokens: the router GEMM, then one grid that routes,
+    # dispatches, runs both expert GEMMs and combines
+    assert bench.kernels_per_forward(wl.get("decode")) == 2
+    assert bench.kernels_per_forward(wl.get("tiny", T=64)) == 2
     assert bench.kernels_per_forward(wl.get("tiny", T=65)) == 7
     # no FFN experts: no dispatch to experts, no GEMM (assign still clears slots)
     assert bench.kernels_per_forward(wl.get("tiny", N=0, Z=12, K=3)) == 4
@@ -97,6 +98,25 @@ def test_decode_one_grid_roofline_is_hbm_bound():
     assert roof["bound"] == "hbm" and roof["kernel"].startswith("gateup_down_gemm")
     assert abs(roof["achieved"] - 2.279e9 / 0.35e-3 / 1e9) < 5
     assert abs(roof["frac_of_nominal_hbm"] - roof["achieved"] / 7700.0) < 1e-12
+
+
+def test_decode_step_kernel_counts_its_phases_bytes():
+    """Decode with the whole step in the one grid: besides the expert GEMMs'
+    2.279 GB the kernel reads the router's 24 K slices of partial logits
+    (24 x 64 x 768 fp32), writes picks, gates and slots (64 x 12 x 3 x 4 B)
+    and zsum, reads x twice, writes the 460 permuted rows, reads the 460 Y
+    rows back and writes out: 18.4 MB more."""
+    w = wl.get("decode")
+    rf = bench.roofline_numbers(w, dict(ffn_pairs=460, experts_hit=30), None, splits=24)
+    phases = (24 * 64 * 768 * 4 + 64 * 12 * 12 + 64 * 4 + 2 * 64 * 6144 * 2 + 460 * 6144 * 2
+              + 460 * 6144 * 2 + 64 * 6144 * 2)
+    assert rf["B_phases"] == phases
+    assert abs(phases / 1e6 - 18.4) < 0.05
+    plan = dict(expert_gemms_one_grid=1, one_grid_step=1)
+    roof = bench.kernel_roofline(w, rf, plan, {"gateup_gemm": 0.36}, _pk(), region_s=1.0)
+    assert roof["kernel"].startswith("decode_step")
+    assert roof["algorithmic_bytes"] == rf["B_gateup"] + rf["B_down"] + phases
+    assert abs(roof["achieved"] - roof["algorithmic_bytes"] / 0.36e-3 / 1e9) < 1e-6
 
 
 def test_clock_samples_outside_the_region_are_dropped():

@@ -181,17 +181,24 @@ def test_hot_expert_fp8():
     assert _check_expert_rows_fp8(case, 3, max_rows=1100) == 1100
 
 
-def test_decode_sized_fp8_one_grid_and_fallback_agree():
-    """48 tokens: gate/up (FP8) and down (bf16) in one grid, and with the one
-    grid switched off, two launches: the same bits, and the oracle agrees."""
-    case = Fp8Case(wl.get("decode", d=1024, I=512, T=48))
-    o1, i1, _, c1 = _gpu_fp8(case)
-    mz.test_one_grid(True)
-    try:
-        o2, i2, _, c2 = _gpu_fp8(case)
-    finally:
-        mz.test_one_grid(False)
-    assert np.array_equal(o1, o2) and np.array_equal(i1, i2) and np.array_equal(c1, c2)
+@pytest.mark.parametrize("over", [dict(d=1024, I=512, T=48), dict(d=384, I=256, T=64, N=40,
+                                                                   Z=20, K=6)])
+def test_decode_sized_fp8_launch_paths_agree(over):
+    """At most 64 tokens: the one grid that also routes, quantises the tokens
+    into their slots and combines (the default); the one grid for gate/up
+    (FP8) and down (bf16) only; and separate launches: the same bits, and the
+    oracle agrees."""
+    case = Fp8Case(wl.get("decode", **over))
+    res = []
+    for path in [dict(off=False, step=True), dict(off=False, step=False), dict(off=True)]:
+        mz.test_one_grid(**path)
+        try:
+            res.append(_gpu_fp8(case))
+        finally:
+            mz.test_one_grid(False)
+    for o, i, _, c in res[1:]:
+        assert np.array_equal(res[0][0], o) and np.array_equal(res[0][1], i)
+        assert np.array_equal(res[0][3], c)
     _check_fp8(case)
 
 

@@ -262,19 +262,67 @@ def test_decode_sized_expert_gemms_match_two_kernel_path():
         assert torch.equal(fused[k][0], plain[k][0]) and torch.equal(fused[k][1], plain[k][1]), k
 
 
+# The launch paths of a batch of at most 64 tokens, through the test hook:
+# the one grid routing, dispatching, running both expert GEMMs and combining
+# (the default: two kernels per forward); the one grid running the expert
+# GEMMs only; and separate launches (the path taken when the cooperative
+# launch is refused).
+PATHS = [dict(off=False, step=True), dict(off=False, step=False), dict(off=True)]
+
+
+def _result_on_path(case, path, fn):
+    mz.test_one_grid(**path)
+    try:
+        return fn(case)
+    finally:
+        mz.test_one_grid(False)
+
+
+@pytest.mark.parametrize("over", [dict(d=1024, I=512), dict(T=1, d=512, I=256),
+                                  dict(T=37, d=192, I=256, N=40, Z=20, K=6),
+                                  dict(T=64, d=320, I=384, N=24, Z=8, K=8)])
+def test_small_batch_launch_paths_give_the_same_bits(over):
+    """Output, routing and histogram are the same bits on every path, and
+    the default path is the oracle's within the parity bounds."""
+    case = Case(wl.get("decode", **over))
+    w = case.w
+    p = mz.plan(case.T, w.d, w.N, w.Z, w.K, w.I)
+    assert p["one_grid_step"] == 1 and p["kernels"] == 2
+    res = [_result_on_path(case, path, _gpu_result) for path in PATHS]
+    for o, i, g, c in res[1:]:
+        assert np.array_equal(res[0][0], o) and np.array_equal(res[0][1], i)
+        assert np.array_equal(res[0][2], g) and np.array_equal(res[0][3], c)
+    _full_check(case)
+
+
+def test_small_batch_step_assigns_valid_slots():
+    """The slots the one grid assigns: the rows of FFN expert e's range (from
+    its first row, count rows) hold exactly the tokens that picked e, each
+    once; and those rows' H and Y are the oracle's."""
+    case = Case(wl.get("decode", d=512, I=256))
+    w = case.w
+    _gpu_result(case)
+    idx, _ = mz.last_routing(case.T, w.K)
+    cnt = mz.expert_load(w.E)[: w.N]
+    hit = np.unique(idx[idx < w.N])
+    for e in hit:
+        tok, _, _, n = mz.last_expert(int(e), w.d, w.I, case.T)
+        want = np.nonzero((idx == e).any(axis=1))[0]
+        assert n == cnt[e] == len(want)
+        assert np.array_equal(np.sort(tok), want)
+    for e in hit[:6]:
+        check_expert_rows(case, int(e))
+
+
 def test_one_grid_fallback_gives_the_same_bits():
-    """A decode-sized batch with the one-grid expert GEMMs switched off (the
-    path taken when their cooperative launch is refused) gives the same
-    output, routing and histogram, bit for bit."""
+    """A decode-sized batch with the one grid switched off (the path taken
+    when its cooperative launch is refused) gives the same output, routing
+    and histogram, bit for bit."""
     case = Case(wl.get("decode", d=1024, I=512))
     assert mz.plan(case.T, case.w.d, case.w.N, case.w.Z, case.w.K,
                    case.w.I)["expert_gemms_one_grid"] == 1
     o1, i1, g1, c1 = _gpu_result(case)
-    mz.test_one_grid(True)
-    try:
-        o2, i2, g2, c2 = _gpu_result(case)
-    finally:
-        mz.test_one_grid(False)
+    o2, i2, g2, c2 = _result_on_path(case, dict(off=True), _gpu_result)
     assert np.array_equal(o1, o2) and np.array_equal(i1, i2) and np.array_equal(c1, c2)
     _full_check(case)
 

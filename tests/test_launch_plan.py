@@ -1,6 +1,7 @@
 """moe_zc_plan: the launch decisions a forward takes, checked on the host
-(no GPU): the router GEMM's tiling, and whether the two expert GEMMs of a
-small batch run as one persistent grid or fall back to two launches."""
+(no GPU): the router GEMM's tiling, and whether a small batch runs the rest
+of the forward (route, dispatch, both expert GEMMs, combine) in one
+persistent grid or falls back to separate launches."""
 import pytest
 
 from mixture_experts_layer_28_b200 import build as mb
@@ -20,7 +21,8 @@ def _lib():
 
 def test_decode_runs_expert_gemms_in_one_grid():
     p = mz.plan(**DECODE, sms=148, resident_blocks=148)
-    assert p["expert_gemms_one_grid"] == 1 and p["kernels"] == 6
+    # the router GEMM and the one grid
+    assert p["expert_gemms_one_grid"] == 1 and p["one_grid_step"] == 1 and p["kernels"] == 2
     # tile bound: ceil(64*12/256) + 512 = 515 token tiles; 16 gate/up and 24
     # down weight blocks each -> far more tiles than SMs
     assert p["expert_grid"] == 148
@@ -32,7 +34,7 @@ def test_decode_runs_expert_gemms_in_one_grid():
 def test_one_grid_falls_back_when_not_resident():
     """Fewer resident blocks than the grid needs: two launches instead."""
     p = mz.plan(**DECODE, sms=148, resident_blocks=147)
-    assert p["expert_gemms_one_grid"] == 0 and p["kernels"] == 7
+    assert p["expert_gemms_one_grid"] == 0 and p["one_grid_step"] == 0 and p["kernels"] == 7
     assert p["expert_grid"] == 148       # the gate/up launch
     p = mz.plan(**DECODE, sms=148, resident_blocks=0)   # kernel cannot be resident at all
     assert p["expert_gemms_one_grid"] == 0
@@ -42,7 +44,7 @@ def test_one_grid_only_for_small_batches():
     assert mz.plan(**dict(DECODE, T=65))["expert_gemms_one_grid"] == 0
     assert mz.plan(**dict(DECODE, T=1))["expert_gemms_one_grid"] == 1
     p = mz.plan(**PREFILL)
-    assert p["expert_gemms_one_grid"] == 0 and p["kernels"] == 7
+    assert p["expert_gemms_one_grid"] == 0 and p["one_grid_step"] == 0 and p["kernels"] == 7
     # 16384 tokens, E = 768 in 3 paired blocks: 176-token tiles fill two whole
     # waves (282 tiles) where 256-token tiles would leave the second a third full
     assert p["router_token_tile"] == 176 and p["router_k_slices"] == 1
@@ -52,10 +54,16 @@ def test_one_grid_only_for_small_batches():
 def test_one_grid_test_hook():
     mz.test_one_grid(True)
     try:
-        assert mz.plan(**DECODE)["expert_gemms_one_grid"] == 0
+        p = mz.plan(**DECODE)
+        assert p["expert_gemms_one_grid"] == 0 and p["kernels"] == 7
+        # the expert GEMMs in one grid, route, dispatch and combine apart
+        mz.test_one_grid(step=False)
+        p = mz.plan(**DECODE)
+        assert p["expert_gemms_one_grid"] == 1 and p["one_grid_step"] == 0 and p["kernels"] == 6
     finally:
         mz.test_one_grid(False)
-    assert mz.plan(**DECODE)["expert_gemms_one_grid"] == 1
+    p = mz.plan(**DECODE)
+    assert p["expert_gemms_one_grid"] == 1 and p["one_grid_step"] == 1 and p["kernels"] == 2
 
 
 def test_kernel_counts_of_special_batches():
