@@ -427,7 +427,9 @@ int moe_zc_route_noalloc(const void* x, const void* W_r, const float* b,
  * Test hook for the error paths: make the next n workspace allocations fail
  * (MOE_ZC_ERR_OOM), and/or make every bounded device wait of the next forward
  * give up after `wait_limit` nanoseconds (0 = the normal 2 s), so that the
- * timeout path runs without a fault.  Not for production use.
+ * timeout path runs without a fault.  (Device waits count SM clock cycles at
+ * 2 per nanosecond: at clocks up to 2 GHz a wait lasts at least its limit.)
+ * Not for production use.
  */
 void moe_zc_test_inject(int32_t fail_allocs, int64_t wait_limit);
 

@@ -42,13 +42,15 @@
 // Batches of at most 64 tokens (decode) stream weights: there the gate/up and
 // down tiles run in one persistent grid (MODE_FUSED, see gemm_kernel), so the
 // SMs that the last, part-filled round of gate/up tiles leaves idle stream
-// down weights of the experts whose H rows are already complete.
-// Prefill-sized gate/up and down launches take their tiles in order from a
-// global counter (the producer takes each and hands it to the MMA issuer and
-// the epilogue through a small shared-memory queue), so the tiles running
-// at any moment are neighbours in tile order -- those that share a weight
-// block or a token tile overlap in time and re-read it from L2 -- and the
-// last round is shared out evenly.
+// down weights of the experts whose H rows are already complete; the same
+// grid also routes, dispatches and combines (the decode step's phases,
+// step.cuh).
+// That grid and the prefill-sized gate/up and down launches take their tiles
+// in order from a global counter (the producer takes each and hands it to
+// the MMA issuer and the epilogue through a small shared-memory queue), so
+// the tiles running at any moment are neighbours in tile order -- those that
+// share a weight block or a token tile overlap in time and re-read it from
+// L2 -- and SMs that stream faster take more tiles.
 // Every wait is time-bounded (ptx.cuh); on running out the CTA drains its
 // in-flight copies and MMAs, frees TMEM and returns with the error flag set.
 #include "epilogue.cuh"
@@ -76,6 +78,7 @@ struct Tile {
   int ntt;      // token tiles of the group
   bool has_a1;  // second A block present
   int a0_row, a1_row;
+  int r0;       // router / down: A block 0's first row inside the group
   int ttile;    // expert GEMMs: the tile's index among all token tiles (FP8 scale atoms)
 };
 
@@ -175,11 +178,13 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   tl.nmma = (tl.ntok + 15) & ~15;
   tl.brow0 += tl.tok0;
   if (MODE == MODE_GATEUP) {
-    tl.a0_row = tl.g * p.a_rows + tl.m * GEMM_BM;   // W_gate rows
+    tl.r0 = tl.m * GEMM_BM;
+    tl.a0_row = tl.g * p.a_rows + tl.r0;             // W_gate rows
     tl.a1_row = tl.a0_row;                           // W_up rows
     tl.has_a1 = true;
   } else {
     const int r = tl.m * (p.single_a ? 1 : 2) * GEMM_BM;
+    tl.r0 = r;
     tl.a0_row = tl.g * p.a_rows + r;
     tl.a1_row = tl.a0_row + GEMM_BM;
     tl.has_a1 = !p.single_a && (r + GEMM_BM) < p.a_rows;
@@ -218,6 +223,16 @@ __device__ __forceinline__ bool tile_at(const GemmParams& p, int it, int n0, int
     t = L * F + (c >= r ? k - L : k) * G + c;
   }
   return t < n1;
+}
+
+// Tiles taken in order from p.tile_counter: the u-th is tile u of a
+// one-phase mode; MODE_FUSED hands out its n0 gate/up tiles, then its down
+// tiles in group order.  Gate/up tiles wait on nothing, and all of them are
+// handed out before any down tile, so every down tile's wait ends.
+template <int MODE>
+__device__ __forceinline__ void dyn_tile(int u, int n0, int& tph, int& t) {
+  tph = MODE == MODE_FUSED && u >= n0 ? 1 : 0;
+  t = tph ? u - n0 : u;
 }
 
 // Tile t of the given phase (see tile_at).
@@ -360,10 +375,12 @@ __device__ __forceinline__ void epi_router_f32(uint32_t tacc, uint8_t* stg, int 
 // round of gate/up tiles already stream down weights.  A down tile of group g
 // reads H rows that other CTAs write: its producer waits (bounded) until all
 // GEMM_EPI_WARPS * mblocks * ntt epilogue warps of g's gate/up tiles have
-// counted themselves in p.done[g].  No wait can close a cycle: every CTA
-// holds all its gate/up tiles before its down tiles, gate/up tiles wait on
-// nothing outside their CTA, and the grid (one CTA per SM, at most one per
-// SM of the device) is resident as a whole.
+// counted themselves in p.done[g].  No wait can close a cycle: gate/up tiles
+// wait on nothing outside their CTA, a CTA has issued all loads of its
+// earlier tiles before it waits for a down tile's group, every gate/up tile
+// is handed out before any down tile (from the counter, or in the fixed
+// shares of tile_at), and the grid (one CTA per SM, at most one per SM of
+// the device) is resident as a whole.
 template <int MODE, int NST, int SB, bool FP8>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
@@ -387,13 +404,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   __shared__ __align__(8) uint64_t tq_full[TILE_Q];
   __shared__ __align__(8) uint64_t tq_empty[TILE_Q];
   __shared__ volatile int bar_ok_sh;   // grid barriers of the decode step
-  const bool dyn =
-      (MODE == MODE_GATEUP || MODE == MODE_DOWN) && p.tile_counter != nullptr && !p.pair_tiles;
+  const bool dyn = (MODE == MODE_GATEUP || MODE == MODE_DOWN || MODE == MODE_FUSED) &&
+                   p.tile_counter != nullptr && !p.pair_tiles;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned (128-byte swizzle atoms); an offset from smem_raw, so
+  // that the compiler keeps every access through it in the shared state space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -459,6 +477,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   const uint32_t tmem = tmem_base_sh;
   const int ntiles = total_tiles<MODE == MODE_FUSED ? MODE_GATEUP : MODE, MODE == MODE_FUSED>(p);
   const int ntiles2 = MODE == MODE_FUSED ? total_tiles<MODE_DOWN, true>(p2) : 0;
+  const int ndyn = ntiles + ntiles2;   // tiles the counter hands out
   // gate/up tiles always hold two blocks; router and down tiles hold one
   // when p.single_a is set (1 buffer of 512 columns, or 2 of 256)
   // (MODE_FUSED: both phases hold two blocks)
@@ -497,12 +516,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
           abort_sh = 1;
           break;
         }
-        t = atomicAdd(p.tile_counter, 1);
-        if (t >= ntiles) t = -1;
-        tph = 0;
-        tile_q[qs] = t;
+        const int u = atomicAdd(p.tile_counter, 1);
+        tile_q[qs] = u < ndyn ? u : -1;
         mbar_arrive(&tq_full[qs]);
-        if (t < 0) break;
+        if (u >= ndyn) break;
+        dyn_tile<MODE>(u, ntiles, tph, t);
       } else if (!tile_at<MODE>(p, it, ntiles, ntiles2, tph, t)) {
         break;
       }
@@ -617,10 +635,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
           abort_sh = 1;
           break;
         }
-        t = tile_q[qs];
-        tph = 0;
+        const int u = tile_q[qs];
         mbar_arrive(&tq_empty[qs]);
-        if (t < 0) break;
+        if (u < 0) break;
+        dyn_tile<MODE>(u, ntiles, tph, t);
       } else if (!tile_at<MODE>(p, local, ntiles, ntiles2, tph, t)) {
         break;
       }
@@ -729,11 +747,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
           abort_sh = 1;
           break;
         }
-        t = tile_q[qs];
-        tph = 0;
+        const int u = tile_q[qs];
         __syncwarp();
         if (lane == 0) mbar_arrive(&tq_empty[qs]);
-        if (t < 0) break;
+        if (u < 0) break;
+        dyn_tile<MODE>(u, ntiles, tph, t);
       } else if (!tile_at<MODE>(p, local, ntiles, ntiles2, tph, t)) {
         break;
       }
@@ -746,8 +764,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
       tc_fence_after();
       const uint32_t tacc = tq + buf * 256;
       const bool down_ph = MODE == MODE_FUSED && tph == 1;
-      // router / down (MODE_FUSED's down tiles hold two blocks)
-      const int row_blk = tl.m * ((MODE == MODE_FUSED || !p.single_a) ? 2 : 1) * GEMM_BM + q * 32;
+      // router / down: this warp's first weight row of A block 0
+      const int row_blk = tl.r0 + q * 32;
       if (MODE == MODE_ROUTER) {
         epi_router_f32(tacc, stg, lane, group, tl, p, row_blk);
         tc_fence_before();
@@ -808,9 +826,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     tmem_dealloc(tmem, 512);
   }
   if (MODE == MODE_FUSED && sp.on) {
-    // every Y row is stored once all blocks are here
-    step_ok = grid_barrier(sp.gbar, ++nbar * static_cast<int>(gridDim.x), p.wait_ns, p.err,
-                           &bar_ok_sh, step_ok && !abort_sh);
+    // every Y row is stored once all blocks are here (the combine reads
+    // them with plain loads: no proxy fence)
+    step_ok = grid_barrier<false>(sp.gbar, ++nbar * static_cast<int>(gridDim.x), p.wait_ns,
+                                  p.err, &bar_ok_sh, step_ok && !abort_sh);
     if (step_ok) step_combine<GEMM_THREADS>(sp, ws);
   }
 }

@@ -613,6 +613,10 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       pf.b_box_full = 0;
       pf.done = fill + N + 1;
       pf.down_lead = (d + I / 2) / I;
+      // tiles taken in order from a counter (cleared by the router GEMM or
+      // the given-routing memset), so that SMs that stream faster take more
+      // (measured: -2 us at decode, bf16 and FP8, against fixed shares)
+      pf.tile_counter = fill + 2 * N + 2;
       auto one_grid_launch = [&](const StepParams& sp) {
         return f8 ? launch_gemm_fused_fp8(mWg, mWu, mXp, mWd, mH, pf, pd,
                                           static_cast<int>(plan.fused_grid), st, sp)

@@ -61,24 +61,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
+// The time bound of the device waits counts this SM's own clock (clock64),
+// not the global nanosecond timer: reads of that timer were measured to take
+// microseconds when the SMs of a grid read it together, as waiting CTAs do.
+// A limit of L ns is taken as 2 L cycles, so that at SM clocks up to 2 GHz
+// (B200 runs at most 1965 MHz) a wait lasts at least L ns.
+constexpr long long kWaitCyclesPerNs = 2;
+__device__ __forceinline__ long long wait_cycles(long long limit_ns) {
+  return limit_ns > (1LL << 61) ? (1LL << 62) : limit_ns * kWaitCyclesPerNs;
 }
 
 // Wait until the phase of `bar` with the given parity has completed, for at
-// most `limit_ns` nanoseconds.  On running out, record DEV_TIMEOUT in *err
-// (unless an error is already there) and return false.
+// most `limit_ns` nanoseconds (as above).  On running out, record DEV_TIMEOUT
+// in *err (unless an error is already there) and return false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit_ns,
                                           int* err) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
+  const long long lim = wait_cycles(limit_ns);
   while (true) {
     for (int i = 0; i < 16; ++i) {
       if (mbar_try_wait(bar, parity)) return true;
     }
-    if (static_cast<long long>(globaltimer_ns() - t0) > limit_ns) {
+    if (clock64() - t0 > lim) {
       atomicCAS(err, DEV_OK, DEV_TIMEOUT);
       return false;
     }
@@ -307,9 +312,10 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(const void* p) {
 __device__ __forceinline__ void pace_until_shared(const void* p, uint32_t target,
                                                   long long limit_ns) {
   if (ld_cluster_u32(p) >= target) return;
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
+  const long long lim = wait_cycles(limit_ns);
   while (ld_cluster_u32(p) < target) {
-    if (static_cast<long long>(globaltimer_ns() - t0) > limit_ns) return;
+    if (clock64() - t0 > lim) return;
   }
 }
 
@@ -330,11 +336,12 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 __device__ __forceinline__ bool wait_count_geq(const int* p, int target, long long limit_ns,
                                                int* err) {
   if (ld_acquire_gpu(p) >= target) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
+  const long long lim = wait_cycles(limit_ns);
   while (true) {
     __nanosleep(128);
     if (ld_acquire_gpu(p) >= target) return true;
-    if (static_cast<long long>(globaltimer_ns() - t0) > limit_ns) {
+    if (clock64() - t0 > lim) {
       atomicCAS(err, DEV_OK, DEV_TIMEOUT);
       return false;
     }

@@ -323,8 +323,8 @@ __device__ __forceinline__ uint32_t quantize32(const uint4 (&v)[4], uint32_t (&c
 // CTA adds one to *ctr once its threads are here and waits, for at most
 // limit_ns, until *ctr reaches `target` (gridDim.x times the number of
 // barriers passed so far; the counter is zero at launch).  Writes before the
-// barrier (also those that bulk-tensor copies read afterwards: the proxy
-// fences) are visible after it.
+// barrier (also, with PROXY, those that bulk-tensor copies read afterwards:
+// the proxy fences) are visible after it.
 //
 // A CTA whose wait runs out records DEV_TIMEOUT in *err, and -- as does a CTA
 // that arrives with arrive_ok false (its own work failed) -- adds
@@ -333,9 +333,10 @@ __device__ __forceinline__ uint32_t quantize32(const uint4 (&v)[4], uint32_t (&c
 // barrier may read.  Returns true when the work after the barrier may run.
 constexpr int STEP_POISON = 1 << 16;
 
+template <bool PROXY = true>
 __device__ __forceinline__ bool grid_barrier(int* ctr, int target, long long limit_ns, int* err,
                                              volatile int* ok_sh, bool arrive_ok) {
-  fence_proxy_async_global();
+  if (PROXY) fence_proxy_async_global();
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -348,7 +349,7 @@ __device__ __forceinline__ bool grid_barrier(int* ctr, int target, long long lim
       atomicAdd(ctr, STEP_POISON);
     }
     *ok_sh = (ok && arrive_ok) ? 1 : 0;
-    fence_proxy_async_global();
+    if (PROXY) fence_proxy_async_global();
   }
   __syncthreads();
   return *ok_sh != 0;
@@ -459,27 +460,34 @@ __device__ __forceinline__ void step_route(const StepParams& sp, uint8_t* ws) {
     }
     __syncthreads();
     if (warp == 0) {
-      // lane w follows warp w's list
+      // merge: lane w follows warp w's list; lane k keeps pick k, and the
+      // picks are stored, and counted, by all lanes at once afterwards
       int pos = 0;
       uint32_t hk = lane < W ? ck[lane * MK] : 0u;
       int hj = lane < W ? cj[lane * MK] : INT_MAX;
       float zs = 0.f;
+      int my_j = -1;
+      float my_p = 0.f;
       for (int k = 0; k < K; ++k) {
         const uint32_t mk = __reduce_max_sync(0xffffffffu, hk);
         const int jw = static_cast<int>(
             __reduce_min_sync(0xffffffffu, hk == mk ? static_cast<uint32_t>(hj) : 0xffffffffu));
         const float pw = p_s[jw];
         if (jw >= N) zs += pw;
-        if (lane == 0) {
-          sp.idx[static_cast<int64_t>(t) * K + k] = jw;
-          sp.gate[static_cast<int64_t>(t) * K + k] = pw;
-          atomicAdd(sp.cnt + jw, 1);
+        if (lane == k) {
+          my_j = jw;
+          my_p = pw;
         }
         if (hj == jw) {
           ++pos;
           hk = pos < K ? ck[lane * MK + pos] : 0u;
           hj = pos < K ? cj[lane * MK + pos] : INT_MAX;
         }
+      }
+      if (lane < K) {
+        sp.idx[static_cast<int64_t>(t) * K + lane] = my_j;
+        sp.gate[static_cast<int64_t>(t) * K + lane] = my_p;
+        atomicAdd(sp.cnt + my_j, 1);
       }
       if (lane == 0) sp.zsum[t] = zs;
     }
