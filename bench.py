@@ -79,13 +79,15 @@ GEMM_SOURCES = ["gemm_tcgen05.cu", "ptx.cuh", "epilogue.cuh", "kernels.cuh", "st
 NCU_TRAFFIC_RATIO = {
     # workload (+ "_fp8" for the FP8 forward): (dominant kernel,
     # DRAM bytes / algorithmic bytes, GEMM sources sha16, the captured case)
-    "prefill": ("gateup_gemm", 3.5935e9 / 2.5460e9, "d892549a292a33dd",
+    "prefill": ("gateup_gemm", 3.4938e9 / 2.5460e9, "87489f0e4c4a3067",
                 "T=8192, N=32, Z=16 prefill-shaped layer, ncu DRAM counters of two launches"),
-    "prefill_fp8": ("gateup_gemm", 1.4650e9 / 1.4260e9, "d892549a292a33dd",
+    "prefill_fp8": ("gateup_gemm", 1.4643e9 / 1.4260e9, "87489f0e4c4a3067",
                     "T=8192, N=32, Z=16 prefill-shaped layer, ncu DRAM counters of two launches"),
-    "decode": ("gateup_down_gemm (one kernel)", 1.4530e9 / 1.4525e9, "d892549a292a33dd",
+    "decode": ("decode_step (route, dispatch, gate/up + down GEMMs, combine: one kernel)",
+               1.4508e9 / 1.4687e9, "87489f0e4c4a3067",
                "T=64, N=32, Z=16 decode-shaped layer, ncu DRAM counters of two launches"),
-    "decode_fp8": ("gateup_down_gemm (one kernel)", 0.9799e9 / 0.9860e9, "d892549a292a33dd",
+    "decode_fp8": ("decode_step (route, dispatch, gate/up + down GEMMs, combine: one kernel)",
+                   0.9797e9 / 0.9989e9, "87489f0e4c4a3067",
                    "T=64, N=32, Z=16 decode-shaped layer, ncu DRAM counters of two launches"),
 }
 SUSTAINED_REGION_S = 2.0   # timed regions at least this long use the sustained bf16 peak
