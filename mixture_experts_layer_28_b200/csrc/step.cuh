@@ -495,27 +495,58 @@ __device__ __forceinline__ void step_route(const StepParams& sp, uint8_t* ws) {
   }
 }
 
-// assign + permute.  Every block with tokens (and block 0, which stores them
-// for the tiles) derives from the histogram each FFN expert's first row
-// (count rounded up to 16) and first token tiles (of GEMM_BN tokens, and of
-// FP8_BN for FP8 gate/up), as the assign kernel does.  Then for each token of
-// the block: a slot for each FFN pick (an atomicAdd on the expert's fill
-// counter; slot -1 for zero-expert picks) and the token's row copied into
-// its slots -- bf16, or quantised once into FP8 codes and scale atoms.
-// (Which slot of its expert a token gets does not change any result: a
-// token's GEMM columns are independent of the others'.)
+// The first gate/up tile whose weights a block prefetches into L2 while the
+// tokens are dispatched: tile blockIdx.x, which some block takes in the
+// grid's first round (tiles come from the counter in order), its first
+// `stages` contraction steps of both A blocks (maps a0 / a1, rows of
+// `a_rows` per expert, `kelems` contraction elements per step).
+struct TilePrefetch {
+  const CUtensorMap* a0;
+  const CUtensorMap* a1;
+  int mblocks, a_rows, kelems, stages;
+};
+
+// assign + permute.  Every block derives from the histogram each FFN
+// expert's first row (count rounded up to 16) and first token tiles (of
+// GEMM_BN tokens, and of FP8_BN for FP8 gate/up), as the assign kernel does
+// (block 0 also stores them for the tiles), and prefetches the weights of
+// its first-round tile (pf).  Then for each token of the block: a slot for
+// each FFN pick (an atomicAdd on the expert's fill counter; slot -1 for
+// zero-expert picks) and the token's row copied into its slots -- bf16, or
+// quantised once into FP8 codes and scale atoms.  (Which slot of its expert
+// a token gets does not change any result: a token's GEMM columns are
+// independent of the others'.)
 template <int NT, bool FP8>
-__device__ __forceinline__ void step_assign_permute(const StepParams& sp, uint8_t* ws) {
-  if (static_cast<int>(blockIdx.x) >= sp.T && blockIdx.x != 0) return;   // (uniform)
+__device__ __forceinline__ void step_assign_permute(const StepParams& sp, uint8_t* ws,
+                                                    const TilePrefetch& pf) {
   const int N = sp.N, K = sp.K, d = sp.d;
   int* off_s = reinterpret_cast<int*>(ws);   // [N] first row
   int* cnt_s = off_s + N;                    // [N]
-  int* ttp8_s = cnt_s + N;                   // [N] first FP8 token tile
-  int* scan_s = ttp8_s + N;                  // [32]
+  int* gtp_s = cnt_s + N;                    // [N] first gate/up token tile (FP8: of FP8_BN)
+  int* scan_s = gtp_s + N;                   // [32]
   int* sl_s = scan_s + 32;                   // [32] slots of the token's FFN picks, k order
   int* tile_s = sl_s + 32;                   // [32] FP8: the slot's token tile
   int* pos_s = tile_s + 32;                  // [32] FP8: its place in the tile
   int* n_s = pos_s + 32;
+  // The block's first token: its picks (warp 0, lane k) and its row (bf16:
+  // chunks tid, tid + NT; FP8: block of 32 tid) are loaded before the scans,
+  // so that their latency overlaps them; later tokens load in turn.
+  const int lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x;
+  const bool first = t0 < sp.T;
+  const int g0 = first && threadIdx.x < 32 && lane < K
+                     ? sp.idx[static_cast<int64_t>(t0) * K + lane] : -1;
+  constexpr int XR = 2;
+  uint4 xr[FP8 ? 4 : XR];
+  {
+    const uint4* src0 = reinterpret_cast<const uint4*>(sp.x) + static_cast<int64_t>(t0) * (d / 8);
+#pragma unroll
+    for (int i = 0; i < (FP8 ? 4 : XR); ++i) {
+      const int c = FP8 ? static_cast<int>(threadIdx.x) * 4 + i : static_cast<int>(threadIdx.x) + i * NT;
+      const bool in = first && (FP8 ? static_cast<int>(threadIdx.x) < d / 32 : c < d / 8);
+      xr[i] = in ? src0[c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
   int carry_r = 0, carry_t = 0, carry_t8 = 0;
   for (int base = 0; base < N; base += NT) {
     const int g = base + static_cast<int>(threadIdx.x);
@@ -527,7 +558,7 @@ __device__ __forceinline__ void step_assign_permute(const StepParams& sp, uint8_
     if (g < N) {
       off_s[g] = carry_r + off;
       cnt_s[g] = c;
-      ttp8_s[g] = carry_t8 + ttp8;
+      gtp_s[g] = FP8 ? carry_t8 + ttp8 : carry_t + ttp;
       if (blockIdx.x == 0) {
         sp.grp_off[g] = carry_r + off;
         sp.grp_ttp[g] = carry_t + ttp;
@@ -544,10 +575,34 @@ __device__ __forceinline__ void step_assign_permute(const StepParams& sp, uint8_
     if (FP8) sp.grp_ttp8[N] = carry_t8;
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    // gate/up tile u = blockIdx.x, decoded as the tiles decode it: expert
+    // g (the last whose first tile is at or below u's token tile), then the
+    // weight block
+    const int gtotal = FP8 ? carry_t8 : carry_t;
+    const int u = blockIdx.x;
+    if (u < gtotal * pf.mblocks) {
+      const int tt = u / pf.mblocks;
+      int lo = 0, hi = N - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (gtp_s[mid] <= tt) lo = mid; else hi = mid - 1;
+      }
+      const int ttp0 = gtp_s[lo];
+      const int ntt = (lo + 1 < N ? gtp_s[lo + 1] : gtotal) - ttp0;
+      const int v = u - ttp0 * pf.mblocks;
+      const int m = ntt == 2 ? v >> 1 : v % pf.mblocks;
+      const int row = lo * pf.a_rows + m * GEMM_BM;
+      for (int k = 0; k < pf.stages; ++k) {
+        tma_prefetch_l2_2d(pf.a0, k * pf.kelems, row);
+        tma_prefetch_l2_2d(pf.a1, k * pf.kelems, row);
+      }
+    }
+  }
   for (int t = blockIdx.x; t < sp.T; t += gridDim.x) {
+    const bool pre = first && t == t0;
     if (threadIdx.x < 32) {
-      const int g = lane < K ? sp.idx[static_cast<int64_t>(t) * K + lane] : -1;
+      const int g = pre ? g0 : (lane < K ? sp.idx[static_cast<int64_t>(t) * K + lane] : -1);
       const bool ffn = g >= 0 && g < N;
       int s = -1;
       if (ffn) s = off_s[g] + atomicAdd(sp.fill + g, 1);
@@ -561,7 +616,7 @@ __device__ __forceinline__ void step_assign_permute(const StepParams& sp, uint8_
           const int tsz = even_tile_size(count, (count + FP8_BN - 1) / FP8_BN, FP8_BN);
           const int u = s - off_s[g];
           const int j = u / tsz;
-          tile_s[k] = ttp8_s[g] + j;
+          tile_s[k] = gtp_s[g] + j;
           pos_s[k] = u - j * tsz;
         }
       }
@@ -574,9 +629,10 @@ __device__ __forceinline__ void step_assign_permute(const StepParams& sp, uint8_
       const uint4* src = reinterpret_cast<const uint4*>(sp.x) + static_cast<int64_t>(t) * (d / 8);
       uint4* Xp8 = reinterpret_cast<uint4*>(sp.Xp8);
       for (int b = threadIdx.x; b < nb; b += NT) {
+        const bool held = pre && b == static_cast<int>(threadIdx.x);
         uint4 v[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) v[q] = src[b * 4 + q];
+        for (int q = 0; q < 4; ++q) v[q] = held ? xr[q] : src[b * 4 + q];
         uint32_t c[8];
         const uint32_t sc = quantize32(v, c);
         const uint4 c0 = make_uint4(c[0], c[1], c[2], c[3]);
@@ -593,7 +649,15 @@ __device__ __forceinline__ void step_assign_permute(const StepParams& sp, uint8_
       const int d8 = d / 8;
       const uint4* src = reinterpret_cast<const uint4*>(sp.x) + static_cast<int64_t>(t) * d8;
       uint4* Xp = reinterpret_cast<uint4*>(sp.Xp);
-      for (int c = threadIdx.x; c < d8; c += NT) {
+#pragma unroll
+      for (int i = 0; i < XR; ++i) {
+        const int c = static_cast<int>(threadIdx.x) + i * NT;
+        if (c < d8) {
+          const uint4 v = pre ? xr[i] : src[c];
+          for (int k = 0; k < n; ++k) Xp[static_cast<int64_t>(sl_s[k]) * d8 + c] = v;
+        }
+      }
+      for (int c = threadIdx.x + XR * NT; c < d8; c += NT) {
         const uint4 v = src[c];
         for (int k = 0; k < n; ++k) Xp[static_cast<int64_t>(sl_s[k]) * d8 + c] = v;
       }
