@@ -192,37 +192,15 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   return tl;
 }
 
-// Tile `it` of this CTA's list: phase 0 tiles are the mode's own (for
-// MODE_FUSED the gate/up tiles), phase 1 the down tiles of MODE_FUSED.
-// One-phase modes and the gate/up phase take tiles blockIdx.x + i * G of the
-// n0.  The n1 down tiles then go out so that the CTAs finish together: the
-// r = n0 % G CTAs that hold one gate/up tile more join p.down_lead down tiles
-// later.  With F = G - r, down tile j belongs to
-//   j <  L * F:  CTA r + j % F (its (j / F)-th down tile),
-//   j >= L * F:  CTA (j - L * F) % G,
-// so that every CTA meets its down tiles, and the groups, in increasing
-// order: the earliest finished gate/up results are read first.
+// Tile `it` of this CTA's list when tiles are not taken from a counter (the
+// router, and the one-phase GEMMs of batches below the counter's size):
+// tiles blockIdx.x + i * G of the n0.  (MODE_FUSED always takes its tiles
+// from the counter.)
 template <int MODE>
-__device__ __forceinline__ bool tile_at(const GemmParams& p, int it, int n0, int n1, int& tph,
-                                        int& t) {
-  const int c = blockIdx.x;
-  const int G = gridDim.x;
-  if (MODE != MODE_FUSED || it < (c < n0 ? (n0 - 1 - c) / G + 1 : 0)) {
-    tph = 0;
-    t = c + it * G;
-    return t < n0;
-  }
-  const int k = it - (c < n0 ? (n0 - 1 - c) / G + 1 : 0);
-  const int r = n0 % G;
-  const int F = G - r;
-  const int L = p.down_lead;
-  tph = 1;
-  if (c >= r && k < L) {
-    t = k * F + (c - r);
-  } else {
-    t = L * F + (c >= r ? k - L : k) * G + c;
-  }
-  return t < n1;
+__device__ __forceinline__ bool tile_at(int it, int n0, int& tph, int& t) {
+  tph = 0;
+  t = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
+  return t < n0;
 }
 
 // Tiles taken in order from p.tile_counter: the u-th is tile u of a
@@ -377,10 +355,9 @@ __device__ __forceinline__ void epi_router_f32(uint32_t tacc, uint8_t* stg, int 
 // GEMM_EPI_WARPS * mblocks * ntt epilogue warps of g's gate/up tiles have
 // counted themselves in p.done[g].  No wait can close a cycle: gate/up tiles
 // wait on nothing outside their CTA, a CTA has issued all loads of its
-// earlier tiles before it waits for a down tile's group, every gate/up tile
-// is handed out before any down tile (from the counter, or in the fixed
-// shares of tile_at), and the grid (one CTA per SM, at most one per SM of
-// the device) is resident as a whole.
+// earlier tiles before it waits for a down tile's group, the counter hands
+// out every gate/up tile before any down tile, and the grid (one CTA per SM,
+// at most one per SM of the device) is resident as a whole.
 template <int MODE, int NST, int SB, bool FP8>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
@@ -404,8 +381,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
   __shared__ __align__(8) uint64_t tq_full[TILE_Q];
   __shared__ __align__(8) uint64_t tq_empty[TILE_Q];
   __shared__ volatile int bar_ok_sh;   // grid barriers of the decode step
-  const bool dyn = (MODE == MODE_GATEUP || MODE == MODE_DOWN || MODE == MODE_FUSED) &&
-                   p.tile_counter != nullptr && !p.pair_tiles;
+  const bool dyn = MODE == MODE_FUSED ||
+                   ((MODE == MODE_GATEUP || MODE == MODE_DOWN) && p.tile_counter != nullptr &&
+                    !p.pair_tiles);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -526,7 +504,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         mbar_arrive(&tq_full[qs]);
         if (u >= ndyn) break;
         dyn_tile<MODE>(u, ntiles, tph, t);
-      } else if (!tile_at<MODE>(p, it, ntiles, ntiles2, tph, t)) {
+      } else if (!tile_at<MODE>(it, ntiles, tph, t)) {
         break;
       }
       const Tile tl = phase_tile<MODE>(p, p2, tph, t);
@@ -644,7 +622,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         mbar_arrive(&tq_empty[qs]);
         if (u < 0) break;
         dyn_tile<MODE>(u, ntiles, tph, t);
-      } else if (!tile_at<MODE>(p, local, ntiles, ntiles2, tph, t)) {
+      } else if (!tile_at<MODE>(local, ntiles, tph, t)) {
         break;
       }
       const Tile tl = phase_tile<MODE>(p, p2, tph, t);
@@ -757,7 +735,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         if (lane == 0) mbar_arrive(&tq_empty[qs]);
         if (u < 0) break;
         dyn_tile<MODE>(u, ntiles, tph, t);
-      } else if (!tile_at<MODE>(p, local, ntiles, ntiles2, tph, t)) {
+      } else if (!tile_at<MODE>(local, ntiles, tph, t)) {
         break;
       }
       const Tile tl = phase_tile<MODE>(p, p2, tph, t);
@@ -923,7 +901,7 @@ cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, cons
                               const StepParams& step) {
   if (grid <= 0) return cudaSuccess;
   if (grid > device_sms() || !pg.small_b || pg.pair_tiles || pg.b_box_full || pd.single_a ||
-      pg.done == nullptr || !step_args_ok(step, pg, false))
+      pg.done == nullptr || pg.tile_counter == nullptr || !step_args_ok(step, pg, false))
     return cudaErrorInvalidValue;
   // (a refused cooperative launch leaves nothing queued: launch_mode's error
   // is returned as is, without cudaGetLastError, for the caller to clear)
@@ -968,8 +946,8 @@ cudaError_t launch_gemm_fused_fp8(const CUtensorMap& wg, const CUtensorMap& wu,
                                   const StepParams& step) {
   if (grid <= 0) return cudaSuccess;
   if (grid > device_sms() || !pg.small_b || pg.pair_tiles || pg.b_box_full || pd.single_a ||
-      pg.done == nullptr || pg.tok_tile != FP8_BN || !pg.sfa0 || !pg.sfa1 || !pg.sfb ||
-      pg.sf_kgroups != pg.ksteps || !step_args_ok(step, pg, true))
+      pg.done == nullptr || pg.tile_counter == nullptr || pg.tok_tile != FP8_BN || !pg.sfa0 ||
+      !pg.sfa1 || !pg.sfb || pg.sf_kgroups != pg.ksteps || !step_args_ok(step, pg, true))
     return cudaErrorInvalidValue;
   return launch_mode<MODE_FUSED, FP8_SMALL_STAGES, FP8_SMALL_STAGE_BYTES, true>(
       wg, wu, xp8, xp8, wd, h, pg, pd, grid, stream, step);

@@ -187,10 +187,7 @@ struct GemmParams {
   // MODE_FUSED (set in the gate/up parameters): done[g] counts the epilogue
   // warps that have stored their part of a gate/up tile of group g (zeroed
   // before the launch); a down tile of group g starts once all of them have.
-  // down_lead: down tiles that the CTAs with one gate/up tile fewer take
-  // first (about a gate/up tile's cost in down tiles).
   int* done;
-  int down_lead;
   // FP8 gate/up (block-scaled E4M3, FP8_BK contraction elements per stage):
   // the UE8M0 scale atoms of W_gate and W_up (rows of the weight matrices,
   // sf_atom_offset with kgroups = sf_kgroups) and of the token tiles (sfb:
@@ -253,10 +250,11 @@ cudaError_t launch_gemm(GemmMode mode, const CUtensorMap& a0, const CUtensorMap&
 
 // Gate/up then down in one persistent grid of `grid` CTAs (batches of at most
 // GEMM_SMALL_B tokens): wg, wu, xp as for the gate/up launch (parameters pg,
-// with pg.done and pg.down_lead set), wd and h as for the down launch
-// (parameters pd).  A cooperative launch: an error return (the grid cannot be
-// resident at once) launches nothing, and the caller runs the two GEMMs as
-// separate launches instead.
+// with pg.done and pg.tile_counter set: the grid takes its tiles from the
+// counter, zero at launch), wd and h as for the down launch (parameters pd).
+// A cooperative launch: an error return (the grid cannot be resident at
+// once) launches nothing, and the caller runs the two GEMMs as separate
+// launches instead.
 cudaError_t launch_gemm_fused(const CUtensorMap& wg, const CUtensorMap& wu, const CUtensorMap& xp,
                               const CUtensorMap& wd, const CUtensorMap& h, const GemmParams& pg,
                               const GemmParams& pd, int grid, cudaStream_t stream,

@@ -608,11 +608,10 @@ int forward_impl(const void* x, const void* W_r, const float* b, const void* W_g
       // At most 64 tokens: both expert GEMMs in one persistent grid, the
       // down tiles of an expert starting as soon as its H rows are stored
       // (the SMs that the last round of gate/up tiles leaves idle stream down
-      // weights meanwhile); a gate/up tile costs about d / I down tiles.
+      // weights meanwhile).
       GemmParams pf = pg;
       pf.b_box_full = 0;
       pf.done = fill + N + 1;
-      pf.down_lead = (d + I / 2) / I;
       // tiles taken in order from a counter (cleared by the router GEMM or
       // the given-routing memset), so that SMs that stream faster take more
       // (measured: -2 us at decode, bf16 and FP8, against fixed shares)
