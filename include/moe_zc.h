@@ -80,13 +80,15 @@ typedef enum moe_zc_status {
  * Batches of 1024 tokens or more leave a copy of their expert-load histogram
  * in pinned host memory (asynchronously); a later forward on the device uses
  * it to choose how the expert GEMMs are launched.  That choice changes speed
- * only: every launch gives the same bits.  Batches of at most 64 tokens run
- * both expert GEMMs in one grid of at most one block per multiprocessor,
- * whose down-projection tiles wait (bounded, like every device wait) for
- * other blocks' gate/up results; that grid is launched as a cooperative
- * launch, so the driver either makes all its blocks resident at once or
- * refuses it, and a refused launch (e.g. too few multiprocessors free to
- * this process) falls back to two launches with the same bits
+ * only: every launch gives the same bits.  A batch of at most 64 tokens is
+ * two kernels: the router GEMM, then one grid of at most one block per
+ * multiprocessor that routes the tokens, assigns their slots and copies
+ * them, runs both expert GEMMs (down-projection tiles wait, bounded like
+ * every device wait, for other blocks' gate/up results) and combines, with
+ * bounded grid-wide barriers between those phases.  That grid is launched as
+ * a cooperative launch, so the driver either makes all its blocks resident
+ * at once or refuses it, and a refused launch (e.g. too few multiprocessors
+ * free to this process) falls back to separate launches with the same bits
  * (moe_zc_plan shows the choice).
  */
 int moe_zc_forward(const void* x, const void* W_r, const float* b,
