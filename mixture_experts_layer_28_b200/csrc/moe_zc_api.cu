@@ -801,14 +801,31 @@ int forward_host_impl(const void* x_host, const void* W_r, const float* b, const
   chunk = 0;
   for (int64_t n : sizes) chunk = n > chunk ? n : chunk;
   const int E = N + Z;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t row_bytes = static_cast<size_t>(d) * 2;
+  if (sizes.size() == 1) {
+    // One chunk (e.g. a decode batch): nothing to overlap, so the copy in,
+    // the forward and the copy out run in order on the caller's stream,
+    // without the pipeline's side streams, events and summed histogram
+    // (decode e2e 56-79 us over the device-resident step before, 43 us with
+    // this path).
+    if ((s = ensure(c, c.xin[0], T * row_bytes)) != MOE_ZC_OK) return s;
+    if ((s = ensure(c, c.yout[0], T * row_bytes)) != MOE_ZC_OK) return s;
+    CK(cudaMemcpyAsync(c.xin[0].p, x_host, T * row_bytes, cudaMemcpyHostToDevice, st));
+    if ((s = forward_impl(c.xin[0].p, W_r, b, W_gate, W_up, W_down, T, d, N, Z, K, I, off,
+                          c.yout[0].p, stream, f8)) != MOE_ZC_OK)
+      return s;
+    CK(cudaMemcpyAsync(out_host, c.yout[0].p, T * row_bytes, cudaMemcpyDeviceToHost, st));
+    CK(cudaEventRecord(c.done, st));
+    c.done_valid = true;
+    return MOE_ZC_OK;
+  }
   if ((s = host_streams(c)) != MOE_ZC_OK) return s;
   if ((s = ensure(c, c.cnt_total, sizeof(int) * E)) != MOE_ZC_OK) return s;
-  const size_t row_bytes = static_cast<size_t>(d) * 2;
   for (int i = 0; i < 2 && T > 0; ++i) {
     if ((s = ensure(c, c.xin[i], chunk * row_bytes)) != MOE_ZC_OK) return s;
     if ((s = ensure(c, c.yout[i], chunk * row_bytes)) != MOE_ZC_OK) return s;
   }
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   CK(cudaMemsetAsync(c.cnt_total.p, 0, sizeof(int) * E, st));
   CK(cudaEventRecord(c.ev_start, st));
   CK(cudaStreamWaitEvent(c.s_in, c.ev_start, 0));
